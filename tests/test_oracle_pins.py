@@ -1,0 +1,362 @@
+"""Pins of the CPU oracle to things other than itself.
+
+Each test ties one oracle step to the pages' formulas by a route that does
+not reuse the oracle's own code: a hand-worked example, exact rational
+arithmetic, brute force over small domains, integer matrix products, closed
+forms and invariants.  Sources: the Falcon-Edge blog (section "Falcon-Edge,
+a series of universal models": activation_norm_quant, _weight_quant,
+BitLinear) and the 2-bit storage remark in the Hacker News comments of
+"BitNet: inference framework for 1-bit LLMs" (GeekNews).
+"""
+
+import itertools
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests.exact import f32_exact, nearest_bf16_bits, nearest_f32
+
+RNG = np.random.default_rng(20260101)
+
+
+def bits_of_bf16(values):
+    return synth.bf16_bits(torch.tensor(values, dtype=torch.bfloat16))
+
+
+# --------------------------------------------------------------------------
+# Hand-worked example (tests/golden/hand_worked_k4.json)
+# --------------------------------------------------------------------------
+
+def check_hand_worked(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "hand_worked_k4.json")))
+    xb = bits_of_bf16([g["x"]])
+    q, s_x, r = oracle.act_quant(xb)
+    assert q.tolist() == [g["q"]]
+    assert s_x[0] == np.float32(g["s_x"])
+    assert int(r[0]) == g["rowsum"]
+    w = np.array(g["w"], dtype=np.float32)
+    mean = oracle.absmean(w)
+    s_w = oracle.weight_scale(mean)
+    assert mean == np.float32(g["mean"])
+    assert s_w == np.float32(g["s_w"])
+    u = oracle.ternarise(w, s_w)
+    assert u.tolist() == g["u"]
+    # K padded to 16 (the packing granule) with zero activations
+    packed = oracle.pack(np.pad(u, ((0, 0), (0, 12))))
+    out = oracle.forward(bits_of_bf16([g["x"] + [0.0] * 12]), packed, np.float32(g["s_w"]))
+    assert out["acc"].tolist() == [g["acc"]]
+    for n in range(2):
+        want = nearest_f32(Fraction(g["y_exact_num"][n], g["y_exact_den"]))
+        assert out["y32"][0, n] == want
+        assert float(oracle.bf16_to_f32(out["y"][0, n])) == g["y_bf16"][n]
+
+
+def test_hand_worked_example(golden_dir):
+    check_hand_worked(golden_dir)
+
+
+def test_pack_layout_fixture(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "pack_layout.json")))
+    u = np.array([g["u"]], dtype=np.int8)
+    assert oracle.pack(u).ravel().tolist() == g["bytes"]
+    assert oracle.unpack(np.array([g["bytes"]], dtype=np.uint8)).tolist() == [g["u"]]
+
+
+# --------------------------------------------------------------------------
+# Step 1: activation quantisation
+# --------------------------------------------------------------------------
+
+def test_act_quant_ties_round_half_even():
+    # a = 127 so s_x = 1 and x*s_x = x exactly
+    xb = bits_of_bf16([[127.0, 2.5, 3.5, -0.5, 0.5, -2.5, 1.5, -63.5]])
+    q, s_x, _ = oracle.act_quant(xb)
+    assert s_x[0] == np.float32(1.0)
+    assert q.tolist() == [[127, 2, 4, 0, 0, -2, 2, -64]]
+
+
+def test_act_quant_zero_row_and_clamp():
+    xb = bits_of_bf16([[0.0] * 16, [1e-7] + [0.0] * 15])
+    q, s_x, r = oracle.act_quant(xb)
+    assert s_x[0] == np.float32(127.0) / np.float32(1e-5)
+    assert s_x[1] == s_x[0]            # |x| below the clamp uses the clamp
+    assert np.all(q[0] == 0) and r[0] == 0
+    # 1e-7 (as bf16) * 12700000 ~ 1.27 -> 1
+    assert q[1, 0] == 1
+
+
+def test_act_quant_exact_against_rationals():
+    """q and s_x from exact rationals with independent rounding."""
+    x = synth.normal_bf16(7, 1, (6, 64))
+    xb = synth.bf16_bits(x)
+    q, s_x, r = oracle.act_quant(xb)
+    xf = x.float().numpy()
+    for m in range(6):
+        a = max(abs(float(v)) for v in xf[m])
+        s = nearest_f32(Fraction(127) / max(Fraction(a), f32_exact(1e-5)))
+        assert s_x[m] == s
+        for k in range(64):
+            t = nearest_f32(Fraction(float(xf[m, k])) * Fraction(float(s)))
+            tf = Fraction(float(t))
+            fl = math.floor(tf)
+            rnd = fl + 1 if (tf - fl > Fraction(1, 2) or (tf - fl == Fraction(1, 2) and fl % 2)) else fl
+            assert int(q[m, k]) == max(-128, min(127, rnd))
+        assert int(r[m]) == int(sum(int(v) for v in q[m]))
+
+
+def test_act_quant_invariants():
+    x = synth.normal_bf16(7, 2, (5, 128), 3.0)
+    xb = synth.bf16_bits(x)
+    q, s_x, _ = oracle.act_quant(xb)
+    # absmax element maps to +-127
+    xf = x.float().numpy()
+    am = np.abs(xf).argmax(axis=1)
+    assert np.all(np.abs(q[np.arange(5), am]) == 127)
+    assert np.all(np.abs(q.astype(int)) <= 127)
+    # sign symmetry
+    qn, sn, _ = oracle.act_quant(synth.bf16_bits(-x))
+    assert np.array_equal(qn, -q) and np.array_equal(sn, s_x)
+    # power-of-two scaling leaves q unchanged and scales s_x by 2**-k
+    for k in (-3, 5):
+        qk, sk, _ = oracle.act_quant(synth.bf16_bits(x * (2.0 ** k)))
+        assert np.array_equal(qk, q)
+        assert np.array_equal(sk, (s_x * np.float32(2.0 ** -k)).astype(np.float32))
+
+
+# --------------------------------------------------------------------------
+# Step 2: absmean scale, ternarisation, packing
+# --------------------------------------------------------------------------
+
+def exact_mean(w):
+    return sum((abs(f32_exact(v)) for v in w.ravel()), Fraction(0)) / w.size
+
+
+@pytest.mark.parametrize("case", ["gauss", "mixed", "denormal", "wide"])
+def test_absmean_exact_vs_fraction(case):
+    if case == "gauss":
+        w = synth.normal_f32(3, 1, (37, 29), 0.02).numpy()
+    elif case == "mixed":
+        w = (RNG.standard_normal(500) * np.exp2(RNG.integers(-40, 40, 500))).astype(np.float32)
+    elif case == "denormal":
+        w = (RNG.standard_normal(300) * 2.0 ** -140).astype(np.float32)
+        w[::7] = np.float32(3e-45)
+    else:
+        w = np.array([3.0e38, 1e-38, 2.0 ** -149, 1.0, -7.5, 1e-3] * 9, dtype=np.float32)
+    assert oracle.absmean(w) == nearest_f32(exact_mean(w))
+
+
+def test_absmean_ties_to_even():
+    one = np.float32(1.0)
+    up1 = np.nextafter(one, np.float32(2))
+    up2 = np.nextafter(up1, np.float32(2))
+    # mean of (1, 1+2^-23) is 1 + 2^-24: a tie, the even neighbour is 1
+    assert oracle.absmean(np.array([one, up1], np.float32)) == one
+    # mean of (1+2^-23, 1+2^-22) is 1 + 1.5*2^-23: a tie, the even neighbour is 1+2^-22
+    assert oracle.absmean(np.array([up1, up2], np.float32)) == up2
+
+
+def test_absmean_order_independent():
+    w = synth.normal_f32(3, 2, (64, 64), 0.02).numpy()
+    m = oracle.absmean(w)
+    perm = RNG.permutation(w.size)
+    assert oracle.absmean(w.ravel()[perm]) == m
+
+
+def test_weight_scale_and_clamp():
+    assert oracle.weight_scale(np.float32(0.2)) == np.float32(5.0)
+    z = np.zeros((4, 16), np.float32)
+    m = oracle.absmean(z)
+    assert m == 0
+    assert oracle.weight_scale(m) == np.float32(1.0) / np.float32(1e-5)
+    assert np.all(oracle.ternarise(z, oracle.weight_scale(m)) == 0)
+
+
+def test_ternarise_ties_and_clamp():
+    w = np.array([0.5, -0.5, 1.5, -1.5, 0.49, 0.51, 7.0, -7.0, 0.0, -0.0], np.float32)
+    assert oracle.ternarise(w, np.float32(1.0)).tolist() == [0, 0, 1, -1, 0, 1, 1, -1, 0, 0]
+
+
+def test_ternarise_power_of_two_invariance():
+    w = synth.normal_f32(3, 3, (32, 64), 0.02).numpy()
+    _, s_w, _ = oracle.pack_weights(w)
+    u = oracle.ternarise(w, s_w)
+    for k in (-4, 6):
+        wk = (w * np.float32(2.0 ** k)).astype(np.float32)
+        _, s_k, _ = oracle.pack_weights(wk)
+        assert s_k == np.float32(s_w * np.float32(2.0 ** -k))
+        assert np.array_equal(oracle.ternarise(wk, s_k), u)
+
+
+def test_zero_fraction_gaussian():
+    """|w| <= mean|w|/2 has probability erf(1/(2 sqrt(pi))) ~ 0.3101 for
+    Gaussian w (mean|w| = sigma sqrt(2/pi))."""
+    w = synth.normal_f32(3, 4, (1000, 1024), 0.02).numpy()
+    packed, s_w, _ = oracle.pack_weights(w)
+    frac0 = float((oracle.ternarise(w, s_w) == 0).mean())
+    assert abs(frac0 - math.erf(1.0 / (2.0 * math.sqrt(math.pi)))) < 2e-3
+
+
+def test_pack_bruteforce_all_bytes():
+    codes = np.array(list(itertools.product([-1, 0, 1], repeat=4)), dtype=np.int8)  # 81 x (i=0..3 at j=0)
+    u = np.zeros((81, 16), np.int8)
+    u[:, 0::4] = codes                      # k = 4i + 0 -> byte 0, bit pair i
+    p = oracle.pack(u)
+    want = ((codes.astype(int) + 1) * np.array([1, 4, 16, 64])).sum(axis=1)
+    assert np.array_equal(p[:, 0], want)
+    assert np.all(p[:, 1:] == 0x55)
+    assert np.array_equal(oracle.unpack(p), u)
+
+
+def test_pack_roundtrip_all_words():
+    """All 3**16 ternary 16-tuples round-trip through pack/unpack (so the
+    packing is injective) and no packed bit pair ever holds the code 3."""
+    total = 3 ** 16
+    step = 1 << 21
+    digits = 3 ** np.arange(16, dtype=np.int64)
+    for s in range(0, total, step):
+        idx = np.arange(s, min(total, s + step), dtype=np.int64)
+        u = ((idx[:, None] // digits[None, :]) % 3 - 1).astype(np.int8)
+        p = oracle.pack(u)
+        assert np.array_equal(oracle.unpack(p), u)
+        words = np.ascontiguousarray(p).view("<u4").ravel()
+        for i in range(4):
+            pairs = ((words >> np.uint32(2 * i)) & np.uint32(0x03030303)).view(np.uint8)
+            assert not np.any(pairs == 3)
+
+
+def test_unpack_rejects_code3():
+    bad = np.zeros((1, 4), np.uint8)
+    bad[0, 2] = 0x0C                          # bit pair 1 of byte 2 holds 3
+    with pytest.raises(ValueError):
+        oracle.unpack(bad)
+
+
+# --------------------------------------------------------------------------
+# Step 3: contraction
+# --------------------------------------------------------------------------
+
+def test_contract_bruteforce_all_ternary_2x3():
+    q = RNG.integers(-128, 128, (5, 3)).astype(np.int8)
+    for t in itertools.product([-1, 0, 1], repeat=6):
+        u = np.array(t, dtype=np.int8).reshape(2, 3)
+        acc = oracle.contract(q, u)
+        for m in range(5):
+            for n in range(2):
+                assert acc[m, n] == sum(int(q[m, k]) * int(u[n, k]) for k in range(3))
+
+
+def test_contract_vs_int64_matmul():
+    q = RNG.integers(-128, 128, (33, 1000)).astype(np.int8)
+    u = RNG.integers(-1, 2, (2100, 1000)).astype(np.int8)
+    want = np.matmul(q.astype(np.int64), u.astype(np.int64).T)
+    assert np.array_equal(oracle.contract(q, u).astype(np.int64), want)
+
+
+def test_contract_extreme_magnitude():
+    K = 28672
+    q = np.full((2, K), 127, np.int8)
+    q[1] = -128
+    u = np.ones((3, K), np.int8)
+    u[1] = -1
+    acc = oracle.contract(q, u)
+    assert acc[0, 0] == 127 * K and acc[1, 1] == 128 * K and acc[0, 2] == 127 * K
+
+
+def test_permutation_and_row_independence():
+    x = synth.normal_bf16(9, 1, (4, 256))
+    w = synth.normal_f32(9, 2, (48, 256), 0.02).numpy()
+    packed, s_w, _ = oracle.pack_weights(w)
+    out = oracle.forward(synth.bf16_bits(x), packed, s_w)
+    perm = RNG.permutation(256)
+    q, _, _ = oracle.act_quant(synth.bf16_bits(x))
+    u = oracle.unpack(packed)
+    assert np.array_equal(oracle.contract(q[:, perm], u[:, perm]), out["acc"])
+    x2 = x.clone()
+    x2[2] = x2[2] * 3 + 1
+    out2 = oracle.forward(synth.bf16_bits(x2), packed, s_w)
+    for key in ("q", "acc", "y32", "y"):
+        assert np.array_equal(np.delete(out2[key], 2, axis=0), np.delete(out[key], 2, axis=0))
+
+
+def test_dequant_invariant_float64_linear():
+    """The integer path equals F.linear on the dequantised operands
+    x ~ q/s_x and w ~ u/s_w, times s_x*s_w, up to float64 rounding."""
+    x = synth.normal_bf16(9, 3, (8, 512))
+    w = synth.normal_f32(9, 4, (64, 512), 0.02).numpy()
+    packed, s_w, _ = oracle.pack_weights(w)
+    out = oracle.forward(synth.bf16_bits(x), packed, s_w)
+    q, s_x, _ = oracle.act_quant(synth.bf16_bits(x))
+    u = oracle.unpack(packed)
+    xd = torch.from_numpy(q.astype(np.float64) / s_x.astype(np.float64)[:, None])
+    wd = torch.from_numpy(u.astype(np.float64) / np.float64(s_w))
+    y = torch.nn.functional.linear(xd, wd).numpy()
+    scale = s_x.astype(np.float64)[:, None] * np.float64(s_w)
+    assert np.allclose(y * scale, out["acc"].astype(np.float64), rtol=0, atol=1e-6 * 127 * 512)
+    # and the float32 epilogue is within float32 rounding of the float64 value
+    rel = np.abs(out["y32"].astype(np.float64) - y) / np.maximum(np.abs(y), 1e-30)
+    assert np.all(rel[np.abs(y) > 1e-6] < 3e-7)
+
+
+# --------------------------------------------------------------------------
+# Step 4: epilogue
+# --------------------------------------------------------------------------
+
+def test_epilogue_exact_rational():
+    acc = RNG.integers(-400000, 400000, (7, 9)).astype(np.int32)
+    s_x = (RNG.random(7) * 100 + 1).astype(np.float32)
+    s_w = np.float32(37.125)
+    bias = synth.bf16_bits(synth.normal_bf16(9, 5, (9,), 0.01))
+    y32, y = oracle.epilogue(acc, s_x, s_w, bias)
+    bf = oracle.bf16_to_f32(bias)
+    for m in range(7):
+        d = nearest_f32(f32_exact(s_x[m]) * f32_exact(s_w))
+        for n in range(9):
+            q = nearest_f32(Fraction(int(acc[m, n])) / Fraction(float(d)))
+            want = nearest_f32(Fraction(float(q)) + Fraction(float(bf[n])))
+            assert y32[m, n] == want
+            assert int(y[m, n]) == nearest_bf16_bits(want)
+
+
+def test_bf16_conversions():
+    v = np.array([1.0, -2.5, 3.0e-39, 65504.0, 1.00390625, 1.005859375], np.float32)
+    b = oracle.f32_to_bf16_rne(v)
+    assert [int(t) for t in b] == [nearest_bf16_bits(t) for t in v]
+    assert np.array_equal(oracle.bf16_to_f32(b), torch.tensor(v).to(torch.bfloat16).float().numpy())
+
+
+# --------------------------------------------------------------------------
+# The pins catch planted mistakes (mutations planted in the oracle, on CPU)
+# --------------------------------------------------------------------------
+
+def test_pins_catch_planted_mistakes(golden_dir, monkeypatch):
+    orig_act, orig_epi, orig_pack = oracle.act_quant, oracle.epilogue, oracle.pack
+
+    def act_floor(xb):                      # floor instead of round
+        q, s, r = orig_act(xb)
+        x = oracle.bf16_to_f32(xb)
+        qf = np.clip(np.floor(x * s[:, None]), -128, 127).astype(np.int8)
+        return qf, s, qf.astype(np.int64).sum(1).astype(np.int32)
+
+    def epi_mul(acc, s_x, s_w, bias_bits=None):  # multiply instead of divide
+        y32 = acc.astype(np.float32) * (np.asarray(s_x, np.float32) * np.float32(s_w))[:, None]
+        return y32, oracle.f32_to_bf16_rne(y32)
+
+    def pack_swapped(u):                     # i and j swapped in the layout
+        N, K = u.shape
+        t = u.reshape(N, K // 16, 4, 4).transpose(0, 1, 3, 2).reshape(N, K)
+        return orig_pack(t)
+
+    for name, bad in (("act_quant", act_floor), ("epilogue", epi_mul), ("pack", pack_swapped)):
+        monkeypatch.setattr(oracle, name, bad)
+        with pytest.raises(AssertionError):
+            check_hand_worked(golden_dir)
+            if name == "pack":
+                test_pack_layout_fixture(golden_dir)
+        monkeypatch.undo()
+    check_hand_worked(golden_dir)
