@@ -1,0 +1,223 @@
+"""Python binding of libbitlinear.so (BitNet b1.58 BitLinear forward, B200).
+
+Argument marshalling only: every function allocates its outputs (and a
+workspace, unless one is passed) with torch on the tensors' device and calls
+the C entry point of the same name on the current CUDA stream.  All the
+arithmetic runs in the library's CUDA kernels; there is no fallback.  If the
+shared library is missing, loading it raises with the build command.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbitlinear.so")
+
+_c_i64 = ctypes.c_int64
+_c_p = ctypes.c_void_p
+_c_sz = ctypes.c_size_t
+
+_SIGS = {
+    "bitlinear_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "bitlinear_version": (ctypes.c_int, []),
+    "bitlinear_packed_bytes": (_c_sz, [_c_i64, _c_i64]),
+    "bitlinear_pack_workspace_bytes": (_c_sz, [_c_i64, _c_i64]),
+    "bitlinear_workspace_bytes": (_c_sz, [_c_i64, _c_i64, _c_i64]),
+    "bitlinear_host_workspace_bytes": (_c_sz, [_c_i64, _c_i64, _c_i64]),
+    "bitlinear_pack_weights": (ctypes.c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_p, _c_p, _c_p, _c_sz, _c_p]),
+    "bitlinear_quant_act": (ctypes.c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_p, _c_p, _c_p]),
+    "bitlinear_forward": (ctypes.c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_i64, _c_p, _c_p, _c_p, _c_p, _c_sz,
+                                         _c_p]),
+    "bitlinear_forward_q8": (ctypes.c_int, [_c_p, _c_p, _c_p, _c_i64, _c_i64, _c_p, _c_i64, _c_p, _c_p, _c_p,
+                                            _c_p, _c_sz, _c_p]),
+    "bitlinear_forward_debug": (ctypes.c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_i64, _c_p, _c_p, _c_p, _c_p,
+                                               _c_p, _c_p, _c_p, ctypes.c_int, _c_p, _c_sz, _c_p]),
+    "bitlinear_forward_host": (ctypes.c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_i64, _c_p, _c_p, _c_p, _c_p,
+                                              _c_sz, _c_p]),
+    "bitlinear_check_status": (ctypes.c_int, [_c_p, _c_sz, _c_p]),
+}
+
+_lib = None
+
+
+class BitLinearError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded shared library (loaded on first use)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing; build it with `python -m bitlinear_fwd_b200.build`")
+        h = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(h, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = h
+    return _lib
+
+
+def exported_symbols() -> list[str]:
+    return list(_SIGS)
+
+
+def status_string(status: int) -> str:
+    return lib().bitlinear_status_string(int(status)).decode()
+
+
+def _check(st: int, where: str) -> None:
+    if st != 0:
+        raise BitLinearError(st, where)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(dev: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def _bits(t: torch.Tensor) -> torch.Tensor:
+    if t.dtype != torch.bfloat16:
+        raise TypeError("expected a bfloat16 tensor")
+    return t.contiguous()
+
+
+def packed_bytes(N: int, K: int) -> int:
+    return int(lib().bitlinear_packed_bytes(N, K))
+
+
+def workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(lib().bitlinear_workspace_bytes(M, N, K))
+
+
+def host_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(lib().bitlinear_host_workspace_bytes(M, N, K))
+
+
+def pack_workspace_bytes(N: int, K: int) -> int:
+    return int(lib().bitlinear_pack_workspace_bytes(N, K))
+
+
+def workspace(M: int, N: int, K: int, device, host: bool = False) -> torch.Tensor:
+    n = host_workspace_bytes(M, N, K) if host else workspace_bytes(M, N, K)
+    if n == 0:
+        raise BitLinearError(-2, "workspace")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def bitlinear_pack_weights(w: torch.Tensor, ws: Optional[torch.Tensor] = None):
+    """_weight_quant + 2-bit packing.  w: float32 [N, K] on the GPU.
+    Returns (packed uint8 [N, K/4], w_scale float32 [1], w_mean float32 [1])."""
+    w = w.contiguous()
+    if w.dtype != torch.float32 or w.dim() != 2:
+        raise TypeError("w must be a float32 [N, K] tensor")
+    N, K = w.shape
+    packed = torch.empty((N, K // 4), dtype=torch.uint8, device=w.device)
+    w_scale = torch.empty(1, dtype=torch.float32, device=w.device)
+    w_mean = torch.empty(1, dtype=torch.float32, device=w.device)
+    if ws is None:
+        ws = torch.empty(pack_workspace_bytes(N, K), dtype=torch.uint8, device=w.device)
+    _check(lib().bitlinear_pack_weights(_ptr(w), N, K, _ptr(packed), _ptr(w_scale), _ptr(w_mean), _ptr(ws),
+                                        ws.numel(), _stream(w.device)), "bitlinear_pack_weights")
+    return packed, w_scale, w_mean
+
+
+def bitlinear_quant_act(x: torch.Tensor):
+    """activation_norm_quant.  x: bf16 [M, K].  Returns (xq int8, s_x f32, rowsum i32)."""
+    x = _bits(x)
+    M, K = x.shape
+    xq = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    s_x = torch.empty(M, dtype=torch.float32, device=x.device)
+    rs = torch.empty(M, dtype=torch.int32, device=x.device)
+    _check(lib().bitlinear_quant_act(_ptr(x), M, K, _ptr(xq), _ptr(s_x), _ptr(rs), _stream(x.device)),
+           "bitlinear_quant_act")
+    return xq, s_x, rs
+
+
+def bitlinear_forward(x: torch.Tensor, packed: torch.Tensor, w_scale: torch.Tensor,
+                      bias: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                      out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """BitLinear.forward: y bf16 [M, N] from x bf16 [M, K] and packed weights."""
+    x = _bits(x)
+    M, K = x.shape
+    N = packed.shape[0]
+    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    if ws is None:
+        ws = workspace(M, N, K, x.device)
+    b = None if bias is None else _bits(bias)
+    _check(lib().bitlinear_forward(_ptr(x), M, K, _ptr(packed), N, _ptr(w_scale), _ptr(b), _ptr(y), _ptr(ws),
+                                   ws.numel(), _stream(x.device)), "bitlinear_forward")
+    return y
+
+
+def bitlinear_forward_q8(xq: torch.Tensor, s_x: torch.Tensor, rowsum: torch.Tensor, packed: torch.Tensor,
+                         w_scale: torch.Tensor, bias: Optional[torch.Tensor] = None,
+                         ws: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Contraction + epilogue on activations from bitlinear_quant_act."""
+    M, K = xq.shape
+    N = packed.shape[0]
+    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=xq.device)
+    if ws is None:
+        ws = torch.zeros(256, dtype=torch.uint8, device=xq.device)
+    b = None if bias is None else _bits(bias)
+    _check(lib().bitlinear_forward_q8(_ptr(xq), _ptr(s_x), _ptr(rowsum), M, K, _ptr(packed), N, _ptr(w_scale),
+                                      _ptr(b), _ptr(y), _ptr(ws), ws.numel(), _stream(xq.device)),
+           "bitlinear_forward_q8")
+    return y
+
+
+def bitlinear_forward_debug(x: torch.Tensor, packed: torch.Tensor, w_scale: torch.Tensor,
+                            bias: Optional[torch.Tensor] = None, engine: int = 0,
+                            ws: Optional[torch.Tensor] = None) -> dict:
+    """Forward with intermediates: y, xq, s_x, acc (int32), y32 (float32)."""
+    x = _bits(x)
+    M, K = x.shape
+    N = packed.shape[0]
+    dev = x.device
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    xq = torch.empty((M, K), dtype=torch.int8, device=dev)
+    s_x = torch.empty(M, dtype=torch.float32, device=dev)
+    acc = torch.empty((M, N), dtype=torch.int32, device=dev)
+    y32 = torch.empty((M, N), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = workspace(M, N, K, dev)
+    b = None if bias is None else _bits(bias)
+    _check(lib().bitlinear_forward_debug(_ptr(x), M, K, _ptr(packed), N, _ptr(w_scale), _ptr(b), _ptr(y),
+                                         _ptr(xq), _ptr(s_x), _ptr(acc), _ptr(y32), engine, _ptr(ws),
+                                         ws.numel(), _stream(dev)), "bitlinear_forward_debug")
+    return {"y": y, "xq": xq, "s_x": s_x, "acc": acc, "y32": y32, "ws": ws}
+
+
+def bitlinear_forward_host(x_host: torch.Tensor, packed: torch.Tensor, w_scale: torch.Tensor,
+                           bias: Optional[torch.Tensor] = None, y_host: Optional[torch.Tensor] = None,
+                           ws: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Forward from host activations to a host output (synchronous)."""
+    x_host = _bits(x_host)
+    M, K = x_host.shape
+    N = packed.shape[0]
+    dev = packed.device
+    if y_host is None:
+        y_host = torch.empty((M, N), dtype=torch.bfloat16, pin_memory=True)
+    if ws is None:
+        ws = workspace(M, N, K, dev, host=True)
+    b = None if bias is None else _bits(bias)
+    _check(lib().bitlinear_forward_host(_ptr(x_host), M, K, _ptr(packed), N, _ptr(w_scale), _ptr(b),
+                                        _ptr(y_host), _ptr(ws), ws.numel(), _stream(dev)),
+           "bitlinear_forward_host")
+    return y_host
+
+
+def bitlinear_check_status(ws: torch.Tensor) -> int:
+    """Status of the most recent call that used workspace ws (synchronises)."""
+    return int(lib().bitlinear_check_status(_ptr(ws), ws.numel(), _stream(ws.device)))

@@ -1,0 +1,161 @@
+// Per-token activation quantisation (activation_norm_quant of the
+// Falcon-Edge blog, section "Falcon-Edge, a series of universal models"):
+//   s_x = 127 / max(max_k |x|, 1e-5),  q = clamp(round_half_even(x * s_x), -128, 127)
+// in float32, plus the row sum of q that the contraction engines use.
+//
+// One CTA per row.  The row is read once with 16-byte loads and kept in
+// registers between the absmax pass and the quantisation pass (rows of up
+// to 32768 elements; longer rows are read twice).  The absmax runs on the
+// bf16 bit patterns: for finite values |x| orders like its bits & 0x7FFF.
+#include "kernels.h"
+
+namespace bitlinear {
+
+namespace {
+
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ uint32_t absmax_pair(uint32_t acc, uint32_t w) {
+  return __vmaxu2(acc, w & 0x7FFF7FFFu);
+}
+
+__device__ __forceinline__ uint32_t reduce_max_u32(uint32_t v, uint32_t* red) {
+  for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    uint32_t t = threadIdx.x < (kThreads / 32) ? red[threadIdx.x] : 0u;
+    for (int o = 16; o > 0; o >>= 1) t = max(t, __shfl_xor_sync(0xffffffffu, t, o));
+    if (threadIdx.x == 0) red[0] = t;
+  }
+  __syncthreads();
+  const uint32_t r = red[0];
+  __syncthreads();
+  return r;
+}
+
+__device__ __forceinline__ int reduce_add_i32(int v, int* red) {
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  int t = 0;
+  if (threadIdx.x == 0)
+    for (int i = 0; i < kThreads / 32; ++i) t += red[i];
+  return t;  // valid in thread 0
+}
+
+// Quantises 16 bf16 values (two 16-byte vectors) into one 16-byte vector of int8.
+__device__ __forceinline__ uint4 quant16(uint4 lo, uint4 hi, float s, int& sum) {
+  const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+  uint32_t out[4];
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    uint32_t packed = 0;
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      const int e = 4 * b + h;  // element 0..15
+      const uint32_t bits = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu);
+      const float t = __fmul_rn(bf16_bits_to_f32(bits), s);
+      int q = __float2int_rn(t);
+      q = min(127, max(-128, q));
+      sum += q;
+      packed |= (static_cast<uint32_t>(q) & 0xFFu) << (8 * h);
+    }
+    out[b] = packed;
+  }
+  return make_uint4(out[0], out[1], out[2], out[3]);
+}
+
+template <int CPT>  // 16-element chunks cached per thread; 0 = read the row twice
+__global__ void __launch_bounds__(kThreads) act_quant_kernel(const uint16_t* __restrict__ x, int K,
+                                                             int8_t* __restrict__ xq,
+                                                             float* __restrict__ s_x,
+                                                             int32_t* __restrict__ rowsum,
+                                                             uint32_t* status_clear) {
+  pdl_launch_dependents();
+  if (status_clear && blockIdx.x == 0 && threadIdx.x == 0) *status_clear = 0u;
+  __shared__ uint32_t red[kThreads / 32];
+
+  const int row = blockIdx.x;
+  const int chunks = K >> 4;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<size_t>(row) * K);
+  uint4* qr = reinterpret_cast<uint4*>(xq + static_cast<size_t>(row) * K);
+
+  uint4 cache[CPT > 0 ? 2 * CPT : 1];
+  uint32_t amax = 0;
+  if constexpr (CPT > 0) {
+#pragma unroll
+    for (int i = 0; i < CPT; ++i) {
+      const int c = threadIdx.x + i * kThreads;
+      if (c < chunks) {
+        cache[2 * i] = __ldg(xr + 2 * c);
+        cache[2 * i + 1] = __ldg(xr + 2 * c + 1);
+      } else {
+        cache[2 * i] = make_uint4(0, 0, 0, 0);
+        cache[2 * i + 1] = make_uint4(0, 0, 0, 0);
+      }
+      amax = absmax_pair(amax, cache[2 * i].x);
+      amax = absmax_pair(amax, cache[2 * i].y);
+      amax = absmax_pair(amax, cache[2 * i].z);
+      amax = absmax_pair(amax, cache[2 * i].w);
+      amax = absmax_pair(amax, cache[2 * i + 1].x);
+      amax = absmax_pair(amax, cache[2 * i + 1].y);
+      amax = absmax_pair(amax, cache[2 * i + 1].z);
+      amax = absmax_pair(amax, cache[2 * i + 1].w);
+    }
+  } else {
+    for (int c = threadIdx.x; c < chunks; c += kThreads) {
+      const uint4 a = __ldg(xr + 2 * c), b = __ldg(xr + 2 * c + 1);
+      amax = absmax_pair(amax, a.x); amax = absmax_pair(amax, a.y);
+      amax = absmax_pair(amax, a.z); amax = absmax_pair(amax, a.w);
+      amax = absmax_pair(amax, b.x); amax = absmax_pair(amax, b.y);
+      amax = absmax_pair(amax, b.z); amax = absmax_pair(amax, b.w);
+    }
+  }
+  amax = max(amax & 0xFFFFu, amax >> 16);
+  amax = reduce_max_u32(amax, red);
+
+  const float a = bf16_bits_to_f32(amax);
+  const float s = __fdiv_rn(127.0f, fmaxf(a, 1e-5f));
+
+  int sum = 0;
+  if constexpr (CPT > 0) {
+#pragma unroll
+    for (int i = 0; i < CPT; ++i) {
+      const int c = threadIdx.x + i * kThreads;
+      if (c < chunks) qr[c] = quant16(cache[2 * i], cache[2 * i + 1], s, sum);
+    }
+  } else {
+    for (int c = threadIdx.x; c < chunks; c += kThreads)
+      qr[c] = quant16(__ldg(xr + 2 * c), __ldg(xr + 2 * c + 1), s, sum);
+  }
+  sum = reduce_add_i32(sum, reinterpret_cast<int*>(red));
+  if (threadIdx.x == 0) {
+    s_x[row] = s;
+    if (rowsum) rowsum[row] = sum;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_act_quant(const uint16_t* x, int M, int K, int8_t* xq, float* s_x,
+                             int32_t* rowsum, uint32_t* status_clear, cudaStream_t stream) {
+  if (M <= 0) return cudaSuccess;
+  const int chunks = K / 16;
+  const dim3 grid(M), block(kThreads);
+  if (chunks <= kThreads)
+    act_quant_kernel<1><<<grid, block, 0, stream>>>(x, K, xq, s_x, rowsum, status_clear);
+  else if (chunks <= 2 * kThreads)
+    act_quant_kernel<2><<<grid, block, 0, stream>>>(x, K, xq, s_x, rowsum, status_clear);
+  else if (chunks <= 4 * kThreads)
+    act_quant_kernel<4><<<grid, block, 0, stream>>>(x, K, xq, s_x, rowsum, status_clear);
+  else if (chunks <= 8 * kThreads)
+    act_quant_kernel<8><<<grid, block, 0, stream>>>(x, K, xq, s_x, rowsum, status_clear);
+  else
+    act_quant_kernel<0><<<grid, block, 0, stream>>>(x, K, xq, s_x, rowsum, status_clear);
+  return cudaGetLastError();
+}
+
+}  // namespace bitlinear

@@ -1,0 +1,291 @@
+// C ABI of libbitlinear.so: argument checks, workspace layout and the
+// choice of contraction engine.  Declarations and the contract of each
+// entry point are in include/bitlinear.h.
+#include <stdint.h>
+#include <string.h>
+
+#include "../../include/bitlinear.h"
+#include "kernels.h"
+
+using namespace bitlinear;
+
+namespace {
+
+constexpr int64_t kMaxMN = int64_t(1) << 23;
+constexpr int64_t kMaxK = int64_t(1) << 19;
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+bool misaligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
+
+// Forward workspace: [status | s_x | rowsum | xq | (host staging: x | y)]
+struct FwdLayout {
+  size_t off_sx, off_rs, off_xq, end_dev, off_xh, off_yh, end_host;
+};
+
+FwdLayout fwd_layout(int64_t M, int64_t N, int64_t K) {
+  FwdLayout L;
+  L.off_sx = 256;
+  L.off_rs = align_up(L.off_sx + 4 * size_t(M), 256);
+  L.off_xq = align_up(L.off_rs + 4 * size_t(M), 1024);
+  L.end_dev = align_up(L.off_xq + size_t(M) * size_t(K), 256);
+  L.off_xh = L.end_dev;
+  L.off_yh = align_up(L.off_xh + 2 * size_t(M) * size_t(K), 256);
+  L.end_host = align_up(L.off_yh + 2 * size_t(M) * size_t(N), 256);
+  return L;
+}
+
+struct DevInfo {
+  int checked = 0;  // 0 unknown, 1 ok, -1 not sm_100
+  int sms = 148;
+};
+DevInfo g_dev[64];
+
+int check_device(int* sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BITLINEAR_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return BITLINEAR_ERR_DEVICE;
+  DevInfo& d = g_dev[dev];
+  if (d.checked == 0) {
+    int major = 0, minor = 0, n = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return BITLINEAR_ERR_CUDA;
+    d.sms = n;
+    d.checked = (major == 10 && minor == 0) ? 1 : -1;
+  }
+  if (sms) *sms = d.sms;
+  return d.checked == 1 ? BITLINEAR_OK : BITLINEAR_ERR_DEVICE;
+}
+
+int check_shape(int64_t M, int64_t N, int64_t K) {
+  if (M < 0 || M > kMaxMN || N < 1 || N > kMaxMN || K < 64 || K > kMaxK || (K % 64) != 0)
+    return BITLINEAR_ERR_SHAPE;
+  return BITLINEAR_OK;
+}
+
+int status_of(cudaError_t e) { return e == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA; }
+
+// Shared body of the forward entry points; x is a device pointer.
+int forward_impl(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed_w, int64_t N,
+                 const float* w_scale, const uint16_t* bias, uint16_t* y, int8_t* xq_out, float* sx_out,
+                 int32_t* acc_out, float* y32_out, int engine, void* ws, size_t ws_bytes,
+                 cudaStream_t stream) {
+  int sms = 148;
+  int st = check_device(&sms);
+  if (st != BITLINEAR_OK) return st;
+  const FwdLayout L = fwd_layout(M, N, K);
+  char* base = static_cast<char*>(ws);
+  uint32_t* status = reinterpret_cast<uint32_t*>(base);
+  float* s_x = reinterpret_cast<float*>(base + L.off_sx);
+  int32_t* rowsum = reinterpret_cast<int32_t*>(base + L.off_rs);
+  int8_t* xq = reinterpret_cast<int8_t*>(base + L.off_xq);
+
+  cudaError_t e = launch_act_quant(x, int(M), int(K), xq, s_x, rowsum, status, stream);
+  if (e != cudaSuccess) return BITLINEAR_ERR_CUDA;
+
+  ForwardArgs a;
+  a.xq = xq;
+  a.s_x = s_x;
+  a.rowsum = rowsum;
+  a.packed = packed_w;
+  a.w_scale = w_scale;
+  a.bias = bias;
+  a.y = y;
+  a.acc_out = acc_out;
+  a.y32_out = y32_out;
+  a.status = status;
+  a.M = int(M);
+  a.N = int(N);
+  a.K = int(K);
+  a.pdl = true;
+  const bool decode = engine == 1 || (engine == 0 && M <= 16);
+  e = decode ? launch_gemv_decode(a, sms, stream) : launch_gemm_prefill(a, sms, stream);
+  if (e != cudaSuccess) return BITLINEAR_ERR_CUDA;
+  if (xq_out) e = cudaMemcpyAsync(xq_out, xq, size_t(M) * size_t(K), cudaMemcpyDeviceToDevice, stream);
+  if (e == cudaSuccess && sx_out) e = cudaMemcpyAsync(sx_out, s_x, 4 * size_t(M), cudaMemcpyDeviceToDevice, stream);
+  return status_of(e);
+}
+
+int check_forward_args(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed_w, int64_t N,
+                       const float* w_scale, const uint16_t* bias, uint16_t* y, void* ws, size_t ws_bytes,
+                       size_t need, bool host) {
+  int st = check_shape(M, N, K);
+  if (st != BITLINEAR_OK) return st;
+  if (!x || !packed_w || !w_scale || !y) return BITLINEAR_ERR_NULL;
+  if ((!host && (misaligned(x) || misaligned(y))) || misaligned(packed_w) || misaligned(w_scale) ||
+      misaligned(bias))
+    return BITLINEAR_ERR_ALIGN;
+  if (!ws || ws_bytes < need) return BITLINEAR_ERR_WORKSPACE;
+  if (misaligned(ws)) return BITLINEAR_ERR_ALIGN;
+  return BITLINEAR_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* bitlinear_status_string(int status) {
+  switch (status) {
+    case BITLINEAR_OK: return "BITLINEAR_OK";
+    case BITLINEAR_ERR_NULL: return "BITLINEAR_ERR_NULL: a required pointer is NULL";
+    case BITLINEAR_ERR_SHAPE: return "BITLINEAR_ERR_SHAPE: bad M, N or K (K must be a positive multiple of 64)";
+    case BITLINEAR_ERR_ALIGN: return "BITLINEAR_ERR_ALIGN: a device pointer is not 16-byte aligned";
+    case BITLINEAR_ERR_WORKSPACE: return "BITLINEAR_ERR_WORKSPACE: workspace missing or too small";
+    case BITLINEAR_ERR_CUDA: return "BITLINEAR_ERR_CUDA: a CUDA call or kernel launch failed";
+    case BITLINEAR_ERR_TIMEOUT: return "BITLINEAR_ERR_TIMEOUT: a device-side wait gave up";
+    case BITLINEAR_ERR_DEVICE: return "BITLINEAR_ERR_DEVICE: the current GPU is not sm_100 (B200)";
+    default: return "BITLINEAR: unknown status";
+  }
+}
+
+int bitlinear_version(void) { return (1 << 16) | 0; }
+
+size_t bitlinear_packed_bytes(int64_t N, int64_t K) {
+  if (N < 1 || K < 64 || (K % 64) != 0) return 0;
+  return size_t(N) * size_t(K) / 4;
+}
+
+size_t bitlinear_pack_workspace_bytes(int64_t N, int64_t K) {
+  (void)N;
+  (void)K;
+  return kPackWsBytes;
+}
+
+size_t bitlinear_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (check_shape(M, N, K) != BITLINEAR_OK) return 0;
+  return fwd_layout(M, N, K).end_dev;
+}
+
+size_t bitlinear_host_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (check_shape(M, N, K) != BITLINEAR_OK) return 0;
+  return fwd_layout(M, N, K).end_host;
+}
+
+int bitlinear_pack_weights(const float* w, int64_t N, int64_t K, uint8_t* packed, float* w_scale,
+                           float* w_mean, void* ws, size_t ws_bytes, void* stream) {
+  if (N < 1 || K < 64 || (K % 64) != 0 || N > kMaxMN || K > kMaxK || N * K >= (int64_t(1) << 40))
+    return BITLINEAR_ERR_SHAPE;
+  if (!w || !packed || !w_scale) return BITLINEAR_ERR_NULL;
+  if (misaligned(w) || misaligned(packed) || misaligned(w_scale) || misaligned(w_mean))
+    return BITLINEAR_ERR_ALIGN;
+  if (!ws || ws_bytes < kPackWsBytes) return BITLINEAR_ERR_WORKSPACE;
+  if (misaligned(ws)) return BITLINEAR_ERR_ALIGN;
+  int st = check_device(nullptr);
+  if (st != BITLINEAR_OK) return st;
+  return status_of(launch_pack(w, N, K, packed, w_scale, w_mean, pack_workspace(ws),
+                               static_cast<cudaStream_t>(stream)));
+}
+
+int bitlinear_quant_act(const uint16_t* x, int64_t M, int64_t K, int8_t* xq, float* x_scale,
+                        int32_t* xq_rowsum, void* stream) {
+  if (M < 0 || M > kMaxMN || K < 64 || K > kMaxK || (K % 64) != 0) return BITLINEAR_ERR_SHAPE;
+  if (M == 0) return BITLINEAR_OK;
+  if (!x || !xq || !x_scale) return BITLINEAR_ERR_NULL;
+  if (misaligned(x) || misaligned(xq) || misaligned(x_scale) || misaligned(xq_rowsum))
+    return BITLINEAR_ERR_ALIGN;
+  int st = check_device(nullptr);
+  if (st != BITLINEAR_OK) return st;
+  return status_of(launch_act_quant(x, int(M), int(K), xq, x_scale, xq_rowsum, nullptr,
+                                    static_cast<cudaStream_t>(stream)));
+}
+
+int bitlinear_forward(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed_w, int64_t N,
+                      const float* w_scale, const uint16_t* bias, uint16_t* y, void* ws, size_t ws_bytes,
+                      void* stream) {
+  int st = check_forward_args(x, M, K, packed_w, N, w_scale, bias, y, ws, ws_bytes,
+                              bitlinear_workspace_bytes(M, N, K), false);
+  if (st != BITLINEAR_OK) return st;
+  if (M == 0) return BITLINEAR_OK;
+  return forward_impl(x, M, K, packed_w, N, w_scale, bias, y, nullptr, nullptr, nullptr, nullptr, 0, ws,
+                      ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int bitlinear_forward_q8(const int8_t* xq, const float* x_scale, const int32_t* xq_rowsum, int64_t M,
+                         int64_t K, const uint8_t* packed_w, int64_t N, const float* w_scale,
+                         const uint16_t* bias, uint16_t* y, void* ws, size_t ws_bytes, void* stream) {
+  int st = check_shape(M, N, K);
+  if (st != BITLINEAR_OK) return st;
+  if (!xq || !x_scale || !xq_rowsum || !packed_w || !w_scale || !y) return BITLINEAR_ERR_NULL;
+  if (misaligned(xq) || misaligned(x_scale) || misaligned(xq_rowsum) || misaligned(packed_w) ||
+      misaligned(w_scale) || misaligned(bias) || misaligned(y))
+    return BITLINEAR_ERR_ALIGN;
+  if (!ws || ws_bytes < 256) return BITLINEAR_ERR_WORKSPACE;
+  if (misaligned(ws)) return BITLINEAR_ERR_ALIGN;
+  if (M == 0) return BITLINEAR_OK;
+  int sms = 148;
+  st = check_device(&sms);
+  if (st != BITLINEAR_OK) return st;
+  ForwardArgs a;
+  a.xq = xq;
+  a.s_x = x_scale;
+  a.rowsum = xq_rowsum;
+  a.packed = packed_w;
+  a.w_scale = w_scale;
+  a.bias = bias;
+  a.y = y;
+  a.acc_out = nullptr;
+  a.y32_out = nullptr;
+  a.status = static_cast<uint32_t*>(ws);
+  a.M = int(M);
+  a.N = int(N);
+  a.K = int(K);
+  a.pdl = false;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return status_of(M <= 16 ? launch_gemv_decode(a, sms, s) : launch_gemm_prefill(a, sms, s));
+}
+
+int bitlinear_forward_debug(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed_w, int64_t N,
+                            const float* w_scale, const uint16_t* bias, uint16_t* y, int8_t* xq,
+                            float* x_scale, int32_t* acc, float* y32, int engine, void* ws,
+                            size_t ws_bytes, void* stream) {
+  int st = check_forward_args(x, M, K, packed_w, N, w_scale, bias, y, ws, ws_bytes,
+                              bitlinear_workspace_bytes(M, N, K), false);
+  if (st != BITLINEAR_OK) return st;
+  if (engine < 0 || engine > 2 || (engine == 1 && M > 16)) return BITLINEAR_ERR_SHAPE;
+  if (misaligned(xq) || misaligned(x_scale) || misaligned(acc) || misaligned(y32)) return BITLINEAR_ERR_ALIGN;
+  if (M == 0) return BITLINEAR_OK;
+  return forward_impl(x, M, K, packed_w, N, w_scale, bias, y, xq, x_scale, acc, y32, engine, ws, ws_bytes,
+                      static_cast<cudaStream_t>(stream));
+}
+
+int bitlinear_forward_host(const uint16_t* x_host, int64_t M, int64_t K, const uint8_t* packed_w, int64_t N,
+                           const float* w_scale, const uint16_t* bias, uint16_t* y_host, void* ws,
+                           size_t ws_bytes, void* stream) {
+  int st = check_forward_args(x_host, M, K, packed_w, N, w_scale, bias, y_host, ws, ws_bytes,
+                              bitlinear_host_workspace_bytes(M, N, K), true);
+  if (st != BITLINEAR_OK) return st;
+  if (M == 0) return BITLINEAR_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const FwdLayout L = fwd_layout(M, N, K);
+  char* base = static_cast<char*>(ws);
+  uint16_t* xd = reinterpret_cast<uint16_t*>(base + L.off_xh);
+  uint16_t* yd = reinterpret_cast<uint16_t*>(base + L.off_yh);
+  if (cudaMemcpyAsync(xd, x_host, 2 * size_t(M) * size_t(K), cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return BITLINEAR_ERR_CUDA;
+  st = forward_impl(xd, M, K, packed_w, N, w_scale, bias, yd, nullptr, nullptr, nullptr, nullptr, 0, ws,
+                    ws_bytes, s);
+  if (st != BITLINEAR_OK) return st;
+  if (cudaMemcpyAsync(y_host, yd, 2 * size_t(M) * size_t(N), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return BITLINEAR_ERR_CUDA;
+  return status_of(cudaStreamSynchronize(s));
+}
+
+int bitlinear_check_status(const void* ws, size_t ws_bytes, void* stream) {
+  if (!ws) return BITLINEAR_ERR_NULL;
+  if (ws_bytes < 4) return BITLINEAR_ERR_WORKSPACE;
+  uint32_t word = 0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&word, ws, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess) return BITLINEAR_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return BITLINEAR_ERR_CUDA;
+  if (word != 0) {
+    const uint32_t zero = 0;
+    if (cudaMemcpyAsync(const_cast<void*>(ws), &zero, 4, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+      return BITLINEAR_ERR_CUDA;
+  }
+  return (word & kStatusTimeout) ? BITLINEAR_ERR_TIMEOUT : BITLINEAR_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,50 @@
+// Internal launch functions of the BitLinear kernels (not part of the C ABI).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace bitlinear {
+
+// ---- activation quantisation (act_quant.cu) --------------------------------
+cudaError_t launch_act_quant(const uint16_t* x, int M, int K, int8_t* xq, float* s_x,
+                             int32_t* rowsum, uint32_t* status_clear, cudaStream_t stream);
+
+// ---- weight absmean + ternarise + pack (pack.cu) ----------------------------
+// Workspace layout used by the pack kernels.
+struct PackWorkspace {
+  uint32_t* status;   // 1 word
+  float* mean;        // 1 float
+  uint64_t* bins;     // 256 exponent bins
+};
+constexpr size_t kPackWsBytes = 4096;
+PackWorkspace pack_workspace(void* ws);
+cudaError_t launch_pack(const float* w, int64_t N, int64_t K, uint8_t* packed, float* w_scale,
+                        float* w_mean, const PackWorkspace& pws, cudaStream_t stream);
+
+// ---- shared forward arguments ----------------------------------------------
+struct ForwardArgs {
+  const int8_t* xq;       // [M, K]
+  const float* s_x;       // [M]
+  const int32_t* rowsum;  // [M]
+  const uint8_t* packed;  // [N, K/4]
+  const float* w_scale;   // [1]
+  const uint16_t* bias;   // [N] or null
+  uint16_t* y;            // [M, N]
+  int32_t* acc_out;       // [M, N] or null (debug)
+  float* y32_out;         // [M, N] or null (debug)
+  uint32_t* status;       // status word
+  int M, N, K;
+  bool pdl;               // launched as a programmatic dependent of the act-quant kernel
+};
+
+// ---- decode engine, M <= 16 (gemv_decode.cu) --------------------------------
+cudaError_t launch_gemv_decode(const ForwardArgs& a, int num_sms, cudaStream_t stream);
+
+// ---- prefill engine, tcgen05 GEMM (gemm_prefill.cu) -------------------------
+cudaError_t launch_gemm_prefill(const ForwardArgs& a, int num_sms, cudaStream_t stream);
+
+}  // namespace bitlinear

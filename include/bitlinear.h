@@ -1,0 +1,178 @@
+/*
+ * bitlinear.h -- C ABI of libbitlinear.so, the BitNet b1.58 BitLinear forward
+ * for NVIDIA B200 (sm_100a).
+ *
+ * The operation follows the Falcon-Edge blog (Falcon-LLM team, "Falcon-Edge:
+ * a series of powerful, universal and fine-tunable 1.58bit language models";
+ * section "Falcon-Edge, a series of universal models"), whose listings define
+ *   activation_norm_quant(x):  s_x = 127 / max(max_k |x|, 1e-5) per token,
+ *                              q = clamp(round(x * s_x), -128, 127)
+ *   _weight_quant(w):          s_w = 1 / max(mean |w|, 1e-5) over the tensor,
+ *                              u = clamp(round(w * s_w), -1, 1)
+ *   BitLinear.forward(x):      y = F.linear(q, u) / (s_x * s_w) (+ bias)
+ * Weights are ternary {-1, 0, 1} ("The Era of 1-bit LLMs", TL;DR) and are
+ * stored in 2 bits each ("BitNet: inference framework for 1-bit LLMs",
+ * GeekNews, Hacker News comments section).
+ *
+ * Numerics (identical to the CPU oracle that the tests compare against):
+ *   - bf16 inputs widen exactly to float32; scales, x*s_x and w*s_w are
+ *     float32 round-to-nearest; round() is round-half-to-even;
+ *   - mean |w| is the exact sum over the whole tensor divided by N*K and
+ *     rounded once to float32 (independent of summation order);
+ *   - the contraction is exact in int32 (|acc| <= 127*K);
+ *   - d = s_x*s_w (float32), y32 = float(acc) / d (float32, correctly
+ *     rounded), y32 += float(bias) if a bias is given, y = bf16_rne(y32).
+ *
+ * Conventions for every entry point:
+ *   - Shapes: x is [M, K] row-major, W is [N, K] (nn.Linear [out, in]),
+ *     y is [M, N].  K must be a positive multiple of 64; M >= 0, N >= 1.
+ *     M == 0 is a no-op that returns BITLINEAR_OK.
+ *   - bf16 values travel as their uint16_t bit patterns.
+ *   - Every pointer argument is a DEVICE pointer unless its name ends in
+ *     _host.  Device pointers must be 16-byte aligned (BITLINEAR_ERR_ALIGN
+ *     otherwise).  All buffers are owned by the caller; the library
+ *     allocates nothing and keeps no state between calls.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Work
+ *     is enqueued on it and the call returns without synchronising, except
+ *     where stated.  Calls on different streams with distinct workspaces
+ *     may run concurrently.
+ *   - Argument errors are detected on the host before anything is enqueued.
+ *     A failed launch returns BITLINEAR_ERR_CUDA.  Device-side bounded waits
+ *     that give up (never expected in normal operation) set a bit in the
+ *     workspace status word; read it with bitlinear_check_status.
+ *   - Inputs must be finite; the result for Inf/NaN inputs is unspecified.
+ *   - The GPU must be compute capability 10.0 (B200); otherwise
+ *     BITLINEAR_ERR_DEVICE.
+ *
+ * Packed weight layout (the pages leave it open; this is the library's):
+ * the code u + 1 in {0, 1, 2} of each weight takes 2 bits; row n of the
+ * packed matrix is K/4 bytes = K/16 little-endian uint32 words; word g of a
+ * row holds k = 16g + 4i + j in bits 8j + 2i .. 8j + 2i + 1 (byte j, bit
+ * pair i), so that (word >> 2i) & 0x03030303 gives the codes of four
+ * consecutive k in byte lanes.  Code 3 never occurs.
+ */
+#ifndef BITLINEAR_H_
+#define BITLINEAR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BITLINEAR_OK = 0,
+  BITLINEAR_ERR_NULL = -1,      /* a required pointer is NULL */
+  BITLINEAR_ERR_SHAPE = -2,     /* M < 0, N < 1, K < 64 or K % 64 != 0, or too large */
+  BITLINEAR_ERR_ALIGN = -3,     /* a device pointer is not 16-byte aligned */
+  BITLINEAR_ERR_WORKSPACE = -4, /* workspace NULL or smaller than required */
+  BITLINEAR_ERR_CUDA = -5,      /* a CUDA runtime call or launch failed */
+  BITLINEAR_ERR_TIMEOUT = -6,   /* a device-side bounded wait gave up */
+  BITLINEAR_ERR_DEVICE = -7     /* the current GPU is not sm_100 */
+} bitlinear_status;
+
+/* Human-readable name of a status code (static storage; never NULL). */
+const char* bitlinear_status_string(int status);
+
+/* ABI version, (major << 16) | minor. */
+int bitlinear_version(void);
+
+/* Bytes of the packed weight matrix: N * K / 4. */
+size_t bitlinear_packed_bytes(int64_t N, int64_t K);
+
+/* Workspace bytes needed by bitlinear_pack_weights (exponent-binned exact
+ * sums, the mean, and the status word).  Independent of the shape. */
+size_t bitlinear_pack_workspace_bytes(int64_t N, int64_t K);
+
+/* Workspace bytes needed by bitlinear_forward and bitlinear_forward_debug
+ * for this shape: the status word, s_x [M], the row sums [M] and the int8
+ * activations [M, K].  Returns 0 for an invalid shape. */
+size_t bitlinear_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/* Workspace bytes needed by bitlinear_forward_host: the above plus device
+ * staging for x [M, K] and y [M, N].  Returns 0 for an invalid shape. */
+size_t bitlinear_host_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/* Weight ternarisation and 2-bit packing (_weight_quant followed by the
+ * storage packing that BitLinear.forward's unpack_weights undoes).
+ *   w        [N, K] float32, finite
+ *   packed   [N, K/4] uint8 out (bitlinear_packed_bytes)
+ *   w_scale  [1] float32 out: s_w = 1 / max(mean|w|, 1e-5); stays on the
+ *            device so that packing and the forward need no host sync
+ *   w_mean   [1] float32 out, the exactly rounded mean |w|; may be NULL
+ *   ws       workspace of bitlinear_pack_workspace_bytes bytes; its
+ *            contents on entry do not matter
+ * N * K must be below 2^40. */
+int bitlinear_pack_weights(const float* w, int64_t N, int64_t K, uint8_t* packed,
+                           float* w_scale, float* w_mean, void* ws, size_t ws_bytes,
+                           void* stream);
+
+/* Per-token activation quantisation (activation_norm_quant).
+ *   x          [M, K] bf16
+ *   xq         [M, K] int8 out
+ *   x_scale    [M] float32 out, s_x
+ *   xq_rowsum  [M] int32 out, sum_k xq (used by the contraction engines);
+ *              may be NULL */
+int bitlinear_quant_act(const uint16_t* x, int64_t M, int64_t K, int8_t* xq, float* x_scale,
+                        int32_t* xq_rowsum, void* stream);
+
+/* The BitLinear forward: y = BitLinear(x) with packed ternary weights.
+ *   x         [M, K] bf16
+ *   packed_w  [N, K/4] uint8 from bitlinear_pack_weights
+ *   w_scale   [1] float32 (device) from bitlinear_pack_weights
+ *   bias      [N] bf16, or NULL for no bias
+ *   y         [M, N] bf16 out
+ *   ws        workspace of at least bitlinear_workspace_bytes(M, N, K);
+ *             its contents on entry do not matter
+ * M <= 16 runs the decode engine (weight-streaming GEMV on warp-level int8
+ * MMA), M > 16 the prefill engine (tcgen05 int8 GEMM with accumulators in
+ * tensor memory).  Both quantise x first (one extra kernel). */
+int bitlinear_forward(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed_w,
+                      int64_t N, const float* w_scale, const uint16_t* bias, uint16_t* y,
+                      void* ws, size_t ws_bytes, void* stream);
+
+/* The contraction and epilogue of the forward on activations that
+ * bitlinear_quant_act has already quantised (so that several weight
+ * matrices that read the same input -- q/k/v, gate/up -- quantise it once).
+ *   xq [M, K] int8, x_scale [M] float32 and xq_rowsum [M] int32 as written
+ *   by bitlinear_quant_act; packed_w, w_scale, bias, y as for
+ *   bitlinear_forward; ws: at least 256 bytes (only the status word is
+ *   used).  This call does not reset the status word. */
+int bitlinear_forward_q8(const int8_t* xq, const float* x_scale, const int32_t* xq_rowsum, int64_t M,
+                         int64_t K, const uint8_t* packed_w, int64_t N, const float* w_scale,
+                         const uint16_t* bias, uint16_t* y, void* ws, size_t ws_bytes, void* stream);
+
+/* bitlinear_forward with intermediate outputs, for parity tests.  Same
+ * kernels; each extra output may be NULL:
+ *   xq [M, K] int8, x_scale [M] float32, acc [M, N] int32 (the exact
+ *   contraction sum_k q*u), y32 [M, N] float32 (before the bf16 rounding).
+ * engine: 0 = automatic (as bitlinear_forward), 1 = force the decode
+ * engine (requires M <= 16), 2 = force the prefill engine. */
+int bitlinear_forward_debug(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed_w,
+                            int64_t N, const float* w_scale, const uint16_t* bias, uint16_t* y,
+                            int8_t* xq, float* x_scale, int32_t* acc, float* y32, int engine,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/* bitlinear_forward with HOST activations and output: copies x_host to the
+ * device (through the workspace), runs the forward, copies y back to
+ * y_host and synchronises the stream before returning.  The weights,
+ * w_scale and bias stay device-resident.  ws must hold
+ * bitlinear_host_workspace_bytes(M, N, K).  Pinned host memory gives the
+ * fastest copies; pageable memory works. */
+int bitlinear_forward_host(const uint16_t* x_host, int64_t M, int64_t K, const uint8_t* packed_w,
+                           int64_t N, const float* w_scale, const uint16_t* bias,
+                           uint16_t* y_host, void* ws, size_t ws_bytes, void* stream);
+
+/* Reads and clears the status word of a workspace (synchronises
+ * `stream`).  bitlinear_pack_weights, bitlinear_forward, _debug and _host
+ * reset the word when they start; bitlinear_forward_q8 does not.  Returns
+ * BITLINEAR_OK, or BITLINEAR_ERR_TIMEOUT if a device-side bounded wait gave
+ * up since the last reset.  `ws_bytes` is the size the calls were given. */
+int bitlinear_check_status(const void* ws, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BITLINEAR_H_ */

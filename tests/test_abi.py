@@ -1,0 +1,79 @@
+"""Host-only checks of the C ABI: the library loads, exports every function
+that include/bitlinear.h declares, answers size queries, and rejects bad
+arguments before touching the GPU (no compute call is made here)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import bitlinear_fwd_b200 as bl
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bitlinear.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bitlinear_[a-z_0-9]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(bl.LIB_PATH):
+        from bitlinear_fwd_b200 import build
+        build.build()
+    return bl.lib()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(bl.exported_symbols()) == names
+
+
+def test_version_and_status_strings(lib):
+    assert lib.bitlinear_version() >> 16 == 1
+    for st in range(-7, 1):
+        assert bl.status_string(st).startswith("BITLINEAR")
+    assert "unknown" in bl.status_string(-99)
+
+
+def test_size_queries(lib):
+    assert bl.packed_bytes(512, 256) == 512 * 64
+    assert bl.packed_bytes(512, 100) == 0
+    assert bl.pack_workspace_bytes(1, 64) >= 256 + 256 * 8
+    ws = bl.workspace_bytes(8, 512, 256)
+    assert ws >= 8 * 256 + 8 * 4 * 2
+    assert bl.workspace_bytes(8, 512, 100) == 0
+    assert bl.host_workspace_bytes(8, 512, 256) >= ws + 2 * 8 * 256 + 2 * 8 * 512
+
+
+def _fwd(lib, x=16, M=8, K=256, w=16, N=512, s=16, b=None, y=16, ws=16, wsb=1 << 20):
+    return lib.bitlinear_forward(x, M, K, w, N, s, b, y, ws, wsb, None)
+
+
+def test_argument_errors_without_gpu(lib):
+    assert _fwd(lib, x=None) == -1
+    assert _fwd(lib, w=None) == -1
+    assert _fwd(lib, y=None) == -1
+    assert _fwd(lib, K=100) == -2
+    assert _fwd(lib, K=0) == -2
+    assert _fwd(lib, N=0) == -2
+    assert _fwd(lib, M=-1) == -2
+    assert _fwd(lib, x=18) == -3
+    assert _fwd(lib, b=20) == -3
+    assert _fwd(lib, ws=None) == -4
+    assert _fwd(lib, wsb=16) == -4
+    assert lib.bitlinear_pack_weights(16, 512, 100, 16, 16, None, 16, 4096, None) == -2
+    assert lib.bitlinear_pack_weights(None, 512, 256, 16, 16, None, 16, 4096, None) == -1
+    assert lib.bitlinear_pack_weights(16, 512, 256, 16, 16, None, 16, 8, None) == -4
+    assert lib.bitlinear_quant_act(16, 4, 96, 16, 16, None, None) == -2
+    assert lib.bitlinear_quant_act(16, 0, 64, 16, 16, None, None) == 0   # M == 0: nothing to do
+    assert lib.bitlinear_forward_debug(16, 32, 256, 16, 512, 16, None, 16, None, None, None, None, 1, 16,
+                                       1 << 20, None) == -2               # decode engine needs M <= 16
+    assert lib.bitlinear_check_status(None, 0, None) == -1
