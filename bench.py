@@ -1,0 +1,529 @@
+#!/usr/bin/env python
+"""Throughput of the BitNet b1.58 BitLinear forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Headline (one JSON line on rank 0): BitLinear decode GB/s of the decode
+sweep -- M in {1, 4, 16} tokens on the (K, N) = (4096, 4096) and
+(4096, 11008) projections, six bitlinear_forward calls per step -- with the
+packed weights resident in HBM and rotated over copies that total more than
+three times the L2 so that every step streams them from DRAM.  A step is
+captured once as a CUDA graph per weight copy and replayed.
+
+Also on the line:
+  roofline      the decode contraction kernel alone (launched through
+                bitlinear_forward_q8 between CUDA events on its stream):
+                algorithmic bytes per launch / mean launch time, against the
+                measured HBM copy bandwidth
+  prefill       int8 TOPS of the prefill workload (M in {512, 2048, 8192},
+                (K, N) = (3200, 8640) and (8640, 3200)), the same way, with
+                the tcgen05 GEMM's own roofline against the int8 peak
+  e2e           the decode metric through bitlinear_forward_host: host bf16
+                activations copied in and outputs copied back every call
+  cpu_baseline  the CPU oracle on a bounded sample of the decode workload
+  clocks        nvidia-smi samples taken while the workload ran
+
+With --gpus N > 1 (under torchrun) every rank runs the same workload on its
+own GPU (data-parallel replicas: tokens split, weights replicated; the
+forward has no exchange step), elapsed time is the max over ranks and the
+value is the total over ranks.  --impl reference times the CPU oracle (the
+only reference this method has) on the same metric, on rank 0 only.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth                                   # noqa: E402
+from synth import workloads as wl               # noqa: E402
+
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+INT8_OVER_BF16 = 2.0      # nominal dense ratio (4.5 / 2.25 PFLOP/s)
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def decode_bytes(M, N, K, bias=True):
+    """Algorithmic bytes of one BitLinear forward: 2-bit packed weights,
+    bf16 x in, bf16 y out, bf16 bias, fp32 s_w."""
+    return N * K // 4 + 2 * M * K + 2 * M * N + (2 * N if bias else 0) + 4
+
+
+def contraction_bytes(M, N, K, bias=True):
+    """Algorithmic bytes of the contraction kernel alone: packed weights,
+    int8 x, s_x and row sums, bias, bf16 y."""
+    return N * K // 4 + M * K + 8 * M + 2 * M * N + (2 * N if bias else 0) + 4
+
+
+def kernel_src_hash(name):
+    src = os.path.join(ROOT, "bitlinear_fwd_b200", "csrc", name)
+    return hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+
+
+def traffic_from_profile(profile_md, src_name):
+    """DRAM bytes per launch recorded in a committed ncu summary, or None when
+    the summary is missing or the kernel source changed since the capture."""
+    p = os.path.join(ROOT, "profiles", profile_md)
+    if not os.path.exists(p):
+        return None
+    text = open(p).read()
+    m = re.search(r"dram_bytes_per_launch_full_workload:\s*([0-9.eE+]+)", text)
+    h = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
+    if not m or not h or h.group(1) != kernel_src_hash(src_name):
+        return None
+    return float(m.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                       "-lms", "100", "-i", str(device_index)], stdout=self.f,
+                                      stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+
+    def stop(self):
+        if self.p is not None:
+            self.p.terminate()
+            try:
+                self.p.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.p.kill()
+        self.f.flush()
+        self.f.seek(0)
+        rows = [r.split(",") for r in self.f.read().strip().splitlines() if r.strip()]
+        os.unlink(self.f.name)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                s = float(r[1])
+                smax = float(r[2])
+            except (ValueError, IndexError):
+                continue
+            sm.append(s)
+            for nm, v in zip(names, r[5:9]):
+                if v.strip() == "Active":
+                    reasons.add(nm)
+        loaded = [s for s in sm if smax and s > 0.5 * smax] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def elapsed_max_over_ranks(ms):
+    if torch.distributed.is_available() and torch.distributed.is_initialized():
+        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+    return ms
+
+
+def barrier():
+    if torch.distributed.is_available() and torch.distributed.is_initialized():
+        torch.distributed.barrier()
+
+
+def sync_all():
+    barrier()
+    torch.cuda.synchronize()
+
+
+# ---------------------------------------------------------------------------
+# the GPU arm
+# ---------------------------------------------------------------------------
+
+class Problem:
+    def __init__(self, M, N, K, x, w_packed, s_w, bias, copies):
+        import bitlinear_fwd_b200 as bl
+        self.M, self.N, self.K = M, N, K
+        self.x = x
+        self.bias = bias
+        self.s_w = s_w
+        self.packed = [w_packed] + [w_packed.clone() for _ in range(copies - 1)]
+        self.y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        self.ws = bl.workspace(M, N, K, "cuda")
+        self.xq, self.s_x, self.rs = bl.bitlinear_quant_act(x)
+        self.ws_q8 = torch.zeros(256, dtype=torch.uint8, device="cuda")
+
+    def forward(self, r):
+        import bitlinear_fwd_b200 as bl
+        bl.bitlinear_forward(self.x, self.packed[r], self.s_w, self.bias, ws=self.ws, out=self.y,
+                             flags=bl.WEIGHTS_RESIDENT)
+
+    def contract(self, r):
+        import bitlinear_fwd_b200 as bl
+        bl.bitlinear_forward_q8(self.xq, self.s_x, self.rs, self.packed[r], self.s_w, self.bias, ws=self.ws_q8,
+                                out=self.y)
+
+
+def make_problems(cases, l2_bytes, rotate_factor=3.0, max_copies=64, force_copies=0):
+    import bitlinear_fwd_b200 as bl
+    wcache = {}
+    per_step = 0
+    staged = []
+    for c in cases:
+        key = (c.N, c.K, c.tags.get("shape"))
+        if key not in wcache:
+            packed, s_w, _ = bl.bitlinear_pack_weights(c.w().cuda())
+            wcache[key] = (packed, s_w)
+        b = c.bias()
+        staged.append((c, b))
+        per_step += c.N * c.K // 4
+    copies = int(min(max_copies, max(2, np.ceil(rotate_factor * l2_bytes / max(per_step, 1)))))
+    if force_copies:
+        copies = force_copies
+    probs = []
+    for c, b in staged:
+        packed, s_w = wcache[(c.N, c.K, c.tags.get("shape"))]
+        probs.append(Problem(c.M, c.N, c.K, c.x().cuda(), packed, s_w, None if b is None else b.cuda(), copies))
+    torch.cuda.synchronize()
+    return probs, copies
+
+
+def capture_steps(probs, copies, fn_name):
+    graphs = []
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for r in range(copies):
+            for p in probs:                       # warm call outside capture
+                getattr(p, fn_name)(r)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    for r in range(copies):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for p in probs:
+                getattr(p, fn_name)(r)
+        graphs.append(g)
+    torch.cuda.synchronize()
+    return graphs
+
+
+def timed_replays(graphs, steps, warmup, preroll_s=0.0):
+    for i in range(warmup):
+        graphs[i % len(graphs)].replay()
+    torch.cuda.synchronize()
+    if preroll_s > 0:
+        t0 = time.time()
+        i = 0
+        while time.time() - t0 < preroll_s:
+            graphs[i % len(graphs)].replay()
+            i += 1
+            if i % 64 == 0:
+                torch.cuda.synchronize()
+    sync_all()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(steps):
+        graphs[i % len(graphs)].replay()
+    e1.record()
+    e1.synchronize()
+    sync_all()
+    return elapsed_max_over_ranks(e0.elapsed_time(e1))
+
+
+def kernel_times(probs, copies, reps=20, fn="contract"):
+    """Mean duration (ms) of one isolated launch per problem, between CUDA
+    events on the launching stream, launches queued behind a sleep so that
+    the host does not pace them."""
+    out = []
+    for p in probs:
+        evs = []
+        torch.cuda._sleep(20_000_000)
+        for i in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            getattr(p, fn)(i % copies)
+            b.record()
+            evs.append((a, b))
+        torch.cuda.synchronize()
+        out.append(statistics.mean(a.elapsed_time(b) for a, b in evs[2:]))
+    return out
+
+
+def run_decode(args, hbm_gbs, l2_bytes, peak_kind):
+    """The decode forward is one kernel (quantisation, contraction, epilogue),
+    so the timed region is a back-to-back sequence of that kernel alone: its
+    average launch duration is the timed time over the launches, and its
+    algorithmic bytes are the forward's."""
+    cases = wl.workload2()
+    probs, copies = make_problems(cases, l2_bytes, force_copies=args.copies)
+    graphs = capture_steps(probs, copies, "forward")
+    bytes_step = sum(decode_bytes(p.M, p.N, p.K, p.bias is not None) for p in probs)
+    ms = timed_replays(graphs, args.steps, args.warmup, preroll_s=args.preroll)
+    world = torch.distributed.get_world_size() if torch.distributed.is_initialized() else 1
+    value = world * bytes_step * args.steps / (ms * 1e-3) / 1e9
+    launches = len(probs) * args.steps
+    achieved = bytes_step * args.steps / (ms * 1e-3) / 1e9          # this rank's kernel
+    kt = kernel_times(probs, copies, fn="forward")
+    per_case = [{"M": p.M, "N": p.N, "K": p.K, "isolated_us": round(t * 1e3, 3),
+                 "isolated_gbs": round(decode_bytes(p.M, p.N, p.K) / (t * 1e-3) / 1e9, 1)}
+                for p, t in zip(probs, kt)]
+    traffic = traffic_from_profile("decode_kernel_w2.md", "gemv_decode.cu")
+    roof = {"kernel": "decode_kernel", "bound": "hbm", "achieved": round(achieved, 1),
+            "peak": hbm_gbs, "unit": "GB/s", "frac": round(achieved / hbm_gbs, 4),
+            "peak_source": f"{peak_kind} HBM copy bandwidth (burst figure)",
+            "avg_launch_us": round(ms * 1e3 / launches, 3),
+            "algorithmic_bytes_per_launch_avg": round(bytes_step / len(probs)),
+            "traffic": traffic, "per_case_isolated_launch": per_case}
+    return {"value": value, "ms": ms, "bytes_step": bytes_step, "roofline": roof, "copies": copies,
+            "graphs": graphs, "probs": probs, "launches_per_step": len(probs)}
+
+
+def run_e2e(args, probs, steps):
+    import bitlinear_fwd_b200 as bl
+    xs = [p.x.cpu().pin_memory() for p in probs]
+    ys = [torch.empty((p.M, p.N), dtype=torch.bfloat16).pin_memory() for p in probs]
+    wss = [bl.workspace(p.M, p.N, p.K, "cuda", host=True) for p in probs]
+
+    def step(r):
+        for p, x, y, ws in zip(probs, xs, ys, wss):
+            bl.bitlinear_forward_host(x, p.packed[r % len(p.packed)], p.s_w, p.bias, y_host=y, ws=ws)
+
+    for i in range(3):
+        step(i)
+    sync_all()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(steps):
+        step(i)
+    e1.record()
+    e1.synchronize()
+    sync_all()
+    ms = elapsed_max_over_ranks(e0.elapsed_time(e1))
+    world = torch.distributed.get_world_size() if torch.distributed.is_initialized() else 1
+    bytes_step = sum(decode_bytes(p.M, p.N, p.K, p.bias is not None) for p in probs)
+    return {"value": round(world * bytes_step * steps / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "h2d_bytes_per_step": sum(2 * p.M * p.K for p in probs),
+            "d2h_bytes_per_step": sum(2 * p.M * p.N for p in probs),
+            "api": "bitlinear_forward_host (pinned host x in, host y out, synchronous per call)"}
+
+
+def run_prefill(args, bf16_tflops, peak_kind, l2_bytes):
+    cases = wl.workload3()
+    probs, copies = make_problems(cases, l2_bytes, rotate_factor=1.0, max_copies=3, force_copies=args.copies)
+    graphs = capture_steps(probs, copies, "forward")
+    ops_step = sum(2 * p.M * p.N * p.K for p in probs)
+    steps = max(3, args.prefill_steps)
+    ms = timed_replays(graphs, steps, max(3, args.warmup))
+    world = torch.distributed.get_world_size() if torch.distributed.is_initialized() else 1
+    tops = world * ops_step * steps / (ms * 1e-3) / 1e12
+    kt = kernel_times(probs, copies, reps=8)
+    ops = [2 * p.M * p.N * p.K for p in probs]
+    achieved = sum(ops) / (sum(kt) * 1e-3) / 1e12
+    peak = bf16_tflops * INT8_OVER_BF16
+    per_case = [{"M": p.M, "N": p.N, "K": p.K, "us": round(t * 1e3, 2),
+                 "tops": round(o / (t * 1e-3) / 1e12, 1)} for p, t, o in zip(probs, kt, ops)]
+    traffic = traffic_from_profile("gemm_prefill_w3.md", "gemm_prefill.cu")
+    del graphs
+    return {"metric": "BitLinear prefill int8 TOPS (bitlinear_forward incl. activation quantisation)",
+            "value": round(tops, 1), "unit": "TOPS", "ms_per_step": round(ms / steps, 4), "steps": steps,
+            "workload": "prefill: M in {512,2048,8192} x (K,N) in {(3200,8640),(8640,3200)}, x Student-t(4) "
+                        "bf16, W N(0,0.02) ternarised; 6 forwards per step",
+            "roofline": {"kernel": "gemm_prefill_kernel", "bound": "tensor", "achieved": round(achieved, 1),
+                         "peak": round(peak, 1), "unit": "TOPS", "frac": round(achieved / peak, 4),
+                         "peak_source": f"{peak_kind} bf16 dense x {INT8_OVER_BF16:g} (nominal int8/bf16)",
+                         "traffic": traffic, "per_case": per_case}}
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle (cpu_baseline and the reference arm)
+# ---------------------------------------------------------------------------
+
+class OracleDecode:
+    """The CPU oracle on the decode workload (all six problems, every weight
+    row).  Inputs are generated and packed by the oracle once, untimed."""
+
+    def __init__(self):
+        import oracle
+        self.oracle = oracle
+        try:
+            from threadpoolctl import threadpool_info
+            self.blas = max([i.get("num_threads", 1) for i in threadpool_info()
+                             if i.get("user_api") == "blas"] or [1])
+        except Exception:
+            self.blas = 1
+        wcache = {}
+        self.items = []
+        for c in wl.workload2():
+            key = (c.N, c.K)
+            if key not in wcache:
+                wcache[key] = oracle.pack_weights(c.w().numpy())
+            packed, s_w, _ = wcache[key]
+            self.items.append((synth.bf16_bits(c.x()), packed, s_w, synth.bf16_bits(c.bias()),
+                               decode_bytes(c.M, c.N, c.K)))
+        self.desc = ("oracle.forward (act quant, unpack, exact contraction, epilogue) on the 6 decode problems "
+                     "with every weight row, packing untimed; numpy elementwise steps single-threaded, "
+                     f"float64 matmul on {self.blas} BLAS threads")
+
+    def step(self):
+        """One pass over the workload; returns (bytes, seconds)."""
+        b, s = 0, 0.0
+        for xb, packed, s_w, bb, nbytes in self.items:
+            t0 = time.perf_counter()
+            self.oracle.forward(xb, packed, s_w, bb)
+            s += time.perf_counter() - t0
+            b += nbytes
+        return b, s
+
+
+def reference_arm(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    od = OracleDecode()
+    od.step()                                       # warm-up (page-in, BLAS threads)
+    steps = max(1, min(args.steps, 8))
+    b, s = 0, 0.0
+    for _ in range(steps):
+        bb, ss = od.step()
+        b += bb
+        s += ss
+    v = b / s / 1e9
+    line = {"impl": "reference", "metric": "BitLinear decode GB/s (% of HBM peak); prefill int8 TOPS (% TC peak)",
+            "value": round(v, 4), "unit": "GB/s",
+            "n_gpus": args.gpus, "steps": steps, "warmup": 1, "ms_per_step": round(1e3 * s / steps, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32/int64 (numpy)",
+            "data": "synthetic",
+            "config": {"workload": "decode GEMV sweep: M in {1,4,16}, (K,N) in {(4096,4096),(4096,11008)}; "
+                                   "the CPU oracle, the only reference implementation of this method",
+                       "parallelism": "rank 0 host cores"},
+            "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": od.blas, "kind": "oracle",
+                             "sample": f"{steps} passes of " + od.desc},
+            "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--preroll", type=float, default=1.0, help="seconds of untimed replays before timing")
+    ap.add_argument("--prefill-steps", type=int, default=20)
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--only", choices=["decode", "prefill"], default=None,
+                    help="run one workload only (profiling runs; no JSON contract line)")
+    ap.add_argument("--copies", type=int, default=0, help="force the number of rotating weight copies")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    if args.impl == "reference":
+        return reference_arm(args)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    import bitlinear_fwd_b200 as bl
+    bl.lib()
+    hbm_gbs, bf16_tflops, peak_kind = peaks()
+    l2_bytes = torch.cuda.get_device_properties(local).L2_cache_size
+
+    if args.only == "prefill":
+        print(json.dumps(run_prefill(args, bf16_tflops, peak_kind, l2_bytes)), flush=True)
+        return 0
+    if args.only == "decode":
+        d = run_decode(args, hbm_gbs, l2_bytes, peak_kind)
+        print(json.dumps({"value": d["value"], "ms": d["ms"], "roofline": d["roofline"]}), flush=True)
+        return 0
+    sampler = ClockSampler(local)
+    dec = run_decode(args, hbm_gbs, l2_bytes, peak_kind)
+    clocks = sampler.stop()
+    e2e = None if args.no_e2e else run_e2e(args, dec["probs"], max(3, min(200, args.steps // 10)))
+    pre = None if args.no_prefill else run_prefill(args, bf16_tflops, peak_kind, l2_bytes)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        od = OracleDecode()
+        b, s, n = 0, 0.0, 0
+        while s < 10.0 and n < 8:
+            bb, ss = od.step()
+            b, s, n = b + bb, s + ss, n + 1
+        cpu = {"value": round(b / s / 1e9, 4), "unit": "GB/s", "cores": od.blas, "kind": "oracle",
+               "sample": f"{n} passes ({s:.1f} s) of " + od.desc}
+
+    line = {
+        "metric": "BitLinear decode GB/s (% of HBM peak); prefill int8 TOPS (% TC peak)",
+        "value": round(dec["value"], 1),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(dec["ms"] / args.steps, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int8",
+        "data": "synthetic",
+        "config": {"workload": "decode GEMV sweep: M in {1,4,16}, (K,N) in {(4096,4096),(4096,11008)}, "
+                               "x N(0,1) bf16 with 1% channels x20, W N(0,0.02) ternarised + 2-bit packed, "
+                               "bias N(0,0.01); 6 bitlinear_forward calls per step",
+                   "global_batch": 21 * world, "parallelism": f"dp{world} replicas (no collective)",
+                   "l2": f"inputs larger than L2: {dec['copies']} rotating packed-weight copies, "
+                         f"{dec['copies'] * sum(p.N * p.K // 4 for p in dec['probs']) / 1e6:.0f} MB vs "
+                         f"{l2_bytes / 1e6:.0f} MB L2",
+                   "bytes_per_step": dec["bytes_step"], "graph_replay": True},
+        "roofline": dec["roofline"],
+        "gpu_launches": dec["launches_per_step"] * args.steps,
+        "e2e": e2e,
+        "prefill": pre,
+        "cpu_baseline": cpu,
+        "clocks": clocks,
+    }
+    del dec
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

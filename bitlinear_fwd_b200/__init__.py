@@ -33,6 +33,8 @@ _SIGS = {
     "bitlinear_quant_act": (ctypes.c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_p, _c_p, _c_p]),
     "bitlinear_forward": (ctypes.c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_i64, _c_p, _c_p, _c_p, _c_p, _c_sz,
                                          _c_p]),
+    "bitlinear_forward_ex": (ctypes.c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_i64, _c_p, _c_p, _c_p, ctypes.c_uint,
+                                            _c_p, _c_sz, _c_p]),
     "bitlinear_forward_q8": (ctypes.c_int, [_c_p, _c_p, _c_p, _c_i64, _c_i64, _c_p, _c_i64, _c_p, _c_p, _c_p,
                                             _c_p, _c_sz, _c_p]),
     "bitlinear_forward_debug": (ctypes.c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_i64, _c_p, _c_p, _c_p, _c_p,
@@ -145,10 +147,14 @@ def bitlinear_quant_act(x: torch.Tensor):
     return xq, s_x, rs
 
 
+WEIGHTS_RESIDENT = 1
+
+
 def bitlinear_forward(x: torch.Tensor, packed: torch.Tensor, w_scale: torch.Tensor,
                       bias: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
-                      out: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """BitLinear.forward: y bf16 [M, N] from x bf16 [M, K] and packed weights."""
+                      out: Optional[torch.Tensor] = None, flags: int = 0) -> torch.Tensor:
+    """BitLinear.forward: y bf16 [M, N] from x bf16 [M, K] and packed weights.
+    flags=WEIGHTS_RESIDENT calls bitlinear_forward_ex (see the C header)."""
     x = _bits(x)
     M, K = x.shape
     N = packed.shape[0]
@@ -156,8 +162,13 @@ def bitlinear_forward(x: torch.Tensor, packed: torch.Tensor, w_scale: torch.Tens
     if ws is None:
         ws = workspace(M, N, K, x.device)
     b = None if bias is None else _bits(bias)
-    _check(lib().bitlinear_forward(_ptr(x), M, K, _ptr(packed), N, _ptr(w_scale), _ptr(b), _ptr(y), _ptr(ws),
-                                   ws.numel(), _stream(x.device)), "bitlinear_forward")
+    if flags:
+        st = lib().bitlinear_forward_ex(_ptr(x), M, K, _ptr(packed), N, _ptr(w_scale), _ptr(b), _ptr(y), flags,
+                                        _ptr(ws), ws.numel(), _stream(x.device))
+        _check(st, "bitlinear_forward_ex")
+    else:
+        _check(lib().bitlinear_forward(_ptr(x), M, K, _ptr(packed), N, _ptr(w_scale), _ptr(b), _ptr(y),
+                                       _ptr(ws), ws.numel(), _stream(x.device)), "bitlinear_forward")
     return y
 
 

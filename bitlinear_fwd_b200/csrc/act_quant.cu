@@ -75,6 +75,7 @@ __global__ void __launch_bounds__(kThreads) act_quant_kernel(const uint16_t* __r
                                                              int32_t* __restrict__ rowsum,
                                                              uint32_t* status_clear) {
   pdl_launch_dependents();
+  pdl_wait_primary();
   if (status_clear && blockIdx.x == 0 && threadIdx.x == 0) *status_clear = 0u;
   __shared__ uint32_t red[kThreads / 32];
 
@@ -140,22 +141,31 @@ __global__ void __launch_bounds__(kThreads) act_quant_kernel(const uint16_t* __r
 
 }  // namespace
 
+template <int CPT>
+cudaError_t launch_cpt(const uint16_t* x, int M, int K, int8_t* xq, float* s_x, int32_t* rowsum,
+                       uint32_t* status_clear, bool pdl, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(M, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, act_quant_kernel<CPT>, x, K, xq, s_x, rowsum, status_clear);
+}
+
 cudaError_t launch_act_quant(const uint16_t* x, int M, int K, int8_t* xq, float* s_x,
-                             int32_t* rowsum, uint32_t* status_clear, cudaStream_t stream) {
+                             int32_t* rowsum, uint32_t* status_clear, bool pdl, cudaStream_t stream) {
   if (M <= 0) return cudaSuccess;
   const int chunks = K / 16;
-  const dim3 grid(M), block(kThreads);
-  if (chunks <= kThreads)
-    act_quant_kernel<1><<<grid, block, 0, stream>>>(x, K, xq, s_x, rowsum, status_clear);
-  else if (chunks <= 2 * kThreads)
-    act_quant_kernel<2><<<grid, block, 0, stream>>>(x, K, xq, s_x, rowsum, status_clear);
-  else if (chunks <= 4 * kThreads)
-    act_quant_kernel<4><<<grid, block, 0, stream>>>(x, K, xq, s_x, rowsum, status_clear);
-  else if (chunks <= 8 * kThreads)
-    act_quant_kernel<8><<<grid, block, 0, stream>>>(x, K, xq, s_x, rowsum, status_clear);
-  else
-    act_quant_kernel<0><<<grid, block, 0, stream>>>(x, K, xq, s_x, rowsum, status_clear);
-  return cudaGetLastError();
+  if (chunks <= kThreads) return launch_cpt<1>(x, M, K, xq, s_x, rowsum, status_clear, pdl, stream);
+  if (chunks <= 2 * kThreads) return launch_cpt<2>(x, M, K, xq, s_x, rowsum, status_clear, pdl, stream);
+  if (chunks <= 4 * kThreads) return launch_cpt<4>(x, M, K, xq, s_x, rowsum, status_clear, pdl, stream);
+  if (chunks <= 8 * kThreads) return launch_cpt<8>(x, M, K, xq, s_x, rowsum, status_clear, pdl, stream);
+  return launch_cpt<0>(x, M, K, xq, s_x, rowsum, status_clear, pdl, stream);
 }
 
 }  // namespace bitlinear

@@ -68,23 +68,53 @@ int check_shape(int64_t M, int64_t N, int64_t K) {
 int status_of(cudaError_t e) { return e == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA; }
 
 // Shared body of the forward entry points; x is a device pointer.
+//
+// Decode (M <= 16) is one kernel that quantises x itself.  Prefill is the
+// act-quant kernel followed by the tcgen05 GEMM, launched as its
+// programmatic dependent so that its launch and weight loads overlap the
+// act-quant kernel.  The first kernel is an ordinary stream launch -- every
+// earlier write to the packed weights is complete before they are read --
+// unless BITLINEAR_WEIGHTS_RESIDENT is set, which lets the forward start
+// streaming weights while the previous kernel on the stream finishes.
 int forward_impl(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed_w, int64_t N,
                  const float* w_scale, const uint16_t* bias, uint16_t* y, int8_t* xq_out, float* sx_out,
-                 int32_t* acc_out, float* y32_out, int engine, void* ws, size_t ws_bytes,
+                 int32_t* acc_out, float* y32_out, int engine, unsigned flags, void* ws, size_t ws_bytes,
                  cudaStream_t stream) {
+  (void)ws_bytes;
   int sms = 148;
   int st = check_device(&sms);
   if (st != BITLINEAR_OK) return st;
   const FwdLayout L = fwd_layout(M, N, K);
   char* base = static_cast<char*>(ws);
   uint32_t* status = reinterpret_cast<uint32_t*>(base);
+  const bool resident = (flags & BITLINEAR_WEIGHTS_RESIDENT) != 0;
+  const bool decode = engine == 1 || (engine == 0 && M <= 16);
+  cudaError_t e;
+  if (decode) {
+    DecodeArgs d;
+    d.x = x;
+    d.xq = nullptr;
+    d.s_x = nullptr;
+    d.packed = packed_w;
+    d.w_scale = w_scale;
+    d.bias = bias;
+    d.y = y;
+    d.xq_out = xq_out;
+    d.sx_out = sx_out;
+    d.acc_out = acc_out;
+    d.y32_out = y32_out;
+    d.status = status;
+    d.M = int(M);
+    d.N = int(N);
+    d.K = int(K);
+    d.weights_early = resident ? 1 : 0;
+    return status_of(launch_decode(d, sms, stream));
+  }
   float* s_x = reinterpret_cast<float*>(base + L.off_sx);
   int32_t* rowsum = reinterpret_cast<int32_t*>(base + L.off_rs);
   int8_t* xq = reinterpret_cast<int8_t*>(base + L.off_xq);
-
-  cudaError_t e = launch_act_quant(x, int(M), int(K), xq, s_x, rowsum, status, stream);
+  e = launch_act_quant(x, int(M), int(K), xq, s_x, rowsum, status, resident, stream);
   if (e != cudaSuccess) return BITLINEAR_ERR_CUDA;
-
   ForwardArgs a;
   a.xq = xq;
   a.s_x = s_x;
@@ -100,8 +130,7 @@ int forward_impl(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed_
   a.N = int(N);
   a.K = int(K);
   a.pdl = true;
-  const bool decode = engine == 1 || (engine == 0 && M <= 16);
-  e = decode ? launch_gemv_decode(a, sms, stream) : launch_gemm_prefill(a, sms, stream);
+  e = launch_gemm_prefill(a, sms, stream);
   if (e != cudaSuccess) return BITLINEAR_ERR_CUDA;
   if (xq_out) e = cudaMemcpyAsync(xq_out, xq, size_t(M) * size_t(K), cudaMemcpyDeviceToDevice, stream);
   if (e == cudaSuccess && sx_out) e = cudaMemcpyAsync(sx_out, s_x, 4 * size_t(M), cudaMemcpyDeviceToDevice, stream);
@@ -187,7 +216,7 @@ int bitlinear_quant_act(const uint16_t* x, int64_t M, int64_t K, int8_t* xq, flo
     return BITLINEAR_ERR_ALIGN;
   int st = check_device(nullptr);
   if (st != BITLINEAR_OK) return st;
-  return status_of(launch_act_quant(x, int(M), int(K), xq, x_scale, xq_rowsum, nullptr,
+  return status_of(launch_act_quant(x, int(M), int(K), xq, x_scale, xq_rowsum, nullptr, false,
                                     static_cast<cudaStream_t>(stream)));
 }
 
@@ -198,7 +227,19 @@ int bitlinear_forward(const uint16_t* x, int64_t M, int64_t K, const uint8_t* pa
                               bitlinear_workspace_bytes(M, N, K), false);
   if (st != BITLINEAR_OK) return st;
   if (M == 0) return BITLINEAR_OK;
-  return forward_impl(x, M, K, packed_w, N, w_scale, bias, y, nullptr, nullptr, nullptr, nullptr, 0, ws,
+  return forward_impl(x, M, K, packed_w, N, w_scale, bias, y, nullptr, nullptr, nullptr, nullptr, 0, 0u, ws,
+                      ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int bitlinear_forward_ex(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed_w, int64_t N,
+                         const float* w_scale, const uint16_t* bias, uint16_t* y, unsigned flags, void* ws,
+                         size_t ws_bytes, void* stream) {
+  if (flags & ~static_cast<unsigned>(BITLINEAR_WEIGHTS_RESIDENT)) return BITLINEAR_ERR_SHAPE;
+  int st = check_forward_args(x, M, K, packed_w, N, w_scale, bias, y, ws, ws_bytes,
+                              bitlinear_workspace_bytes(M, N, K), false);
+  if (st != BITLINEAR_OK) return st;
+  if (M == 0) return BITLINEAR_OK;
+  return forward_impl(x, M, K, packed_w, N, w_scale, bias, y, nullptr, nullptr, nullptr, nullptr, 0, flags, ws,
                       ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
@@ -233,7 +274,27 @@ int bitlinear_forward_q8(const int8_t* xq, const float* x_scale, const int32_t* 
   a.K = int(K);
   a.pdl = false;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return status_of(M <= 16 ? launch_gemv_decode(a, sms, s) : launch_gemm_prefill(a, sms, s));
+  if (M > 16) return status_of(launch_gemm_prefill(a, sms, s));
+  // the previous operation on the stream is unknown: read the weights only
+  // after the dependency wait
+  DecodeArgs d;
+  d.x = nullptr;
+  d.xq = xq;
+  d.s_x = x_scale;
+  d.packed = packed_w;
+  d.w_scale = w_scale;
+  d.bias = bias;
+  d.y = y;
+  d.xq_out = nullptr;
+  d.sx_out = nullptr;
+  d.acc_out = nullptr;
+  d.y32_out = nullptr;
+  d.status = a.status;
+  d.M = int(M);
+  d.N = int(N);
+  d.K = int(K);
+  d.weights_early = 0;
+  return status_of(launch_decode(d, sms, s));
 }
 
 int bitlinear_forward_debug(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed_w, int64_t N,
@@ -246,7 +307,7 @@ int bitlinear_forward_debug(const uint16_t* x, int64_t M, int64_t K, const uint8
   if (engine < 0 || engine > 2 || (engine == 1 && M > 16)) return BITLINEAR_ERR_SHAPE;
   if (misaligned(xq) || misaligned(x_scale) || misaligned(acc) || misaligned(y32)) return BITLINEAR_ERR_ALIGN;
   if (M == 0) return BITLINEAR_OK;
-  return forward_impl(x, M, K, packed_w, N, w_scale, bias, y, xq, x_scale, acc, y32, engine, ws, ws_bytes,
+  return forward_impl(x, M, K, packed_w, N, w_scale, bias, y, xq, x_scale, acc, y32, engine, 0u, ws, ws_bytes,
                       static_cast<cudaStream_t>(stream));
 }
 
@@ -264,7 +325,7 @@ int bitlinear_forward_host(const uint16_t* x_host, int64_t M, int64_t K, const u
   uint16_t* yd = reinterpret_cast<uint16_t*>(base + L.off_yh);
   if (cudaMemcpyAsync(xd, x_host, 2 * size_t(M) * size_t(K), cudaMemcpyHostToDevice, s) != cudaSuccess)
     return BITLINEAR_ERR_CUDA;
-  st = forward_impl(xd, M, K, packed_w, N, w_scale, bias, yd, nullptr, nullptr, nullptr, nullptr, 0, ws,
+  st = forward_impl(xd, M, K, packed_w, N, w_scale, bias, yd, nullptr, nullptr, nullptr, nullptr, 0, 0u, ws,
                     ws_bytes, s);
   if (st != BITLINEAR_OK) return st;
   if (cudaMemcpyAsync(y_host, yd, 2 * size_t(M) * size_t(N), cudaMemcpyDeviceToHost, s) != cudaSuccess)

@@ -9,9 +9,15 @@
 
 namespace bitlinear {
 
+// ---- TMA tensor maps (tensor_map.cu) ---------------------------------------
+bool encode_2d_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                  uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle);
+
 // ---- activation quantisation (act_quant.cu) --------------------------------
+// pdl: launch as a programmatic dependent of the previous kernel on the stream
+// (the kernel waits for it before touching memory).
 cudaError_t launch_act_quant(const uint16_t* x, int M, int K, int8_t* xq, float* s_x,
-                             int32_t* rowsum, uint32_t* status_clear, cudaStream_t stream);
+                             int32_t* rowsum, uint32_t* status_clear, bool pdl, cudaStream_t stream);
 
 // ---- weight absmean + ternarise + pack (pack.cu) ----------------------------
 // Workspace layout used by the pack kernels.
@@ -42,7 +48,29 @@ struct ForwardArgs {
 };
 
 // ---- decode engine, M <= 16 (gemv_decode.cu) --------------------------------
-cudaError_t launch_gemv_decode(const ForwardArgs& a, int num_sms, cudaStream_t stream);
+struct DecodeArgs {
+  const uint16_t* x;      // bf16 [M, K], quantised inside the kernel; or null
+  const int8_t* xq;       // int8 [M, K] with s_x when x is null
+  const float* s_x;       // [M]
+  const uint8_t* packed;  // [N, K/4]
+  const float* w_scale;   // [1]
+  const uint16_t* bias;   // [N] or null
+  uint16_t* y;            // [M, N]
+  int8_t* xq_out;         // [M, K] or null (debug, fused path)
+  float* sx_out;          // [M] or null (debug, fused path)
+  int32_t* acc_out;       // [M, N] or null (debug)
+  float* y32_out;         // [M, N] or null (debug)
+  uint32_t* status;       // status word or null
+  int M, N, K;
+  int boxes_per_cta, ring, xs_stride;   // set by launch_decode
+  int weights_early;      // the packed weights may be read before the dependency wait
+};
+struct DecodePlan {
+  int cluster, boxes_per_cta, ring, row_blocks;
+  size_t smem;
+};
+DecodePlan plan_decode(int M, int N, int K, int num_sms);
+cudaError_t launch_decode(DecodeArgs a, int num_sms, cudaStream_t stream);
 
 // ---- prefill engine, tcgen05 GEMM (gemm_prefill.cu) -------------------------
 cudaError_t launch_gemm_prefill(const ForwardArgs& a, int num_sms, cudaStream_t stream);

@@ -125,12 +125,27 @@ int bitlinear_quant_act(const uint16_t* x, int64_t M, int64_t K, int8_t* xq, flo
  *   y         [M, N] bf16 out
  *   ws        workspace of at least bitlinear_workspace_bytes(M, N, K);
  *             its contents on entry do not matter
- * M <= 16 runs the decode engine (weight-streaming GEMV on warp-level int8
- * MMA), M > 16 the prefill engine (tcgen05 int8 GEMM with accumulators in
- * tensor memory).  Both quantise x first (one extra kernel). */
+ * M <= 16 runs the decode engine: one kernel that quantises x, streams
+ * the packed weights through warp-level int8 MMA and applies the epilogue.
+ * M > 16 runs the prefill engine: an activation-quantisation kernel, then a
+ * tcgen05 int8 GEMM with accumulators in tensor memory and the epilogue. */
 int bitlinear_forward(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed_w,
                       int64_t N, const float* w_scale, const uint16_t* bias, uint16_t* y,
                       void* ws, size_t ws_bytes, void* stream);
+
+/* Flags of bitlinear_forward_ex. */
+#define BITLINEAR_WEIGHTS_RESIDENT 1u
+/*   packed_w (and w_scale) were completely written before the operation
+ *   enqueued on `stream` just ahead of this call started -- e.g. weights
+ *   packed once at load time.  The decode engine may then start streaming
+ *   the weights while that operation is still finishing (programmatic
+ *   dependent launch), which overlaps consecutive layers.  Never set it when
+ *   the previous operation on the stream writes packed_w or w_scale. */
+
+/* bitlinear_forward with flags (0 = identical to bitlinear_forward). */
+int bitlinear_forward_ex(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed_w, int64_t N,
+                         const float* w_scale, const uint16_t* bias, uint16_t* y, unsigned flags, void* ws,
+                         size_t ws_bytes, void* stream);
 
 /* The contraction and epilogue of the forward on activations that
  * bitlinear_quant_act has already quantised (so that several weight

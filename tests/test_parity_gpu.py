@@ -190,3 +190,17 @@ def test_device_argument_errors():
     assert lib.bitlinear_forward(x.data_ptr(), 4, 128, packed.data_ptr(), 64, s_w.data_ptr(), None,
                                  y.data_ptr(), ws.data_ptr(), ws.numel(), st) == 0
     assert bl.bitlinear_check_status(ws) == 0
+
+
+def test_forward_ex_resident_flag_matches():
+    """Weights packed earlier on the stream, then a chain of forwards with the
+    resident-weights flag (weights streamed before the dependency wait)."""
+    c = _W2[1]
+    w, b = c.w().cuda(), c.bias().cuda()
+    packed, s_w, _ = bl.bitlinear_pack_weights(w)
+    torch.cuda.synchronize()
+    xs = [synth.normal_bf16(82, i, (c.M, c.K)).cuda() for i in range(4)]
+    want = [bl.bitlinear_forward(x, packed, s_w, b).cpu() for x in xs]
+    got = [bl.bitlinear_forward(x, packed, s_w, b, flags=bl.WEIGHTS_RESIDENT) for x in xs]
+    for g_, w_ in zip(got, want):
+        assert torch.equal(g_.cpu().view(torch.int16), w_.view(torch.int16))
