@@ -42,6 +42,7 @@ _SIGS = {
     "bitlinear_forward_host": (ctypes.c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_i64, _c_p, _c_p, _c_p, _c_p,
                                               _c_sz, _c_p]),
     "bitlinear_check_status": (ctypes.c_int, [_c_p, _c_sz, _c_p]),
+    "bitlinear_forward_noalloc": (ctypes.c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_i64, _c_p, _c_p, _c_p, _c_p]),
 }
 
 _lib = None
@@ -227,6 +228,20 @@ def bitlinear_forward_host(x_host: torch.Tensor, packed: torch.Tensor, w_scale: 
                                         _ptr(y_host), _ptr(ws), ws.numel(), _stream(dev)),
            "bitlinear_forward_host")
     return y_host
+
+
+def bitlinear_forward_noalloc(x: torch.Tensor, packed: torch.Tensor, w_scale: torch.Tensor,
+                              bias: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """bitlinear_forward with the library's fixed device scratch instead of a
+    workspace (for callers that cannot allocate; see the C header)."""
+    x = _bits(x)
+    M, K = x.shape
+    N = packed.shape[0]
+    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    b = None if bias is None else _bits(bias)
+    _check(lib().bitlinear_forward_noalloc(_ptr(x), M, K, _ptr(packed), N, _ptr(w_scale), _ptr(b), _ptr(y),
+                                           _stream(x.device)), "bitlinear_forward_noalloc")
+    return y
 
 
 def bitlinear_check_status(ws: torch.Tensor) -> int:

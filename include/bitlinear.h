@@ -179,6 +179,27 @@ int bitlinear_forward_host(const uint16_t* x_host, int64_t M, int64_t K, const u
                            int64_t N, const float* w_scale, const uint16_t* bias,
                            uint16_t* y_host, void* ws, size_t ws_bytes, void* stream);
 
+/* bitlinear_forward for callers that cannot allocate device memory (code
+ * running inside someone else's CUDA-graph capture, server plugins given no
+ * allocator, paths that must never allocate).  It takes no workspace: the
+ * library uses one fixed device array of BITLINEAR_NOALLOC_SCRATCH_BYTES
+ * bytes, held by every GPU that loads the library until the process exits.
+ * The paper has no counterpart to this entry point.
+ *   - Returns BITLINEAR_ERR_WORKSPACE when bitlinear_workspace_bytes(M, N, K)
+ *     exceeds that fixed size (roughly M * K <= 16 MiB), and
+ *     BITLINEAR_ERR_SHAPE for an invalid shape; other arguments and errors
+ *     as for bitlinear_forward.
+ *   - All calls share the array: calls that overlap on the GPU (on
+ *     different streams or from racing host threads) race and corrupt each
+ *     other.  Serialise them, e.g. on one stream.
+ *   - The first call on a device looks up the array's device address on that
+ *     device (make the device current first); make that first call before
+ *     any stream capture.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call. */
+#define BITLINEAR_NOALLOC_SCRATCH_BYTES (16u << 20)
+int bitlinear_forward_noalloc(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed_w, int64_t N,
+                              const float* w_scale, const uint16_t* bias, uint16_t* y, void* stream);
+
 /* Reads and clears the status word of a workspace (synchronises
  * `stream`).  bitlinear_pack_weights, bitlinear_forward, _debug and _host
  * reset the word when they start; bitlinear_forward_q8 does not.  Returns
