@@ -3,57 +3,78 @@
 // universal models": F.linear, then post_quant_process and the bias add) as
 // a dense int8 GEMM on the 5th-generation tensor cores.
 //
-// Tile: 128 tokens x 256 weight rows, k-blocks of 128; one CTA per tile.
-//   warp 0      TMA producer: x_q tile (128 x 128 int8, 128-byte swizzle) and
-//               the packed weight tile (256 rows x 32 bytes) per k-block
-//   warp 1      MMA issuer: 4 x tcgen05.mma.kind::i8 (M=128, N=256, K=32)
-//               per k-block into a 128 x 256 int32 accumulator in tensor memory
-//   warp 2      tensor-memory allocation
-//   warps 4..7  unpack each packed tile into the K-major, 128-byte-swizzled
-//               int8 operand (one 32-bit word -> one 16-byte chunk of codes
-//               c = u + 1 in {0,1,2}); after the last k-block, the epilogue:
-//               tcgen05.ld of the accumulator, acc - sum_k q (removes the code
-//               offset), y = acc / (s_x * s_w) (+ bias), bf16 stores.
-// A 4-stage ring of (x tile, packed tile, unpacked tile) with three mbarriers
-// per stage: full (TMA bytes landed), ready (unpacked), empty (MMAs done).
-// Out-of-range rows/columns of a tile are zero-filled by TMA, so a code 0
-// or an activation 0 adds nothing; the epilogue masks rows >= M, cols >= N.
-// Every wait is bounded in time; a wait that gives up sets the status word,
-// and the CTA still drains its copies and MMAs before freeing tensor memory.
+// The weights are the MMA's A operand and come from tensor memory; the
+// tokens are the B operand and come from shared memory:
+//   D[weight row n][token m] += A[n][k] * B[m][k],  M_mma = 128 weight rows,
+//   N_mma = 128 tokens, K = 32 per instruction.
+// Persistent kernel: one CTA per SM walks the 128 x 128 tiles
+// (weight tile fastest, so the CTAs running at the same time share the
+// token tile in L2), k-blocks of 128, with a 6-stage operand ring and a
+// double-buffered accumulator in tensor memory:
+//   warp 0       TMA producer: x tile (128 tokens x 128 int8, 128-byte
+//                swizzle) + packed weight tile (128 rows x 32 bytes) per stage
+//   warp 1       MMA issuer: 4 x tcgen05.mma.kind::i8 per k-block, A from
+//                tensor memory, into accumulator buffer (tile & 1)
+//   warp 2       tensor-memory allocation
+//   warps 4..7   weight unpack: thread = weight row; its 32 packed bytes become
+//                32 registers of codes c = u + 1 (one word -> four registers
+//                of four consecutive k) and one tcgen05.st of 32 columns
+//   warps 8..11  epilogue of the previous tile while the MMAs of the next one
+//                run: tcgen05.ld of a row's 128 accumulators, acc - sum_k q
+//                (code offset), y = acc / (s_x s_w) (+ bias), bf16 stores
+//                (coalesced along weight rows)
+// Barriers: per stage full (TMA bytes landed), ready (A stage written),
+// empty (MMAs done); per accumulator buffer acc_full (tile's MMAs done) and
+// acc_empty (epilogue has read it).  Shared memory carries only x and the
+// 2-bit codes.  Out-of-range rows/columns are zero-filled by TMA, so a code
+// 0 or an activation 0 adds nothing; the epilogue masks rows >= N and
+// tokens >= M.  Every wait is bounded in time; a wait that gives up sets the
+// status word, and the CTA drains its copies and MMAs before freeing tensor
+// memory.
 #include "kernels.h"
 
 namespace bitlinear {
 
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 128, STAGES = 4;
-constexpr int kThreads = 256;
-constexpr uint32_t kABytes = BM * BK;          // 16 KB
-constexpr uint32_t kBuBytes = BN * BK;         // 32 KB
-constexpr uint32_t kBpBytes = BN * BK / 4;     // 8 KB
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kOffA = 0;
-constexpr uint32_t kOffBu = kOffA + STAGES * kABytes;
-constexpr uint32_t kOffBp = kOffBu + STAGES * kBuBytes;
-constexpr uint32_t kOffBar = kOffBp + STAGES * kBpBytes;
-constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;   // barriers + alignment slack
+constexpr int BW = 128;                      // weight rows per tile (MMA M)
+constexpr int BT = 128;                      // tokens per tile (MMA N)
+constexpr int BK = 128;                      // k per block
+constexpr int STAGES = 6;
+constexpr int kThreads = 384;
+constexpr uint32_t kXBytes = BT * BK;        // 16 KB x tile per stage
+constexpr uint32_t kWpBytes = BW * BK / 4;   // 4 KB packed weights per stage
+constexpr uint32_t kACols = BK / 4;          // tensor-memory columns of one A stage
+constexpr uint32_t kTmemCols = 512;          // 2 x 128 accumulator + 6 x 32 A
 constexpr uint32_t kCodeMask = 0x03030303u;
+
+constexpr uint32_t kOffX = 0;
+constexpr uint32_t kOffWp = kOffX + STAGES * kXBytes;
+constexpr uint32_t kOffD = kOffWp + STAGES * kWpBytes;       // s_x * s_w per token [BT]
+constexpr uint32_t kOffRs = kOffD + 4 * BT;                  // row sums per token [BT]
+constexpr uint32_t kOffBar = kOffRs + 4 * BT;
+constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;        // + barriers, alignment slack
 
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_prefill_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                         const ForwardArgs a, uint64_t wait_ns) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint64_t* ready = full + STAGES;
   uint64_t* empty = ready + STAGES;
-  uint64_t* accum = empty + STAGES;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
+  uint64_t* acc_full = empty + STAGES;        // [2]
+  uint64_t* acc_empty = acc_full + 2;         // [2]
+  uint64_t* drain = acc_empty + 2;            // every issued MMA has completed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* failed = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* d_s = reinterpret_cast<float*>(smem + kOffD);
+  int* rs_s = reinterpret_cast<int*>(smem + kOffRs);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
   const int num_kb = (a.K + BK - 1) / BK;
+  const int wtiles = (a.N + BW - 1) / BW;
+  const int ntiles = wtiles * ((a.M + BT - 1) / BT);
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -61,7 +82,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&ready[s], 4);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(accum, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 4);
+    }
+    mbar_init(drain, 1);
     *failed = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_x);
@@ -75,126 +100,159 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  const uint32_t tmem_a = tmem_base + 2 * BT;     // A stages after the two accumulators
 
   if (warp == 0) {
     if (lane == 0) {
       // ---------------- TMA producer ----------------
-      int kb = 0;
-      for (; kb < num_kb; ++kb) {
-        const int s = kb % STAGES, round = kb / STAGES;
-        if (round > 0 && !mbar_wait(&empty[s], (round - 1) & 1, wait_ns)) {
-          *failed = 1;
-          break;
+      int g = 0;                                  // k-blocks issued by this CTA
+      bool waited = false;
+      for (int tile = blockIdx.x; tile < ntiles && !*failed; tile += gridDim.x) {
+        const int n0 = (tile % wtiles) * BW, m0 = (tile / wtiles) * BT;
+        for (int kb = 0; kb < num_kb; ++kb, ++g) {
+          const int s = g % STAGES, round = g / STAGES;
+          if (round > 0 && !mbar_wait(&empty[s], (round - 1) & 1, wait_ns)) {
+            *failed = 1;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[s], kXBytes + kWpBytes);
+          // packed weights do not depend on the activation kernel
+          tma_load_2d(smem + kOffWp + s * kWpBytes, &tm_w, &full[s], kb * (BK / 4), n0);
+          if (!waited) {
+            pdl_wait_primary();
+            waited = true;
+          }
+          tma_load_2d(smem + kOffX + s * kXBytes, &tm_x, &full[s], kb * BK, m0);
         }
-        mbar_arrive_expect_tx(&full[s], kABytes + kBpBytes);
-        // packed weights do not depend on the activation kernel
-        tma_load_2d(smem + kOffBp + s * kBpBytes, &tm_w, &full[s], kb * (BK / 4), n0);
-        if (kb == 0) pdl_wait_primary();
-        tma_load_2d(smem + kOffA + s * kABytes, &tm_x, &full[s], kb * BK, m0);
       }
       // drain: the last copy issued into each stage has landed
       for (int s = 0; s < STAGES; ++s) {
-        const int cnt = kb > s ? (kb - 1 - s) / STAGES + 1 : 0;   // copies issued into stage s
+        const int cnt = g > s ? (g - 1 - s) / STAGES + 1 : 0;
         if (cnt > 0 && !mbar_wait(&full[s], (cnt - 1) & 1, wait_ns)) *failed = 1;
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- MMA issuer ----------------
-      constexpr uint32_t idesc = umma_idesc_i8(BM, BN, true, true);
-      for (int kb = 0; kb < num_kb; ++kb) {
-        const int s = kb % STAGES;
-        if (!mbar_wait(&ready[s], (kb / STAGES) & 1, wait_ns)) {
+      constexpr uint32_t idesc = umma_idesc_i8(BW, BT, true, true);
+      int g = 0, j = 0;
+      for (int tile = blockIdx.x; tile < ntiles && !*failed; tile += gridDim.x, ++j) {
+        const int b = j & 1;
+        // the epilogue has read this buffer's previous tile (fresh barriers pass parity 1)
+        if (!mbar_wait(&acc_empty[b], ((j >> 1) & 1) ^ 1, wait_ns)) {
           *failed = 1;
           break;
         }
         tc_fence_after();
-        const uint32_t a_addr = smem_u32(smem + kOffA + s * kABytes);
-        const uint32_t b_addr = smem_u32(smem + kOffBu + s * kBuBytes);
-#pragma unroll
-        for (int j = 0; j < BK / 32; ++j)
-          umma_i8(tmem_base, umma_desc_sw128(a_addr + 32 * j), umma_desc_sw128(b_addr + 32 * j), idesc,
-                  (kb | j) != 0);
-        umma_commit(&empty[s]);
-      }
-      umma_commit(accum);   // fires once every MMA issued above has completed
-    }
-  } else if (warp >= 4) {
-    // ---------------- unpack ----------------
-    const int ut = threadIdx.x - 128;
-    for (int kb = 0; kb < num_kb; ++kb) {
-      const int s = kb % STAGES;
-      if (!mbar_wait(&full[s], (kb / STAGES) & 1, wait_ns)) {
-        *failed = 1;
-        break;
-      }
-      const uint8_t* bp = smem + kOffBp + s * kBpBytes;
-      uint8_t* bu = smem + kOffBu + s * kBuBytes;
-#pragma unroll
-      for (int it = 0; it < (BN * 2) / 128; ++it) {
-        const int idx = ut + 128 * it;
-        const int row = idx >> 1, half = idx & 1;
-        const uint4 q = *reinterpret_cast<const uint4*>(bp + row * 32 + half * 16);
-        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int c = half * 4 + j;   // 16-byte chunk = k 16c .. 16c + 15 of the block
-          const uint4 out = make_uint4(w[j] & kCodeMask, (w[j] >> 2) & kCodeMask, (w[j] >> 4) & kCodeMask,
-                                       (w[j] >> 6) & kCodeMask);
-          *reinterpret_cast<uint4*>(bu + row * 128 + ((c ^ (row & 7)) << 4)) = out;
-        }
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ready[s]);
-    }
-
-    // ---------------- epilogue ----------------
-    const int ew = warp - 4;                  // tensor-memory lanes 32*ew .. 32*ew + 31
-    const bool acc_ok = mbar_wait(accum, 0, wait_ns);
-    tc_fence_after();
-    pdl_wait_primary();
-    if (!acc_ok) *failed = 1;
-    if (acc_ok && !*failed) {
-      const int m = m0 + 32 * ew + lane;
-      const bool mv = m < a.M;
-      const float s_w = *a.w_scale;
-      const float d = mv ? __fmul_rn(a.s_x[m], s_w) : 1.0f;
-      const int rs = mv ? a.rowsum[m] : 0;
-      const bool vec = (a.N & 7) == 0;
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(32 * ew) << 16) + 32 * c, r);
-        tmem_wait_ld();
-        const int nb = n0 + 32 * c;
-        if (!mv || nb >= a.N) continue;
-        const size_t o = static_cast<size_t>(m) * a.N + nb;
-        uint32_t yb[16];
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          float v[2];
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int accv = static_cast<int>(r[i + h]) - rs;
-            float y32 = __fdiv_rn(static_cast<float>(accv), d);
-            if (a.bias && nb + i + h < a.N) y32 = __fadd_rn(y32, bf16_bits_to_f32(a.bias[nb + i + h]));
-            v[h] = y32;
-            if (nb + i + h < a.N) {
-              if (a.acc_out) a.acc_out[o + i + h] = accv;
-              if (a.y32_out) a.y32_out[o + i + h] = y32;
-            }
+        const uint32_t tmem_d = tmem_base + b * BT;
+        for (int kb = 0; kb < num_kb; ++kb, ++g) {
+          const int s = g % STAGES;
+          if (!mbar_wait(&ready[s], (g / STAGES) & 1, wait_ns)) {
+            *failed = 1;
+            break;
           }
-          yb[i / 2] = static_cast<uint32_t>(f32_to_bf16_bits(v[0])) |
-                      (static_cast<uint32_t>(f32_to_bf16_bits(v[1])) << 16);
-        }
-        if (vec && nb + 32 <= a.N) {
-          uint4* dst = reinterpret_cast<uint4*>(a.y + o);
+          tc_fence_after();
+          const uint32_t x_addr = smem_u32(smem + kOffX + s * kXBytes);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) dst[q] = make_uint4(yb[4 * q], yb[4 * q + 1], yb[4 * q + 2], yb[4 * q + 3]);
-        } else {
-          for (int i = 0; i < 32 && nb + i < a.N; ++i)
-            a.y[o + i] = static_cast<uint16_t>((i & 1) ? (yb[i / 2] >> 16) : (yb[i / 2] & 0xFFFFu));
+          for (int jj = 0; jj < BK / 32; ++jj)
+            umma_i8_ts(tmem_d, tmem_a + s * kACols + 8 * jj, umma_desc_sw128(x_addr + 32 * jj), idesc,
+                       (kb | jj) != 0);
+          umma_commit(&empty[s]);
+        }
+        if (*failed) break;
+        umma_commit(&acc_full[b]);                // the tile's accumulator is complete
+      }
+      // every MMA issued above has completed before tensor memory is freed
+      umma_commit(drain);
+      if (!mbar_wait(drain, 0, wait_ns)) *failed = 1;
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ---------------- weight unpack into tensor memory ----------------
+    const int q = warp & 3;
+    const int row = 32 * q + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
+    int g = 0;
+    for (int tile = blockIdx.x; tile < ntiles && !*failed; tile += gridDim.x) {
+      for (int kb = 0; kb < num_kb; ++kb, ++g) {
+        const int s = g % STAGES;
+        if (!mbar_wait(&full[s], (g / STAGES) & 1, wait_ns)) {
+          *failed = 1;
+          break;
+        }
+        const uint4* wp = reinterpret_cast<const uint4*>(smem + kOffWp + s * kWpBytes + row * 32);
+        const uint4 p0 = wp[0], p1 = wp[1];
+        const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+        uint32_t codes[32];
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {          // word jj = k 16jj .. 16jj + 15 of the block
+          codes[4 * jj + 0] = w[jj] & kCodeMask;
+          codes[4 * jj + 1] = (w[jj] >> 2) & kCodeMask;
+          codes[4 * jj + 2] = (w[jj] >> 4) & kCodeMask;
+          codes[4 * jj + 3] = (w[jj] >> 6) & kCodeMask;
+        }
+        tmem_st_32x32b_x32(tmem_a + lane_base + s * kACols, codes);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ready[s]);
+      }
+    }
+  } else if (warp >= 8) {
+    // ---------------- epilogue ----------------
+    const int q = warp & 3;
+    const int et = threadIdx.x - 256;             // 0..127
+    const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
+    pdl_wait_primary();
+    const float s_w = *a.w_scale;
+    int j = 0;
+    // The four epilogue warps meet at a named barrier twice per tile; every
+    // one of them runs every iteration (a failure only skips work), so the
+    // barrier always gets its 128 threads.
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++j) {
+      const int b = j & 1;
+      const int n0 = (tile % wtiles) * BW, m0 = (tile / wtiles) * BT;
+      // per-token d = s_x * s_w and row sums of this tile
+      asm volatile("bar.sync 1, 128;" ::: "memory");   // previous tile's readers are done
+      {
+        const int m = m0 + et;
+        d_s[et] = m < a.M ? __fmul_rn(a.s_x[m], s_w) : 1.0f;
+        rs_s[et] = m < a.M ? a.rowsum[m] : 0;
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      bool ok = !__any_sync(0xffffffffu, *failed != 0);
+      if (ok) ok = mbar_wait(&acc_full[b], (j >> 1) & 1, wait_ns);
+      ok = __all_sync(0xffffffffu, ok);             // warp-uniform decision
+      if (!ok) {
+        *failed = 1;
+        continue;
+      }
+      tc_fence_after();
+      const int n = n0 + 32 * q + lane;
+      const bool nv = n < a.N;
+      const float bv = (a.bias && nv) ? bf16_bits_to_f32(a.bias[n]) : 0.0f;
+#pragma unroll 1
+      for (int c = 0; c < BT / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tmem_base + b * BT + lane_base + 32 * c, r);
+        tmem_wait_ld();
+        if (c == BT / 32 - 1) {
+          // the whole accumulator is in registers: hand the buffer back
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[b]);
+        }
+        if (!nv) continue;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int mi = 32 * c + i, m = m0 + mi;
+          if (m >= a.M) continue;
+          const int accv = static_cast<int>(r[i]) - rs_s[mi];
+          float y32 = __fdiv_rn(static_cast<float>(accv), d_s[mi]);
+          if (a.bias) y32 = __fadd_rn(y32, bv);
+          const size_t o = static_cast<size_t>(m) * a.N + n;
+          a.y[o] = f32_to_bf16_bits(y32);
+          if (a.acc_out) a.acc_out[o] = accv;
+          if (a.y32_out) a.y32_out[o] = y32;
         }
       }
     }
@@ -212,7 +270,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 cudaError_t launch_gemm_prefill(const ForwardArgs& a, int num_sms, cudaStream_t stream) {
-  (void)num_sms;
   if (a.M <= 0) return cudaSuccess;
   static bool attr_done = false;
   if (!attr_done) {
@@ -222,12 +279,12 @@ cudaError_t launch_gemm_prefill(const ForwardArgs& a, int num_sms, cudaStream_t 
     attr_done = true;
   }
   CUtensorMap tm_x, tm_w;
-  if (!encode_2d_u8(&tm_x, a.xq, a.K, a.M, a.K, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B)) return cudaErrorInvalidValue;
-  if (!encode_2d_u8(&tm_w, a.packed, a.K / 4, a.N, a.K / 4, BK / 4, BN, CU_TENSOR_MAP_SWIZZLE_NONE))
+  if (!encode_2d_u8(&tm_x, a.xq, a.K, a.M, a.K, BK, BT, CU_TENSOR_MAP_SWIZZLE_128B)) return cudaErrorInvalidValue;
+  if (!encode_2d_u8(&tm_w, a.packed, a.K / 4, a.N, a.K / 4, BK / 4, BW, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
-
+  const long tiles = static_cast<long>((a.N + BW - 1) / BW) * ((a.M + BT - 1) / BT);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((a.N + BN - 1) / BN, (a.M + BM - 1) / BM, 1);
+  cfg.gridDim = dim3(static_cast<unsigned>(tiles < num_sms ? tiles : num_sms), 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = stream;

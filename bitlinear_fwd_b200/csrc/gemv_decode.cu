@@ -211,6 +211,9 @@ __global__ void __launch_bounds__(kThreads, 2)
       for (int b = 0; b < min(nb, ring); ++b) issue(b);
     s_w = *a.w_scale;
   }
+  // every peer's barriers exist from here on; the wait overlaps the
+  // dependency wait below instead of the activation phase
+  if (C > 1) cluster_wait();
   pdl_wait_primary();
   if (a.status && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *a.status = 0u;
   if (!a.weights_early) {
@@ -270,7 +273,6 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     __syncthreads();
     if (C > 1) {
-      cluster_wait();
       if (threadIdx.x < M * C) {                      // thread (m, r) sends token m's maximum to rank r
         const int m = threadIdx.x / C, r = threadIdx.x - m * C;
         const uint32_t v = sm.red_max[m];
@@ -321,7 +323,6 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
   } else {
     // pre-quantised input: copy the int8 slice, sum it per token
-    if (C > 1) cluster_wait();
     const int items = M * chunks;
     for (int j = 0; j * kThreads < items; ++j) {
       const int it = threadIdx.x + kThreads * j;
