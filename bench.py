@@ -144,16 +144,39 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def _dist_on():
+    return torch.distributed.is_available() and torch.distributed.is_initialized()
+
+
+def world_size():
+    return torch.distributed.get_world_size() if _dist_on() else 1
+
+
+def _reduce_device():
+    # NCCL reduces device tensors; gloo (the CPU test harness) host tensors
+    if torch.distributed.get_backend() == "nccl":
+        return torch.device("cuda", torch.cuda.current_device())
+    return torch.device("cpu")
+
+
 def elapsed_max_over_ranks(ms):
-    if torch.distributed.is_available() and torch.distributed.is_initialized():
-        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+    """The job's time is its slowest rank's: every rank passes its own
+    device-timed milliseconds and gets the maximum back."""
+    if _dist_on():
+        t = torch.tensor([ms], dtype=torch.float64, device=_reduce_device())
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         return float(t.item())
     return ms
 
 
+def whole_job_gbs(bytes_per_rank_step, steps, ms_max, world):
+    """Whole-job throughput: the bytes all replicas processed over the
+    slowest rank's time (every rank runs the same step)."""
+    return world * bytes_per_rank_step * steps / (ms_max * 1e-3) / 1e9
+
+
 def barrier():
-    if torch.distributed.is_available() and torch.distributed.is_initialized():
+    if _dist_on():
         torch.distributed.barrier()
 
 
@@ -286,8 +309,8 @@ def run_decode(args, hbm_gbs, l2_bytes, peak_kind):
     graphs = capture_steps(probs, copies, "forward")
     bytes_step = sum(decode_bytes(p.M, p.N, p.K, p.bias is not None) for p in probs)
     ms = timed_replays(graphs, args.steps, args.warmup, preroll_s=args.preroll)
-    world = torch.distributed.get_world_size() if torch.distributed.is_initialized() else 1
-    value = world * bytes_step * args.steps / (ms * 1e-3) / 1e9
+    world = world_size()
+    value = whole_job_gbs(bytes_step, args.steps, ms, world)
     launches = len(probs) * args.steps
     achieved = bytes_step * args.steps / (ms * 1e-3) / 1e9          # this rank's kernel
     kt = kernel_times(probs, copies, fn="forward")
@@ -326,9 +349,8 @@ def run_e2e(args, probs, steps):
     e1.synchronize()
     sync_all()
     ms = elapsed_max_over_ranks(e0.elapsed_time(e1))
-    world = torch.distributed.get_world_size() if torch.distributed.is_initialized() else 1
     bytes_step = sum(decode_bytes(p.M, p.N, p.K, p.bias is not None) for p in probs)
-    return {"value": round(world * bytes_step * steps / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+    return {"value": round(whole_job_gbs(bytes_step, steps, ms, world_size()), 2), "unit": "GB/s",
             "h2d_bytes_per_step": sum(2 * p.M * p.K for p in probs),
             "d2h_bytes_per_step": sum(2 * p.M * p.N for p in probs),
             "api": "bitlinear_forward_host (pinned host x in, host y out, synchronous per call)"}
@@ -341,8 +363,7 @@ def run_prefill(args, bf16_tflops, peak_kind, l2_bytes):
     ops_step = sum(2 * p.M * p.N * p.K for p in probs)
     steps = max(3, args.prefill_steps)
     ms = timed_replays(graphs, steps, max(3, args.warmup))
-    world = torch.distributed.get_world_size() if torch.distributed.is_initialized() else 1
-    tops = world * ops_step * steps / (ms * 1e-3) / 1e12
+    tops = world_size() * ops_step * steps / (ms * 1e-3) / 1e12
     kt = kernel_times(probs, copies, reps=8)
     ops = [2 * p.M * p.N * p.K for p in probs]
     achieved = sum(ops) / (sum(kt) * 1e-3) / 1e12

@@ -4,61 +4,66 @@
 // post_quant_process and the bias add) in one kernel that streams the 2-bit
 // packed weights once.
 //
-// Work split: a CTA owns 128 weight rows (8 warps x 16 rows) and a K-slice
-// of whole "boxes" (512 k = 128 packed bytes per row); the C CTAs of a
-// thread-block cluster (C in {1,2,4,8}, along K) own the slices of the same
-// 128 rows.
-//   1. At launch one thread issues TMA loads of the CTA's weight boxes
-//      (128 rows x 128 bytes, 128-byte swizzle) into a shared-memory ring.
-//      With resident weights this happens before the wait for the previous
-//      kernel on the stream, so the stream overlaps that kernel's tail.
-//   2. Activation quantisation of the CTA's slice of x: the per-token absmax
-//      of the slice is exchanged across the cluster through distributed
-//      shared memory, so every CTA derives the whole-row
-//      s_x = 127 / max(absmax, 1e-5) (float32) and the same int8 values; the
-//      int8 slice goes to shared memory (padded, swizzled for conflict-free
-//      fragment loads) with its row sums.  TMA copies are asynchronous, so
-//      the cluster barrier's release fence does not wait for the weight
-//      stream.  Pre-quantised int8 input is copied in instead.
-//   3. Warp w walks the boxes: per 256-k unit each thread takes one 16-byte
-//      vector of two weight rows and the x words of the same k, and issues
-//      mma.sync m16n8k32 (weights as A, u8; tokens as B, s8; a second
-//      8-token tile for M > 8).  The codes c = u + 1 enter unshifted:
-//      A_i = word & (0x03030303 << 2i) holds 4^i * c per byte lane, so field i
-//      accumulates 4^i * sum(c q) in its own int32 accumulator; the fields
-//      are combined with exact arithmetic shifts, and the slice's sum of q
-//      is subtracted (sum(c q) - sum(q) = sum(u q)).
-//   4. The cluster sums the slices' partial sums through distributed shared
-//      memory; CTA r of the cluster finishes rows r*128/C ..:
-//      y = acc / (s_x s_w) (+ bias) -> bf16.
-// Rows beyond N and k beyond K are zero-filled by TMA (code 0) and x is
-// zero-padded, so they add nothing.
+// Work split.  The N weight rows form 16-row units; the grid is one wave of
+// CTAs (at most one per SM) and CTA c owns a contiguous, balanced range of
+// units over the whole of K.  CTAs never talk to each other.
 //
-// Fragment layout.  MMA row g of a warp's 16-row group is shared-memory row
-// pi(g) = (g >> 1) | ((g & 1) << 2) (and pi(g) + 8), so that the two rows a
-// quarter-warp reads differ in bit 2 and the 128-byte swizzle puts their
-// chunks in disjoint bank groups.  Inside a unit thread (g, t) covers
-// k = 64t .. 64t + 63: register a0 of field i / pair p holds
-// k = 64t + 32p + 4i + {0..3}, a2 the same + 16; the B registers are the x
-// words at byte offsets 64t + 32p + 4i and 64t + 32p + 16 + 4i.
-#include <cooperative_groups.h>
-
+// Inside a CTA (8 consumer warps + 1 producer warp):
+//   * The producer thread streams the CTA's weights through a shared-memory
+//     ring with TMA and full/empty mbarriers, one load per (4096-k round,
+//     unit): a 3-D box of up to 8 sub-boxes of 16 rows x 128 bytes (512 k
+//     each, 128-byte swizzle), so each TMA instruction moves 16 KB (per-SM
+//     TMA throughput on B200 is set by the number of loads more than by their
+//     size), plus a 2-D box for a last 512-k chunk that K only partly fills
+//     (the 3-D view cannot bound it).  When the weights are resident it starts
+//     before the wait on the previous kernel of the stream, so the stream
+//     overlaps that kernel's tail.
+//   * The consumer warps form each token's absmax over the row, s_x =
+//     127 / max(absmax, 1e-5) in float32, and q = round_half_even(x s_x) as
+//     int8 into shared memory, one 4096-k round at a time, with the sum of q
+//     per token.  Pre-quantised int8 input is copied in instead.
+//   * In round r warp w takes sub-box w (k = 4096r + 512w ..) of every unit
+//     of the CTA, so it loads its x fragment once per round and reuses it for
+//     all units.  Per sub-box a thread
+//     takes one 16-byte vector of two weight rows and issues mma.sync
+//     m16n8k32 (weights as A, u8; tokens as B, s8; a second 8-token tile for
+//     M > 8).  The codes c = u + 1 enter unshifted: A_i = word &
+//     (0x03030303 << 2i) holds 4^i c per byte lane, so field i accumulates
+//     4^i sum(c q); the fields are combined with exact shifts and added to the
+//     unit's int32 sums in shared memory.
+//   * Epilogue: acc = sum(c q) - sum(q) = sum(u q); y = acc / (s_x s_w)
+//     (+ bias) -> bf16.
+// Rows beyond N and k beyond K are zero-filled by TMA (code 0), so they add
+// nothing whatever the x bytes there are.
+//
+// Fragment layout.  MMA row g of a unit is box row pi(g) = (g >> 1) |
+// ((g & 1) << 2) (and pi(g) + 8), so the two rows a quarter-warp reads
+// differ in bit 2 and the 128-byte swizzle puts their chunks in disjoint bank
+// groups.  Inside a sub-box, thread (g, t) covers k = 64t .. 64t + 63 of each
+// 256-k half v: register a0 of field i / pair p holds k = 64t + 32p + 4i +
+// {0..3}, a2 the same + 16; the B registers are the x words at byte offsets
+// 64t + 32p + 4i and 64t + 32p + 16 + 4i.
 #include "kernels.h"
-
-namespace cg = cooperative_groups;
 
 namespace bitlinear {
 
 namespace {
 
-constexpr int kWarps = 8;
-constexpr int kThreads = 32 * kWarps;
-constexpr int kRowsPerCta = 16 * kWarps;              // 128
-constexpr int kBoxK = 512;                            // k per TMA box
-constexpr int kBoxBytes = kRowsPerCta * kBoxK / 4;    // 16 KB
-constexpr int kMaxRing = 4;                           // boxes in flight per CTA
-constexpr int kSmemBudget = 110 * 1024;               // keeps two CTAs per SM
+constexpr int kConsumerWarps = 8;
+constexpr int kThreads = 32 * (kConsumerWarps + 1);   // + one producer warp
+constexpr int kConsumerThreads = 32 * kConsumerWarps;
+constexpr int kUnitRows = 16;
+constexpr int kBoxK = 512;                            // k per sub-box
+constexpr int kSubBytes = kUnitRows * kBoxK / 4;      // 2 KB
+constexpr int kChunkK = kConsumerWarps * kBoxK;       // k per round (one sub-box per warp)
+constexpr int kMaxRing = 16;
+constexpr int kMaxUnits = 16;                         // units per CTA
+constexpr int kXB = 8;                                // bf16 x loads in flight per lane (absmax)
+constexpr int kQB = 2;                                // the same in the quantising pass
+constexpr int kHold = 4;                              // 32-byte x chunks per lane and token held in
+                                                      // registers by the one-pass path
 constexpr uint32_t kCodeMask = 0x03030303u;
+constexpr float kRoundMagic = 12582912.0f;            // 1.5 * 2^23
 
 __device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
@@ -69,12 +74,21 @@ __device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, 
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// 16-byte chunk position in a token row of the x slice: within every 16
+// Barrier among the consumer warps only (the producer warp is busy).
+__device__ __forceinline__ void consumer_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads) : "memory");
+}
+
+__device__ __forceinline__ void red_shared_add(int* p, int v) {
+  asm volatile("red.shared.add.s32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+
+// 16-byte chunk position in a token row of the x chunk: within every 16
 // chunks, chunks 8..15 swap pairs (p ^ 2), so the four quad lanes t of a
 // fragment load hit four different bank groups.
 __device__ __forceinline__ int xs_chunk(int ch) { return ch ^ (((ch >> 3) & 1) << 1); }
 
-__device__ __forceinline__ int mma_row_to_smem(int g) { return (g >> 1) | ((g & 1) << 2); }
+__device__ __forceinline__ int mma_row_to_box(int g) { return (g >> 1) | ((g & 1) << 2); }
 
 // largest |x| of 16 bf16 values, as bf16 bits (finite values order like bits & 0x7FFF)
 __device__ __forceinline__ uint32_t absmax16_bits(uint4 lo, uint4 hi) {
@@ -86,372 +100,430 @@ __device__ __forceinline__ uint32_t absmax16_bits(uint4 lo, uint4 hi) {
   return max(m & 0xFFFFu, m >> 16);
 }
 
-// q = clamp(round_half_even(x * s), -128, 127) for 16 bf16 values; adds sum(q)
+// Four bf16 values (two words) -> four int8 q = round_half_even(x * s), packed.
+// p = x * s is rounded to float32 first; adding 1.5 * 2^23 then rounds p to an
+// integer with ties to even (the sum lies in [2^23, 2^24), where the float
+// spacing is 1, and the magic constant is even), and the low byte of the sum's
+// bits is q as a two's-complement byte.  |p| <= 127 for finite x because s was
+// formed from the row's absmax, so the [-128, 127] clamp never acts.
+__device__ __forceinline__ uint32_t quant4(uint32_t w01, uint32_t w23, float s) {
+  const float f0 = __uint_as_float(w01 << 16), f1 = __uint_as_float(w01 & 0xFFFF0000u);
+  const float f2 = __uint_as_float(w23 << 16), f3 = __uint_as_float(w23 & 0xFFFF0000u);
+  const uint32_t b0 = __float_as_uint(__fadd_rn(__fmul_rn(f0, s), kRoundMagic));
+  const uint32_t b1 = __float_as_uint(__fadd_rn(__fmul_rn(f1, s), kRoundMagic));
+  const uint32_t b2 = __float_as_uint(__fadd_rn(__fmul_rn(f2, s), kRoundMagic));
+  const uint32_t b3 = __float_as_uint(__fadd_rn(__fmul_rn(f3, s), kRoundMagic));
+  return __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
+}
+
 __device__ __forceinline__ uint4 quant16(uint4 lo, uint4 hi, float s, int& sum) {
-  const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-  uint32_t out[4];
-#pragma unroll
-  for (int b = 0; b < 4; ++b) {
-    uint32_t packed = 0;
-#pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      const int e = 4 * b + h;
-      const uint32_t bits = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu);
-      int q = __float2int_rn(__fmul_rn(bf16_bits_to_f32(bits), s));
-      q = min(127, max(-128, q));
-      sum += q;
-      packed |= (static_cast<uint32_t>(q) & 0xFFu) << (8 * h);
-    }
-    out[b] = packed;
-  }
-  return make_uint4(out[0], out[1], out[2], out[3]);
+  uint4 q;
+  q.x = quant4(lo.x, lo.y, s);
+  q.y = quant4(lo.z, lo.w, s);
+  q.z = quant4(hi.x, hi.y, s);
+  q.w = quant4(hi.z, hi.w, s);
+  sum = __dp4a(static_cast<int>(q.x), 0x01010101, sum);
+  sum = __dp4a(static_cast<int>(q.y), 0x01010101, sum);
+  sum = __dp4a(static_cast<int>(q.z), 0x01010101, sum);
+  sum = __dp4a(static_cast<int>(q.w), 0x01010101, sum);
+  return q;
 }
 
-__device__ __forceinline__ int bytesum16(uint4 v) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  int s = 0;
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-    s += static_cast<int8_t>(w[i] & 0xFF) + static_cast<int8_t>((w[i] >> 8) & 0xFF) +
-         static_cast<int8_t>((w[i] >> 16) & 0xFF) + static_cast<int8_t>(w[i] >> 24);
-  return s;
+__device__ __forceinline__ int bytesum16(uint4 v, int sum) {
+  sum = __dp4a(static_cast<int>(v.x), 0x01010101, sum);
+  sum = __dp4a(static_cast<int>(v.y), 0x01010101, sum);
+  sum = __dp4a(static_cast<int>(v.z), 0x01010101, sum);
+  return __dp4a(static_cast<int>(v.w), 0x01010101, sum);
 }
-
-__device__ __forceinline__ uint32_t mapa_u32(uint32_t local_smem_addr, int rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_smem_addr), "r"(rank));
-  return r;
-}
-// 32-bit / 64-bit store into a peer CTA's shared memory that completes
-// bytes on the peer's mbarrier.
-__device__ __forceinline__ void st_async_u32(uint32_t raddr, uint32_t v, uint32_t rbar) {
-  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(raddr), "r"(v),
-               "r"(rbar)
-               : "memory");
-}
-__device__ __forceinline__ void st_async_v2(uint32_t raddr, uint32_t v0, uint32_t v1, uint32_t rbar) {
-  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.b32 [%0], {%1, %2}, [%3];" ::"r"(raddr),
-               "r"(v0), "r"(v1), "r"(rbar)
-               : "memory");
-}
-__device__ __forceinline__ void cluster_arrive_relaxed() { asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory"); }
-__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
-
-constexpr int kChunkRegs = 4;   // 16-element x chunks a lane keeps in registers
 
 struct SmemTail {
-  uint64_t bar[kMaxRing];      // weight boxes
-  uint64_t bar_amax;           // slice maxima from the peers
-  uint64_t bar_red;            // partial sums from the peers
-  uint32_t amax[8][16];        // [source rank][token] slice absmax (bf16 bits)
-  uint32_t red_max[16];        // this slice's absmax per token, then the row's
-  int red[8 * 16 * 16];        // [source rank][row_local][token] partials for this CTA's rows
-  int rsum[16];                // this slice's sum of q per token
-  float sx[16];                // s_x per token
-  uint16_t bias[kRowsPerCta];  // bias of this CTA's output rows
+  uint64_t full[kMaxRing];
+  uint64_t empty[kMaxRing];
+  uint32_t amax[16];                 // absmax per token (bf16 bits)
+  int rsum[16];                      // sum of q per token
+  float sx[16];                      // s_x per token
+  float sw;
+  int issued;                        // loads issued (producer)
+  int failed;                        // a wait of this CTA timed out
 };
 
-size_t smem_bytes(int ntok, int ring, int boxes_per_cta) {
-  return 1024 + static_cast<size_t>(ring) * kBoxBytes + static_cast<size_t>(ntok) * (boxes_per_cta * kBoxK + 16) +
-         sizeof(SmemTail);
+struct SmemLayout {
+  size_t ring, xs, acc, bias, tail, total;
+};
+
+// ring slots of slot_bytes (1024-aligned base), x rows of one round for the
+// M tokens, per-unit int32 sums [unit][row][8 * token tiles], bias, tail
+__host__ __device__ SmemLayout smem_layout(int M, int ring, size_t slot_bytes, int units) {
+  const int ntok = M <= 8 ? 8 : 16;
+  SmemLayout L;
+  L.ring = 0;
+  L.xs = L.ring + static_cast<size_t>(ring) * slot_bytes;
+  L.acc = L.xs + static_cast<size_t>(M) * (kChunkK + 16);
+  L.bias = L.acc + static_cast<size_t>(units) * kUnitRows * ntok * 4;
+  L.tail = (L.bias + static_cast<size_t>(units) * kUnitRows * 2 + 15) & ~size_t(15);
+  L.total = 1024 + L.tail + sizeof(SmemTail);
+  return L;
 }
 
-template <int NT, int C>
-__global__ void __launch_bounds__(kThreads, 2)
-    decode_kernel(const __grid_constant__ CUtensorMap tm_w, const DecodeArgs a) {
+template <int NT>
+__global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
+    decode_kernel(const __grid_constant__ CUtensorMap tm3, const __grid_constant__ CUtensorMap tm2,
+                  const DecodeArgs a) {
   constexpr int NTOK = NT * 8;
-  constexpr int R = kRowsPerCta / C;                  // output rows finished by this CTA
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   const int ring = a.ring;
-  const int S = a.xs_stride;                          // bytes per token row of the x slice
-  uint8_t* rbuf = base;                               // ring of weight boxes, 1024-aligned
-  int8_t* xs = reinterpret_cast<int8_t*>(base + ring * kBoxBytes);
-  SmemTail& sm = *reinterpret_cast<SmemTail*>(base + ring * kBoxBytes + NTOK * S);
+  const int kc = a.kc;                               // sub-boxes per 3-D load (0 when K < 512)
+  const size_t slot_bytes = static_cast<size_t>(kc + a.tail) * kSubBytes;
+  const SmemLayout L = smem_layout(a.M, ring, slot_bytes, a.units_max);
+  uint8_t* rbuf = base + L.ring;
+  int8_t* xs = reinterpret_cast<int8_t*>(base + L.xs);
+  int* acc_s = reinterpret_cast<int*>(base + L.acc);            // [unit][row][token]
+  uint16_t* bias_s = reinterpret_cast<uint16_t*>(base + L.bias);
+  SmemTail& sm = *reinterpret_cast<SmemTail*>(base + L.tail);
+  constexpr int S = kChunkK + 16;                    // bytes per token row of the x round
 
   pdl_launch_dependents();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, t = lane & 3;
-  const int crank = blockIdx.x, rb = blockIdx.y;
   const int K = a.K, N = a.N, M = a.M;
-  const int nbox_total = (K + kBoxK - 1) / kBoxK;
-  const int b_begin = crank * a.boxes_per_cta;
-  const int nb = max(0, min(nbox_total, b_begin + a.boxes_per_cta) - b_begin);
-  const int npairs = (M + 1) >> 1;                    // token pairs exchanged per row
+  const int units_total = (N + kUnitRows - 1) / kUnitRows;
+  const int u_begin = static_cast<int>(static_cast<long long>(blockIdx.x) * units_total / gridDim.x);
+  const int U = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * units_total / gridDim.x) - u_begin;
+  const int nbox = (K + kBoxK - 1) / kBoxK;          // 512-k chunks, the last maybe partial
+  const int F = K / kBoxK;                           // full 512-k chunks (the 3-D view's extent)
+  const int nround = (K + kChunkK - 1) / kChunkK;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < ring; ++s) mbar_init(&sm.bar[s], 1);
-    mbar_init(&sm.bar_amax, 1);
-    mbar_init(&sm.bar_red, 1);
-    fence_mbar_init();
-    tma_prefetch_desc(&tm_w);
-    if (C > 1) {
-      mbar_arrive_expect_tx(&sm.bar_amax, a.x ? static_cast<uint32_t>((C - 1) * M * 4) : 0u);
-      mbar_arrive_expect_tx(&sm.bar_red, static_cast<uint32_t>((C - 1) * R * npairs * 8));
+    for (int s = 0; s < ring; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], kConsumerWarps);
     }
+    fence_mbar_init();
+    if (kc > 0) tma_prefetch_desc(&tm3);
+    if (a.tail) tma_prefetch_desc(&tm2);
   }
   if (threadIdx.x < 16) {
-    sm.red_max[threadIdx.x] = 0u;
+    sm.amax[threadIdx.x] = 0u;
     sm.rsum[threadIdx.x] = 0;
   }
-  __syncthreads();
-  if (C > 1) cluster_arrive_relaxed();                // peers may push once their barriers exist
-
-  int issued = 0;                                     // meaningful in thread 0 only
-  auto issue = [&](int b) {
-    const int s = b % ring;
-    mbar_arrive_expect_tx(&sm.bar[s], kBoxBytes);
-    tma_load_2d(rbuf + s * kBoxBytes, &tm_w, &sm.bar[s], (b_begin + b) * (kBoxK / 4), rb * kRowsPerCta);
-    issued = b + 1;
-  };
-  float s_w = 0.0f;
-  if (a.weights_early) {
-    if (threadIdx.x == 0)
-      for (int b = 0; b < min(nb, ring); ++b) issue(b);
-    s_w = *a.w_scale;
+  if (threadIdx.x == 0) {
+    sm.issued = 0;
+    sm.failed = 0;
   }
-  // every peer's barriers exist from here on; the wait overlaps the
-  // dependency wait below instead of the activation phase
-  if (C > 1) cluster_wait();
-  pdl_wait_primary();
-  if (a.status && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *a.status = 0u;
-  if (!a.weights_early) {
-    if (threadIdx.x == 0)
-      for (int b = 0; b < min(nb, ring); ++b) issue(b);
-    s_w = *a.w_scale;
-  }
-  if (threadIdx.x < R) {
-    const int n = rb * kRowsPerCta + crank * R + threadIdx.x;
-    sm.bias[threadIdx.x] = (a.bias && n < N) ? a.bias[n] : static_cast<uint16_t>(0);
-  }
-
-  // ---------------- x slice -> int8 in shared memory ----------------
-  // Items are (token m, 16-element chunk ch) with it = m * chunks + ch; the
-  // chunk count is a multiple of 32, so the 32 items a warp holds at a time
-  // belong to one token and reduce with one warp-wide max / sum.
-  const int chunks = a.boxes_per_cta * (kBoxK / 16);  // 16-element chunks per token row of the slice
-  const int k_begin = b_begin * kBoxK;
-  const bool write_xq = rb == 0 && a.xq_out != nullptr;
-  if (a.x) {
-    const int items = M * chunks;
-    uint4 xr[kChunkRegs][2];
-#pragma unroll
-    for (int j = 0; j < kChunkRegs; ++j) {
-      const int it = threadIdx.x + kThreads * j;
-      const int m = it / chunks, ch = it - m * chunks;
-      const int k0 = k_begin + 16 * ch;
-      uint4 lo = make_uint4(0, 0, 0, 0), hi = make_uint4(0, 0, 0, 0);
-      if (it < items && k0 < K) {
-        const uint4* src = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(m) * K + k0);
-        lo = __ldg(src);
-        hi = __ldg(src + 1);
-      }
-      xr[j][0] = lo;
-      xr[j][1] = hi;
-    }
-    // slice absmax per token: registers, then the rest of the slice
-    for (int j = 0; j * kThreads < items; ++j) {
-      const int it = threadIdx.x + kThreads * j;       // warp-uniform token
-      const int m = min(it, items - 1) / chunks;
-      uint32_t mx = 0;
-      if (it < items) {
-        if (j < kChunkRegs) {
-#pragma unroll
-          for (int jj = 0; jj < kChunkRegs; ++jj)
-            if (jj == j) mx = absmax16_bits(xr[jj][0], xr[jj][1]);
-        } else {
-          const int ch = it - m * chunks, k0 = k_begin + 16 * ch;
-          if (k0 < K) {
-            const uint4* src = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(m) * K + k0);
-            mx = absmax16_bits(__ldg(src), __ldg(src + 1));
-          }
-        }
-      }
-      mx = __reduce_max_sync(0xffffffffu, mx);
-      if (lane == 0 && it < items) atomicMax(&sm.red_max[m], mx);
-    }
-    __syncthreads();
-    if (C > 1) {
-      if (threadIdx.x < M * C) {                      // thread (m, r) sends token m's maximum to rank r
-        const int m = threadIdx.x / C, r = threadIdx.x - m * C;
-        const uint32_t v = sm.red_max[m];
-        if (r == crank) sm.amax[crank][m] = v;
-        else st_async_u32(mapa_u32(smem_u32(&sm.amax[crank][m]), r), v, mapa_u32(smem_u32(&sm.bar_amax), r));
-      }
-      if (!mbar_wait(&sm.bar_amax, 0, kWaitLimitNs)) report_status(a.status, kStatusTimeout);
-      __syncthreads();
-      if (threadIdx.x < M) {
-        uint32_t mx = 0;
-#pragma unroll
-        for (int r = 0; r < C; ++r) mx = max(mx, sm.amax[r][threadIdx.x]);
-        sm.red_max[threadIdx.x] = mx;
-      }
-    }
-    __syncthreads();
-    if (threadIdx.x < M) {
-      const float sxv = __fdiv_rn(127.0f, fmaxf(bf16_bits_to_f32(sm.red_max[threadIdx.x]), 1e-5f));
-      sm.sx[threadIdx.x] = sxv;
-      if (write_xq && crank == 0 && a.sx_out) a.sx_out[threadIdx.x] = sxv;
-    }
-    __syncthreads();
-    for (int j = 0; j * kThreads < items; ++j) {
-      const int it = threadIdx.x + kThreads * j;
-      const int m = min(it, items - 1) / chunks, ch = it - m * chunks;
-      const int k0 = k_begin + 16 * ch;
-      int sum = 0;
-      if (it < items) {
-        uint4 q = make_uint4(0, 0, 0, 0);
-        if (k0 < K) {
-          uint4 lo, hi;
-          if (j < kChunkRegs) {
-#pragma unroll
-            for (int jj = 0; jj < kChunkRegs; ++jj)
-              if (jj == j) { lo = xr[jj][0]; hi = xr[jj][1]; }
-          } else {
-            const uint4* src = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(m) * K + k0);
-            lo = __ldg(src);
-            hi = __ldg(src + 1);
-          }
-          q = quant16(lo, hi, sm.sx[m], sum);
-          if (write_xq) *reinterpret_cast<uint4*>(a.xq_out + static_cast<size_t>(m) * K + k0) = q;
-        }
-        *reinterpret_cast<uint4*>(xs + m * S + 16 * xs_chunk(ch)) = q;
-      }
-      sum = __reduce_add_sync(0xffffffffu, sum);
-      if (lane == 0 && it < items) atomicAdd(&sm.rsum[m], sum);
-    }
-  } else {
-    // pre-quantised input: copy the int8 slice, sum it per token
-    const int items = M * chunks;
-    for (int j = 0; j * kThreads < items; ++j) {
-      const int it = threadIdx.x + kThreads * j;
-      const int m = min(it, items - 1) / chunks, ch = it - m * chunks;
-      const int k0 = k_begin + 16 * ch;
-      int sum = 0;
-      if (it < items) {
-        uint4 q = make_uint4(0, 0, 0, 0);
-        if (k0 < K) {
-          q = __ldg(reinterpret_cast<const uint4*>(a.xq + static_cast<size_t>(m) * K + k0));
-          sum = bytesum16(q);
-        }
-        *reinterpret_cast<uint4*>(xs + m * S + 16 * xs_chunk(ch)) = q;
-      }
-      sum = __reduce_add_sync(0xffffffffu, sum);
-      if (lane == 0 && it < items) atomicAdd(&sm.rsum[m], sum);
-    }
-    if (threadIdx.x < M) sm.sx[threadIdx.x] = a.s_x[threadIdx.x];
-  }
-  // padding token rows M .. NTOK-1 read as zeros
-  for (int it = threadIdx.x; it < (NTOK - M) * chunks; it += kThreads) {
-    const int m = M + it / chunks, ch = it % chunks;
-    *reinterpret_cast<uint4*>(xs + m * S + 16 * xs_chunk(ch)) = make_uint4(0, 0, 0, 0);
-  }
+  for (int i = threadIdx.x; i < U * kUnitRows * NTOK; i += kThreads) acc_s[i] = 0;
   __syncthreads();
 
-  // ---------------- contraction over the slice ----------------
-  int acc[4][NT][4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int r = 0; r < 4; ++r) acc[i][nt][r] = 0;
-
-  const int r0 = warp * 16 + mma_row_to_smem(g);     // shared-memory rows r0 and r0 + 8
   bool ok = true;
-  for (int b = 0; b < nb; ++b) {
-    const int s = b % ring;
-    if (ok) ok = mbar_wait(&sm.bar[s], (b / ring) & 1, kWaitLimitNs);
-    if (ok) {
-      const uint8_t* box = rbuf + s * kBoxBytes;
+  if (warp == kConsumerWarps) {
+    // ======================= producer warp =======================
+    if (!a.weights_early) pdl_wait_primary();
+    for (int i = lane; i < U * kUnitRows; i += 32) {
+      const int n = u_begin * kUnitRows + i;
+      bias_s[i] = (a.bias && n < N) ? a.bias[n] : static_cast<uint16_t>(0);
+    }
+    if (lane == 0) {
+      sm.sw = *a.w_scale;
+      int q = 0;
+      for (int r = 0; r < nround && ok; ++r) {
+        const bool has3 = kc > 0 && 8 * r < F;       // full chunks of this round, one 3-D load
+        const bool hast = a.tail && (F >> 3) == r;   // the partial chunk, one 2-D load
+        const uint32_t bytes = (has3 ? kc * kSubBytes : 0) + (hast ? kSubBytes : 0);
+        for (int u = 0; u < U; ++u, ++q) {
+          const int s = q % ring;
+          if (q >= ring && !mbar_wait(&sm.empty[s], ((q / ring) - 1) & 1, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          uint8_t* dst = rbuf + s * slot_bytes;
+          const int row = (u_begin + u) * kUnitRows;
+          mbar_arrive_expect_tx(&sm.full[s], bytes);
+          if (has3) tma_load_3d(dst, &tm3, &sm.full[s], 0, row, 8 * r);
+          if (hast) tma_load_2d(dst + kc * kSubBytes, &tm2, &sm.full[s], F * (kBoxK / 4), row);
+        }
+      }
+      sm.issued = q;
+    }
+    __syncwarp();
+  } else {
+    // ======================= consumer warps =======================
+    pdl_wait_primary();
+    if (a.status && blockIdx.x == 0 && threadIdx.x == 0) *a.status = 0u;
+    const int g = lane >> 2, t = lane & 3;
+
+    // ---- per-token absmax over the whole row: warp w takes token(s)
+    // m = w / P (+ 8 / P, ...) and a 1/P share of the row, P = max(1, 8 / M)
+    const int cpr = K >> 4;                          // 16-element chunks per row
+    const int P = M >= kConsumerWarps ? 1 : kConsumerWarps / M;
+    const int part = warp % P, mstep = kConsumerWarps / P;
+    const int C = (cpr + 32 * P - 1) / (32 * P);     // chunks per lane per token
+    // One pass over x when the row is one round and this lane's share fits in
+    // registers: the values loaded for the absmax are quantised in place.
+    const bool single = NT == 1 && a.x && nround == 1 && C <= kHold;
+    if (single) {
+      const uint4* xrow0 = reinterpret_cast<const uint4*>(a.x);
+      uint4 v[kHold * NT][2];
 #pragma unroll
-      for (int v = 0; v < 2; ++v) {                   // two 256-k units per box
-        const int cw = 4 * v + t;                     // 16-byte chunk of the 128-byte row
-        const uint4 wa = *reinterpret_cast<const uint4*>(box + r0 * 128 + ((cw ^ (r0 & 7)) << 4));
-        const uint4 wb = *reinterpret_cast<const uint4*>(box + (r0 + 8) * 128 + ((cw ^ ((r0 + 8) & 7)) << 4));
-        const uint32_t w0[4] = {wa.x, wa.y, wa.z, wa.w};
-        const uint32_t w1[4] = {wb.x, wb.y, wb.z, wb.w};
+      for (int i = 0; i < kHold * NT; ++i) {
+        const int j = (NT == 2 && i >= C) ? 1 : 0;   // token slot of this warp
+        const int m = warp / P + j * mstep;
+        const int ch = part * 32 + lane + (i - j * C) * 32 * P;
+        v[i][0] = v[i][1] = make_uint4(0, 0, 0, 0);
+        if (i < NT * C && m < M && ch < cpr) {
+          v[i][0] = __ldg(xrow0 + (static_cast<size_t>(m) * K >> 3) + 2 * ch);
+          v[i][1] = __ldg(xrow0 + (static_cast<size_t>(m) * K >> 3) + 2 * ch + 1);
+        }
+      }
+      uint32_t mx[NT];
 #pragma unroll
-        for (int pr = 0; pr < 2; ++pr) {
-          // x words 8pr .. 8pr + 7 of the thread's 64-byte span (chunks 2pr, 2pr + 1)
-          uint32_t xw[NT][8];
+      for (int j = 0; j < NT; ++j) mx[j] = 0;
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            const int8_t* xrow = xs + (nt * 8 + g) * S;
+      for (int i = 0; i < kHold * NT; ++i) {
+        const uint32_t am = absmax16_bits(v[i][0], v[i][1]);   // zeros where nothing was loaded
+        if (NT == 2 && i >= C) mx[NT - 1] = max(mx[NT - 1], am);
+        else mx[0] = max(mx[0], am);
+      }
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-              const uint4 xv =
-                  *reinterpret_cast<const uint4*>(xrow + 16 * xs_chunk(32 * b + 16 * v + 4 * t + 2 * pr + c));
-              xw[nt][4 * c + 0] = xv.x; xw[nt][4 * c + 1] = xv.y;
-              xw[nt][4 * c + 2] = xv.z; xw[nt][4 * c + 3] = xv.w;
+      for (int j = 0; j < NT; ++j) {
+        const int m = warp / P + j * mstep;
+        const uint32_t r = __reduce_max_sync(0xffffffffu, mx[j]);
+        if (lane == 0 && m < M) atomicMax(&sm.amax[m], r);
+      }
+      consumer_sync();
+      float sxr[NT];
+#pragma unroll
+      for (int j = 0; j < NT; ++j) {
+        const int m = min(warp / P + j * mstep, M - 1);
+        sxr[j] = __fdiv_rn(127.0f, fmaxf(bf16_bits_to_f32(sm.amax[m]), 1e-5f));
+      }
+      if (threadIdx.x < M) {
+        const float sxv = __fdiv_rn(127.0f, fmaxf(bf16_bits_to_f32(sm.amax[threadIdx.x]), 1e-5f));
+        sm.sx[threadIdx.x] = sxv;
+        if (blockIdx.x == 0 && a.sx_out) a.sx_out[threadIdx.x] = sxv;
+      }
+      int sum[NT];
+#pragma unroll
+      for (int j = 0; j < NT; ++j) sum[j] = 0;
+#pragma unroll
+      for (int i = 0; i < kHold * NT; ++i) {
+        const int j = (NT == 2 && i >= C) ? 1 : 0;
+        const int m = warp / P + j * mstep;
+        const int ch = part * 32 + lane + (i - j * C) * 32 * P;
+        if (i < NT * C && m < M && ch < cpr) {
+          int ps = 0;
+          const uint4 qv = quant16(v[i][0], v[i][1], j ? sxr[NT - 1] : sxr[0], ps);
+          if (j) sum[NT - 1] += ps;
+          else sum[0] += ps;
+          *reinterpret_cast<uint4*>(xs + m * S + 16 * xs_chunk(ch)) = qv;
+          if (blockIdx.x == 0 && a.xq_out) *reinterpret_cast<uint4*>(a.xq_out + static_cast<size_t>(m) * K + 16 * ch) = qv;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < NT; ++j) {
+        const int m = warp / P + j * mstep;
+        const int r = __reduce_add_sync(0xffffffffu, sum[j]);
+        if (lane == 0 && m < M) atomicAdd(&sm.rsum[m], r);
+      }
+    } else if (a.x) {
+      for (int m = warp / P; m < M; m += mstep) {
+        const uint4* row = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(m) * K);
+        uint32_t mx = 0;
+        // kXB 32-byte loads in flight per lane before any is used
+        for (int ch0 = part * 32 + lane; ch0 < cpr; ch0 += 32 * P * kXB) {
+          uint4 v[kXB][2];
+#pragma unroll
+          for (int j = 0; j < kXB; ++j) {
+            const int ch = ch0 + j * 32 * P;
+            v[j][0] = v[j][1] = make_uint4(0, 0, 0, 0);
+            if (ch < cpr) {
+              v[j][0] = __ldg(row + 2 * ch);
+              v[j][1] = __ldg(row + 2 * ch + 1);
             }
           }
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint32_t mask = kCodeMask << (2 * i);
-            const uint32_t a0 = w0[2 * pr] & mask, a1 = w1[2 * pr] & mask;
-            const uint32_t a2 = w0[2 * pr + 1] & mask, a3 = w1[2 * pr + 1] & mask;
+          for (int j = 0; j < kXB; ++j) mx = max(mx, absmax16_bits(v[j][0], v[j][1]));
+        }
+        mx = __reduce_max_sync(0xffffffffu, mx);
+        if (lane == 0) atomicMax(&sm.amax[m], mx);
+      }
+      consumer_sync();
+      if (threadIdx.x < M) {
+        const float sxv = __fdiv_rn(127.0f, fmaxf(bf16_bits_to_f32(sm.amax[threadIdx.x]), 1e-5f));
+        sm.sx[threadIdx.x] = sxv;
+        if (blockIdx.x == 0 && a.sx_out) a.sx_out[threadIdx.x] = sxv;
+      }
+    } else {
+      if (threadIdx.x < M) sm.sx[threadIdx.x] = a.s_x[threadIdx.x];
+    }
+    consumer_sync();
+
+    const int r0 = mma_row_to_box(g);                // sub-box rows r0 and r0 + 8
+    for (int r = 0; r < nround; ++r) {
+      const int c0 = r * kChunkK;
+      const int ccpr = min(kChunkK, K - c0) >> 4;    // 16-element chunks of x in this round
+      if (r > 0) consumer_sync();                    // previous round's fragments are loaded
+      // ---- x round -> int8 in shared memory (tokens < M only)
+      for (int m = warp / P; m < (single ? 0 : M); m += mstep) {
+        int8_t* xrow = xs + m * S;
+        const float sxm = sm.sx[m];
+        int sum = 0;
+        const size_t roff = static_cast<size_t>(m) * K + c0;
+        for (int ch0 = part * 32 + lane; ch0 < ccpr; ch0 += 32 * P * kQB) {
+          if (a.x) {
+            const uint4* src = reinterpret_cast<const uint4*>(a.x + roff);
+            uint4 v[kQB][2];
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) mma_u8s8(acc[i][nt], a0, a1, a2, a3, xw[nt][i], xw[nt][4 + i]);
+            for (int j = 0; j < kQB; ++j) {
+              const int ch = ch0 + j * 32 * P;
+              if (ch < ccpr) {
+                v[j][0] = __ldg(src + 2 * ch);
+                v[j][1] = __ldg(src + 2 * ch + 1);
+              }
+            }
+#pragma unroll
+            for (int j = 0; j < kQB; ++j) {
+              const int ch = ch0 + j * 32 * P;
+              if (ch < ccpr) {
+                const uint4 qv = quant16(v[j][0], v[j][1], sxm, sum);
+                if (blockIdx.x == 0 && a.xq_out) *reinterpret_cast<uint4*>(a.xq_out + roff + 16 * ch) = qv;
+                *reinterpret_cast<uint4*>(xrow + 16 * xs_chunk(ch)) = qv;
+              }
+            }
+          } else {
+            const uint4* src = reinterpret_cast<const uint4*>(a.xq + roff);
+            uint4 v[kQB];
+#pragma unroll
+            for (int j = 0; j < kQB; ++j) {
+              const int ch = ch0 + j * 32 * P;
+              if (ch < ccpr) v[j] = __ldg(src + ch);
+            }
+#pragma unroll
+            for (int j = 0; j < kQB; ++j) {
+              const int ch = ch0 + j * 32 * P;
+              if (ch < ccpr) {
+                sum = bytesum16(v[j], sum);
+                *reinterpret_cast<uint4*>(xrow + 16 * xs_chunk(ch)) = v[j];
+              }
+            }
+          }
+        }
+        sum = __reduce_add_sync(0xffffffffu, sum);
+        if (lane == 0) atomicAdd(&sm.rsum[m], sum);
+      }
+      if (!single) consumer_sync();
+
+      // ---- contraction: this warp's sub-box of every unit
+      const int nw = min(kConsumerWarps, nbox - 8 * r);
+      const bool mine = warp < nw;
+      const int sub = (a.tail && 8 * r + warp == F) ? kc : warp;   // partial chunk: the 2-D box
+      uint32_t xw[2][2][NT][8];                      // [v][pair][token tile][word]
+#pragma unroll
+      for (int v = 0; v < 2; ++v)
+#pragma unroll
+        for (int pr = 0; pr < 2; ++pr)
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            const int m = nt * 8 + g;
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+              uint4 xv = make_uint4(0, 0, 0, 0);
+              if (mine && m < M)
+                xv = *reinterpret_cast<const uint4*>(xs + m * S +
+                                                     16 * xs_chunk(32 * warp + 16 * v + 4 * t + 2 * pr + cc));
+              xw[v][pr][nt][4 * cc + 0] = xv.x; xw[v][pr][nt][4 * cc + 1] = xv.y;
+              xw[v][pr][nt][4 * cc + 2] = xv.z; xw[v][pr][nt][4 * cc + 3] = xv.w;
+            }
+          }
+      for (int u = 0; u < U; ++u) {
+        const int q = r * U + u;
+        const int s = q % ring;
+        // every consumer warp waits for every load (also when it has no
+        // sub-box in it): its arrival on the empty barrier must not run ahead
+        // of the slot's phases
+        if (ok && !mbar_wait(&sm.full[s], (q / ring) & 1, kWaitLimitNs)) ok = false;
+        if (!ok) break;
+        int acc[4][NT][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr) acc[i][nt][rr] = 0;
+        if (mine) {
+          const uint8_t* box = rbuf + s * slot_bytes + sub * kSubBytes;
+#pragma unroll
+          for (int v = 0; v < 2; ++v) {
+            const int cw = 4 * v + t;                // 16-byte chunk of the 128-byte row
+            const uint4 wa = *reinterpret_cast<const uint4*>(box + r0 * 128 + ((cw ^ r0) << 4));
+            const uint4 wb = *reinterpret_cast<const uint4*>(box + (r0 + 8) * 128 + ((cw ^ r0) << 4));
+            const uint32_t w0[4] = {wa.x, wa.y, wa.z, wa.w};
+            const uint32_t w1[4] = {wb.x, wb.y, wb.z, wb.w};
+#pragma unroll
+            for (int pr = 0; pr < 2; ++pr)
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const uint32_t mask = kCodeMask << (2 * i);
+                const uint32_t a0 = w0[2 * pr] & mask, a1 = w1[2 * pr] & mask;
+                const uint32_t a2 = w0[2 * pr + 1] & mask, a3 = w1[2 * pr + 1] & mask;
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+                  mma_u8s8(acc[i][nt], a0, a1, a2, a3, xw[v][pr][nt][i], xw[v][pr][nt][4 + i]);
+              }
+          }
+        }
+        // the slot's shared memory is read: hand it back to the producer
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.empty[s]);
+        if (mine) {
+          int* au = acc_s + u * kUnitRows * NTOK;
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            int cv[4];
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr)
+              cv[rr] = acc[0][nt][rr] + (acc[1][nt][rr] >> 2) + (acc[2][nt][rr] >> 4) + (acc[3][nt][rr] >> 6);
+            const int m0 = nt * 8 + 2 * t;
+            if (m0 < M) {
+              red_shared_add(au + r0 * NTOK + m0, cv[0]);
+              red_shared_add(au + (r0 + 8) * NTOK + m0, cv[2]);
+            }
+            if (m0 + 1 < M) {
+              red_shared_add(au + r0 * NTOK + m0 + 1, cv[1]);
+              red_shared_add(au + (r0 + 8) * NTOK + m0 + 1, cv[3]);
+            }
           }
         }
       }
     }
-    if (b + ring < nb) {               // refill the slot once every warp is done with it
-      __syncthreads();
-      if (threadIdx.x == 0 && ok) issue(b + ring);
-    }
   }
-  if (threadIdx.x == 0) {
-    // drain: every box issued into the ring has landed before the CTA exits
-    for (int s = 0; s < ring && s < issued; ++s) {
-      const int last = s + ((issued - 1 - s) / ring) * ring;
-      if (!mbar_wait(&sm.bar[s], (last / ring) & 1, kWaitLimitNs)) ok = false;
-    }
-  }
-  if (!ok) report_status(a.status, kStatusTimeout);
-
-  // ---------------- partial sums -> the CTA that finishes each row ----------------
-  // value (row, token): sum over this slice of c*q, minus the slice's sum of q
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    const int m0 = nt * 8 + 2 * t;                   // tokens m0, m0 + 1 of this thread
-    if (m0 < M) {
-      const int rs0 = sm.rsum[m0], rs1 = (m0 + 1 < M) ? sm.rsum[m0 + 1] : 0;
-      int c[4];
-#pragma unroll
-      for (int r = 0; r < 4; ++r)
-        c[r] = acc[0][nt][r] + (acc[1][nt][r] >> 2) + (acc[2][nt][r] >> 4) + (acc[3][nt][r] >> 6);
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {                  // rows r0 and r0 + 8
-        const int row = r0 + 8 * h;
-        const int owner = row / R, rl = row - owner * R;
-        int* dst = &sm.red[(crank * R + rl) * 16 + m0];
-        const uint32_t v0 = static_cast<uint32_t>(c[2 * h] - rs0), v1 = static_cast<uint32_t>(c[2 * h + 1] - rs1);
-        if (C == 1 || owner == crank) {
-          dst[0] = static_cast<int>(v0);
-          dst[1] = static_cast<int>(v1);
-        } else {
-          st_async_v2(mapa_u32(smem_u32(dst), owner), v0, v1, mapa_u32(smem_u32(&sm.bar_red), owner));
-        }
-      }
-    }
+  if (!ok) {
+    report_status(a.status, kStatusTimeout);
+    sm.failed = 1;
   }
   __syncthreads();
-  if (C > 1 && !mbar_wait(&sm.bar_red, 0, kWaitLimitNs)) report_status(a.status, kStatusTimeout);
+  if (sm.failed && threadIdx.x == kConsumerWarps * 32) {
+    // After a timeout some loads may still be in flight, and every load
+    // issued must land before the CTA exits.  The last load into a slot
+    // completes that slot's latest phase: the loads before it were consumed,
+    // which needed them complete.
+    const int q = sm.issued;
+    for (int s = 0; s < ring && s < q; ++s) {
+      const int last = s + ((q - 1 - s) / ring) * ring;
+      mbar_wait(&sm.full[s], (last / ring) & 1, kWaitLimitNs);
+    }
+  }
 
-  // ---------------- epilogue for this CTA's R rows ----------------
-  for (int idx = threadIdx.x; idx < R * M; idx += kThreads) {
-    const int m = idx / R, rl = idx - m * R;
-    const int n = rb * kRowsPerCta + crank * R + rl;
+  // ---------------- epilogue: U units x 16 rows x M tokens ----------------
+  const int rows = U * kUnitRows;
+  const float s_w = sm.sw;
+  for (int idx = threadIdx.x; idx < rows * M; idx += kThreads) {
+    const int m = idx / rows, rl = idx - m * rows;
+    const int n = u_begin * kUnitRows + rl;
     if (n >= N) continue;
-    int accv = 0;
-#pragma unroll
-    for (int r = 0; r < C; ++r) accv += sm.red[(r * R + rl) * 16 + m];
+    const int accv = acc_s[rl * NTOK + m] - sm.rsum[m];
     const float d = __fmul_rn(sm.sx[m], s_w);
     float y32 = __fdiv_rn(static_cast<float>(accv), d);
-    if (a.bias) y32 = __fadd_rn(y32, bf16_bits_to_f32(sm.bias[rl]));
+    if (a.bias) y32 = __fadd_rn(y32, bf16_bits_to_f32(bias_s[rl]));
     const size_t o = static_cast<size_t>(m) * N + n;
     a.y[o] = f32_to_bf16_bits(y32);
     if (a.acc_out) a.acc_out[o] = accv;
@@ -459,10 +531,10 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
 }
 
-template <int NT, int C>
-cudaError_t launch_c(const CUtensorMap& tm, const DecodeArgs& a, int row_blocks, size_t smem,
-                     cudaStream_t stream) {
-  auto kern = decode_kernel<NT, C>;
+template <int NT>
+cudaError_t launch_nt(const CUtensorMap& tm3, const CUtensorMap& tm2, const DecodeArgs& a, const DecodePlan& p,
+                      cudaStream_t stream) {
+  auto kern = decode_kernel<NT>;
   static bool attr_done = false;
   if (!attr_done) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
@@ -470,69 +542,67 @@ cudaError_t launch_c(const CUtensorMap& tm, const DecodeArgs& a, int row_blocks,
     attr_done = true;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(C, row_blocks, 1);
+  cfg.gridDim = dim3(p.grid, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
+  cfg.dynamicSmemBytes = p.smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = C;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, kern, tm, a);
-}
-
-template <int NT>
-cudaError_t launch_nt(const CUtensorMap& tm, const DecodeArgs& a, int C, int row_blocks, size_t smem,
-                      cudaStream_t stream) {
-  switch (C) {
-    case 1: return launch_c<NT, 1>(tm, a, row_blocks, smem, stream);
-    case 2: return launch_c<NT, 2>(tm, a, row_blocks, smem, stream);
-    case 4: return launch_c<NT, 4>(tm, a, row_blocks, smem, stream);
-    default: return launch_c<NT, 8>(tm, a, row_blocks, smem, stream);
-  }
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, tm3, tm2, a);
 }
 
 }  // namespace
 
 DecodePlan plan_decode(int M, int N, int K, int num_sms) {
   DecodePlan p;
-  const int nbox = (K + kBoxK - 1) / kBoxK;
-  p.row_blocks = (N + kRowsPerCta - 1) / kRowsPerCta;
-  const int ntok = M <= 8 ? 8 : 16;
-  auto fill = [&](int c) {
-    p.cluster = c;
-    p.boxes_per_cta = (nbox + c - 1) / c;
-    p.ring = p.boxes_per_cta < kMaxRing ? p.boxes_per_cta : kMaxRing;
-    p.smem = smem_bytes(ntok, p.ring, p.boxes_per_cta);
-  };
-  int C = 1;
-  fill(C);
-  // split K over a cluster until the grid covers the SMs and a CTA fits twice per SM
-  while (C < 8 && 2 * C <= nbox && (p.row_blocks * C < num_sms || p.smem > static_cast<size_t>(kSmemBudget))) {
-    C *= 2;
-    fill(C);
-  }
+  const int units_total = (N + kUnitRows - 1) / kUnitRows;
+  p.grid = units_total < num_sms ? units_total : num_sms;
+  if ((units_total + p.grid - 1) / p.grid > kMaxUnits) p.grid = (units_total + kMaxUnits - 1) / kMaxUnits;
+  p.units_max = (units_total + p.grid - 1) / p.grid;
+  const int F = K / kBoxK;
+  p.kc = F < kConsumerWarps ? F : kConsumerWarps;
+  p.tail = (K % kBoxK) != 0;
+  p.slot_bytes = static_cast<size_t>(p.kc + p.tail) * kSubBytes;
+  // shared-memory budget: two CTAs per SM for the 8-token kernel (the next
+  // kernel on the stream can start beside this one), one for 16 tokens
+  const long long budget = M <= 8 ? 110 * 1024 : 220 * 1024;
+  const long long room = budget - static_cast<long long>(smem_layout(M, 0, p.slot_bytes, p.units_max).total);
+  long long ring = room > 0 ? room / static_cast<long long>(p.slot_bytes) : 0;
+  ring = ring > kMaxRing ? kMaxRing : ring;
+  p.ring = ring < 2 ? 2 : static_cast<int>(ring);
+  p.smem = smem_layout(M, p.ring, p.slot_bytes, p.units_max).total;
   return p;
 }
 
 cudaError_t launch_decode(DecodeArgs a, int num_sms, cudaStream_t stream) {
   if (a.M <= 0) return cudaSuccess;
   const DecodePlan p = plan_decode(a.M, a.N, a.K, num_sms);
-  a.boxes_per_cta = p.boxes_per_cta;
   a.ring = p.ring;
-  a.xs_stride = p.boxes_per_cta * kBoxK + 16;
+  a.units_max = p.units_max;
+  a.kc = p.kc;
+  a.tail = p.tail;
   if (p.smem > 227 * 1024) return cudaErrorInvalidValue;
-  CUtensorMap tm;
-  if (!encode_2d_u8(&tm, a.packed, static_cast<uint64_t>(a.K) / 4, static_cast<uint64_t>(a.N),
-                    static_cast<uint64_t>(a.K) / 4, kBoxK / 4, kRowsPerCta, CU_TENSOR_MAP_SWIZZLE_128B))
+  // 2-D view [N][K/4] bytes: the partial last chunk (and the 3-D map's stand-in when K < 512)
+  CUtensorMap tm2, tm3;
+  if (!encode_2d_u8(&tm2, a.packed, static_cast<uint64_t>(a.K) / 4, static_cast<uint64_t>(a.N),
+                    static_cast<uint64_t>(a.K) / 4, kBoxK / 4, kUnitRows, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  return a.M <= 8 ? launch_nt<1>(tm, a, p.cluster, p.row_blocks, p.smem, stream)
-                  : launch_nt<2>(tm, a, p.cluster, p.row_blocks, p.smem, stream);
+  tm3 = tm2;
+  if (p.kc > 0) {
+    // 3-D view [full chunk][row][128 bytes]: a box is kc consecutive 512-k
+    // chunks of 16 rows, each chunk landing as its own 16 x 128-byte sub-box
+    const uint64_t dims[3] = {static_cast<uint64_t>(kBoxK / 4), static_cast<uint64_t>(a.N),
+                              static_cast<uint64_t>(a.K / kBoxK)};
+    const uint64_t strides[2] = {static_cast<uint64_t>(a.K) / 4, static_cast<uint64_t>(kBoxK / 4)};
+    const uint32_t box[3] = {static_cast<uint32_t>(kBoxK / 4), static_cast<uint32_t>(kUnitRows),
+                             static_cast<uint32_t>(p.kc)};
+    if (!encode_3d_u8(&tm3, a.packed, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  }
+  return a.M <= 8 ? launch_nt<1>(tm3, tm2, a, p, stream) : launch_nt<2>(tm3, tm2, a, p, stream);
 }
 
 }  // namespace bitlinear

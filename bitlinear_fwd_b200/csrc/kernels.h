@@ -12,6 +12,10 @@ namespace bitlinear {
 // ---- TMA tensor maps (tensor_map.cu) ---------------------------------------
 bool encode_2d_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
                   uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle);
+// 3-D map: dims[0] innermost (contiguous bytes), strides in bytes of dims 1
+// and 2 (multiples of 16), box dims <= 256 each.
+bool encode_3d_u8(CUtensorMap* map, const void* base, const uint64_t dims[3], const uint64_t strides[2],
+                  const uint32_t box[3], CUtensorMapSwizzle swizzle);
 
 // ---- activation quantisation (act_quant.cu) --------------------------------
 // pdl: launch as a programmatic dependent of the previous kernel on the stream
@@ -56,18 +60,18 @@ struct DecodeArgs {
   const float* w_scale;   // [1]
   const uint16_t* bias;   // [N] or null
   uint16_t* y;            // [M, N]
-  int8_t* xq_out;         // [M, K] or null (debug, fused path)
-  float* sx_out;          // [M] or null (debug, fused path)
+  int8_t* xq_out;         // [M, K] or null (debug, quantising path)
+  float* sx_out;          // [M] or null (debug, quantising path)
   int32_t* acc_out;       // [M, N] or null (debug)
   float* y32_out;         // [M, N] or null (debug)
   uint32_t* status;       // status word or null
   int M, N, K;
-  int boxes_per_cta, ring, xs_stride;   // set by launch_decode
-  int weights_early;      // the packed weights may be read before the dependency wait
+  int ring, units_max, kc, tail;  // set by launch_decode
+  int weights_early;      // the packed weights, w_scale and bias may be read before the dependency wait
 };
 struct DecodePlan {
-  int cluster, boxes_per_cta, ring, row_blocks;
-  size_t smem;
+  int grid, units_max, ring, kc, tail;
+  size_t slot_bytes, smem;
 };
 DecodePlan plan_decode(int M, int N, int K, int num_sms);
 cudaError_t launch_decode(DecodeArgs a, int num_sms, cudaStream_t stream);

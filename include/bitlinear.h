@@ -135,12 +135,12 @@ int bitlinear_forward(const uint16_t* x, int64_t M, int64_t K, const uint8_t* pa
 
 /* Flags of bitlinear_forward_ex. */
 #define BITLINEAR_WEIGHTS_RESIDENT 1u
-/*   packed_w (and w_scale) were completely written before the operation
+/*   packed_w, w_scale and bias were completely written before the operation
  *   enqueued on `stream` just ahead of this call started -- e.g. weights
  *   packed once at load time.  The decode engine may then start streaming
- *   the weights while that operation is still finishing (programmatic
- *   dependent launch), which overlaps consecutive layers.  Never set it when
- *   the previous operation on the stream writes packed_w or w_scale. */
+ *   them while that operation is still finishing (programmatic dependent
+ *   launch), which overlaps consecutive layers.  Never set it when the
+ *   previous operation on the stream writes packed_w, w_scale or bias. */
 
 /* bitlinear_forward with flags (0 = identical to bitlinear_forward). */
 int bitlinear_forward_ex(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed_w, int64_t N,

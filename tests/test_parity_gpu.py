@@ -92,6 +92,8 @@ def test_w5_ffn100b(M):
 EDGE = [
     (17, 256, 64), (129, 300, 192), (1, 1, 64), (16, 517, 320), (33, 1000, 640),
     (2, 130, 128), (9, 129, 448), (300, 520, 1088), (16, 8, 64), (255, 777, 2112),
+    # K above the decode engine's 8192-k activation chunk, with a ragged last chunk
+    (5, 97, 17472), (12, 40, 8640),
 ]
 
 
