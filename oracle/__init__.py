@@ -38,6 +38,10 @@ design notes):
   it) stores code u+1 in {0,1,2}; row n of the packed matrix is K/16
   little-endian uint32 words; word g holds k = 16g + 4i + j in bits
   8j + 2i .. 8j + 2i + 1 (byte j, bit pair i).  Code 3 is invalid.
+* The bf16 export of the state-dict loop (``param_value / param_scale``)
+  divides in float32 (the dtype of W) and rounds once to bfloat16 (RNE).
+  It starts from the packed codes, so a zero is +0: ``round()`` can give
+  -0.0 for small negative weights, and two bits do not keep that sign.
 
 Every function here is pinned by ``tests/test_oracle_pins.py`` against
 things other than itself: a hand-worked example, exact rational arithmetic,
@@ -273,3 +277,19 @@ def forward(x_bits: np.ndarray, packed: np.ndarray, s_w: np.float32, bias_bits=N
     acc = contract(q, u)
     y32, y = epilogue(acc, s_x, s_w, bias_bits)
     return {"q": q, "s_x": s_x, "rowsum": rowsum, "acc": acc, "y32": y32, "y": y}
+
+
+# ---------------------------------------------------------------------------
+# bf16 export of the ternary weights
+# ---------------------------------------------------------------------------
+
+def dequant(packed: np.ndarray, s_w: np.float32, K: int | None = None) -> np.ndarray:
+    """[FE-univ] state-dict loop: ``param_value = u / param_scale``, stored
+    as bfloat16.  u comes from the packed codes; u / s_w is rounded to float32
+    once, then to bfloat16 (RNE).  Returns uint16 bf16 bits [N, K]."""
+    u = unpack(packed, K).astype(np.int64)
+    num, den = np.float64(np.float32(s_w)).as_integer_ratio()   # s_w = num / den exactly
+    inv = round_to_f32(den, num)                                  # RN_f32(1 / s_w)
+    w32 = np.where(u > 0, inv, np.where(u < 0, -inv, np.float32(0.0))).astype(np.float32)
+    return f32_to_bf16_rne(w32)
+

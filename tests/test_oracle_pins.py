@@ -360,3 +360,42 @@ def test_pins_catch_planted_mistakes(golden_dir, monkeypatch):
                 test_pack_layout_fixture(golden_dir)
         monkeypatch.undo()
     check_hand_worked(golden_dir)
+
+
+# --------------------------------------------------------------------------
+# bf16 export (state-dict loop: param_value / param_scale, stored as bf16)
+# --------------------------------------------------------------------------
+
+def test_dequant_hand_worked():
+    # s_w = 50: 1/50 = 0.02; the float32 nearest to 0.02 is 0x3CA3D70A; its
+    # upper half 0x3CA3 with 0xD70A > 0x8000 below rounds up to bf16 0x3CA4.
+    u = np.array([[1, 0, -1, 1, -1, 0, 0, 1, 1, 1, -1, -1, 0, 1, 0, -1]], dtype=np.int8)
+    got = oracle.dequant(oracle.pack(u), np.float32(50.0))
+    want = np.array([{1: 0x3CA4, 0: 0x0000, -1: 0xBCA4}[int(v)] for v in u[0]], dtype=np.uint16)
+    assert np.array_equal(got[0], want)
+
+
+def test_dequant_against_exact_rationals():
+    # for arbitrary float32 scales the exported +-1 weight is the bf16 nearest
+    # to the float32 nearest to 1/s_w, computed here from fractions
+    for s in RNG.uniform(0.5, 4000.0, size=200).astype(np.float32).tolist() + [1e5, 1.0, 3.0, 1e-3]:
+        s32 = np.float32(s)
+        inv = nearest_f32(Fraction(1) / f32_exact(s32))
+        pos = nearest_bf16_bits(inv)
+        u = np.array([[1, -1, 0, 0] * 4], dtype=np.int8)
+        got = oracle.dequant(oracle.pack(u), s32)[0]
+        assert int(got[0]) == pos and int(got[1]) == (pos ^ 0x8000) and int(got[2]) == 0, s
+
+
+def test_dequant_invariants_on_packed_weights():
+    w = synth.normal_f32(7, 1, (48, 320), 0.02)
+    packed, s_w, _ = oracle.pack_weights(w.numpy())
+    u = oracle.unpack(packed)
+    deq = oracle.dequant(packed, s_w)
+    assert deq.shape == u.shape and deq.dtype == np.uint16
+    assert np.all(deq[u == 0] == 0)                          # +0, never -0
+    mags = np.unique(deq[u != 0] & 0x7FFF)
+    assert mags.size == 1                                    # one magnitude, 1/s_w
+    assert np.all((deq[u > 0] >> 15) == 0) and np.all((deq[u < 0] >> 15) == 1)
+    v = float(oracle.bf16_to_f32(mags.astype(np.uint16))[0])
+    assert abs(v * float(s_w) - 1.0) < 2.0 ** -8              # bf16 keeps 8 significant bits
