@@ -279,6 +279,26 @@ def forward(x_bits: np.ndarray, packed: np.ndarray, s_w: np.float32, bias_bits=N
     return {"q": q, "s_x": s_x, "rowsum": rowsum, "acc": acc, "y32": y32, "y": y}
 
 
+def forward_grouped(x_bits: np.ndarray, packed: np.ndarray, group_rows, s_ws, bias_bits=None,
+                    K: int | None = None):
+    """Several BitLinear layers that read the same input (q/k/v, gate/up):
+    [FE-univ] BitLinear.forward applied to each group of rows of the stacked
+    packed matrix with that group's scale; the outputs side by side in one
+    [M, sum(rows)] array.  Returns the same dict as ``forward``."""
+    q, s_x, rowsum = act_quant(x_bits)
+    u = unpack(packed, K)
+    acc = contract(q, u)
+    y32 = np.empty(acc.shape, np.float32)
+    y = np.empty(acc.shape, np.uint16)
+    off = 0
+    for rows, s_w in zip(group_rows, s_ws):
+        b = None if bias_bits is None else bias_bits[off:off + rows]
+        y32[:, off:off + rows], y[:, off:off + rows] = epilogue(acc[:, off:off + rows], s_x, s_w, b)
+        off += rows
+    assert off == acc.shape[1]
+    return {"q": q, "s_x": s_x, "rowsum": rowsum, "acc": acc, "y32": y32, "y": y}
+
+
 # ---------------------------------------------------------------------------
 # bf16 export of the ternary weights
 # ---------------------------------------------------------------------------

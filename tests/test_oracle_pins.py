@@ -399,3 +399,38 @@ def test_dequant_invariants_on_packed_weights():
     assert np.all((deq[u > 0] >> 15) == 0) and np.all((deq[u < 0] >> 15) == 1)
     v = float(oracle.bf16_to_f32(mags.astype(np.uint16))[0])
     assert abs(v * float(s_w) - 1.0) < 2.0 ** -8              # bf16 keeps 8 significant bits
+
+
+# --------------------------------------------------------------------------
+# Grouped forward (layers sharing one input)
+# --------------------------------------------------------------------------
+
+def test_grouped_forward_scaled_copy_closed_form():
+    # Group 2 holds 2*W of group 1: same ternary codes, mean doubled, so
+    # s_w2 = s_w1 / 2 exactly, and y2 = acc / (s_x * s_w1 / 2) = 2 * y1.
+    # Doubling commutes with float32 and bf16 rounding, so every nonzero
+    # bf16 output of group 2 has the exponent of group 1's plus one.
+    w1 = synth.normal_f32(41, 3, (24, 128), 0.02).numpy()
+    p1, s1, _ = oracle.pack_weights(w1)
+    p2, s2, _ = oracle.pack_weights(2.0 * w1)
+    assert np.array_equal(p1, p2) and s2 == np.float32(s1 / 2)
+    x = synth.normal_bf16(41, 4, (5, 128))
+    xb = synth.bf16_bits(x)
+    out = oracle.forward_grouped(xb, np.concatenate([p1, p2]), [24, 24], [s1, s2])
+    y1, y2 = out["y"][:, :24].astype(np.int32), out["y"][:, 24:].astype(np.int32)
+    nz = (y1 & 0x7FFF) != 0
+    assert np.array_equal(y2[nz], y1[nz] + (1 << 7))          # exponent field + 1
+    assert np.array_equal(y2[~nz], y1[~nz])
+    # and group 1 alone is the single-layer forward
+    assert np.array_equal(out["y"][:, :24], oracle.forward(xb, p1, s1)["y"])
+
+
+def test_grouped_forward_acc_is_one_integer_matmul():
+    # the contraction of all groups at once is the integer product with the
+    # stacked ternary matrix, whatever the group split
+    u = RNG.integers(-1, 2, size=(40, 64)).astype(np.int8)
+    x = synth.normal_bf16(42, 1, (3, 64))
+    xb = synth.bf16_bits(x)
+    out = oracle.forward_grouped(xb, oracle.pack(u), [7, 30, 3], [np.float32(1.5), np.float32(2.0), np.float32(0.25)])
+    q = oracle.act_quant(xb)[0].astype(np.int64)
+    assert np.array_equal(out["acc"], (q @ u.astype(np.int64).T).astype(np.int32))
