@@ -384,6 +384,113 @@ def run_prefill(args, bf16_tflops, peak_kind, l2_bytes):
 
 # ---------------------------------------------------------------------------
 # the CPU oracle (cpu_baseline and the reference arm)
+def _random_packed(N, K, gen):
+    """Packed ternary rows with valid codes (each 2-bit field in {0, 1, 2})."""
+    lut = torch.tensor([a | (b << 2) | (c << 4) | (d << 6) for a in range(3) for b in range(3)
+                        for c in range(3) for d in range(3)], dtype=torch.uint8, device="cuda")
+    return lut[torch.randint(0, 81, (N, K // 4), device="cuda", generator=gen)]
+
+
+def run_stack3b(hbm_gbs, M=1, layers=26, reps=20):
+    """The 3B-class decoder projection stack at M tokens: per layer q/k/v
+    (3200 -> 3 x 3200), o (3200 -> 3200), gate/up (3200 -> 2 x 8640), down
+    (8640 -> 3200); 26 layers of independent weights (806 MB packed).
+    Timed two ways: one bitlinear_forward per projection (7 launches per
+    layer) and with the shared-input groups fused (q/k/v and gate/up through
+    bitlinear_forward_grouped: 4 launches per layer).  Weights resident,
+    replayed as one CUDA graph per pass."""
+    import bitlinear_fwd_b200 as bl
+    H, F = 3200, 8640
+    gen = torch.Generator(device="cuda").manual_seed(21)
+    lay = []
+    for _ in range(layers):
+        L = {"qkv": _random_packed(3 * H, H, gen), "o": _random_packed(H, H, gen),
+             "gu": _random_packed(2 * F, H, gen), "down": _random_packed(H, F, gen)}
+        L["s3"] = torch.full((3,), 40.0, device="cuda")              # stacked, for the grouped calls
+        L["s2"] = torch.full((2,), 40.0, device="cuda")
+        L["s1"] = [torch.full((1,), 40.0, device="cuda") for _ in range(5)]   # one per separate call
+        lay.append(L)
+    x = (torch.randn((M, H), device="cuda", generator=gen)).to(torch.bfloat16)
+    xf = (torch.randn((M, F), device="cuda", generator=gen)).to(torch.bfloat16)
+    y3 = torch.empty((M, 3 * H), dtype=torch.bfloat16, device="cuda")
+    yo = torch.empty((M, H), dtype=torch.bfloat16, device="cuda")
+    y2 = torch.empty((M, 2 * F), dtype=torch.bfloat16, device="cuda")
+    ws = bl.workspace(M, 2 * F, F, "cuda")
+    R = bl.WEIGHTS_RESIDENT
+
+    def grouped():
+        for L in lay:
+            bl.bitlinear_forward_grouped(x, L["qkv"], [H, H, H], L["s3"], ws=ws, out=y3, flags=R)
+            bl.bitlinear_forward(x, L["o"], L["s3"][:1], ws=ws, out=yo, flags=R)
+            bl.bitlinear_forward_grouped(x, L["gu"], [F, F], L["s2"], ws=ws, out=y2, flags=R)
+            bl.bitlinear_forward(xf, L["down"], L["s2"][:1], ws=ws, out=yo, flags=R)
+
+    def separate():
+        for L in lay:
+            for g in range(3):
+                bl.bitlinear_forward(x, L["qkv"][g * H:(g + 1) * H], L["s1"][g], ws=ws,
+                                     out=y3[:, g * H:(g + 1) * H] if M == 1 else None, flags=R)
+            bl.bitlinear_forward(x, L["o"], L["s3"][:1], ws=ws, out=yo, flags=R)
+            for g in range(2):
+                bl.bitlinear_forward(x, L["gu"][g * F:(g + 1) * F], L["s1"][3 + g], ws=ws,
+                                     out=y2[:, g * F:(g + 1) * F] if M == 1 else None, flags=R)
+            bl.bitlinear_forward(xf, L["down"], L["s2"][:1], ws=ws, out=yo, flags=R)
+
+    out = {"workload": f"3B-class projection stack, {layers} layers, M={M}", "layers": layers, "M": M}
+    wbytes = layers * (3 * H * H + H * H + 2 * F * H + H * F) // 4
+    for name, fn, launches in (("grouped", grouped, 4), ("separate", separate, 7)):
+        fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            g.replay()
+        e1.record()
+        e1.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / reps
+        out[name] = {"us_per_pass": round(us, 1), "tokens_per_s": round(M / (us * 1e-6), 1),
+                     "weights_gbs": round(wbytes / (us * 1e-6) / 1e9, 1),
+                     "frac_of_hbm": round(wbytes / (us * 1e-6) / 1e9 / hbm_gbs, 4),
+                     "launches_per_pass": launches * layers}
+        del g
+    out["weights_bytes_per_pass"] = wbytes
+    return out
+
+
+def run_dequant(hbm_gbs, reps=20):
+    """bf16 export of packed weights at the 100B-class gate/up shape (28672 x
+    8192): 0.25 B read + 2 B written per weight, against the HBM copy peak."""
+    import bitlinear_fwd_b200 as bl
+    N, K = 28672, 8192
+    g = torch.Generator(device="cuda").manual_seed(11)
+    packed = torch.randint(0, 256, (N, K // 4), dtype=torch.uint8, device="cuda", generator=g)
+    s_w = torch.full((1,), 50.0, device="cuda")
+    out = torch.empty((N, K), dtype=torch.bfloat16, device="cuda")
+    lib, st = bl.lib(), torch.cuda.current_stream().cuda_stream
+    call = lambda: lib.bitlinear_dequant_weights(packed.data_ptr(), N, K, s_w.data_ptr(), out.data_ptr(), st)
+    for _ in range(3):
+        assert call() == 0
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        call()
+    e1.record()
+    e1.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / reps
+    nbytes = N * K // 4 + 2 * N * K
+    gbs = nbytes / (us * 1e-6) / 1e9
+    return {"kernel": "dequant_kernel", "shape": [N, K], "us_per_launch": round(us, 2),
+            "bytes_per_launch": nbytes, "achieved": round(gbs, 1), "unit": "GB/s", "peak": hbm_gbs,
+            "frac": round(gbs / hbm_gbs, 4), "note": "output 470 MB > L2, each launch streams it to DRAM"}
+
+
 # ---------------------------------------------------------------------------
 
 class OracleDecode:
@@ -464,7 +571,7 @@ def main():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--only", choices=["decode", "prefill"], default=None,
+    ap.add_argument("--only", choices=["decode", "prefill", "dequant", "stack3b"], default=None,
                     help="run one workload only (profiling runs; no JSON contract line)")
     ap.add_argument("--copies", type=int, default=0, help="force the number of rotating weight copies")
     args = ap.parse_args()
@@ -489,6 +596,12 @@ def main():
     if args.only == "prefill":
         print(json.dumps(run_prefill(args, bf16_tflops, peak_kind, l2_bytes)), flush=True)
         return 0
+    if args.only == "stack3b":
+        print(json.dumps(run_stack3b(hbm_gbs)), flush=True)
+        return 0
+    if args.only == "dequant":
+        print(json.dumps(run_dequant(hbm_gbs)), flush=True)
+        return 0
     if args.only == "decode":
         d = run_decode(args, hbm_gbs, l2_bytes, peak_kind)
         print(json.dumps({"value": d["value"], "ms": d["ms"], "roofline": d["roofline"]}), flush=True)
@@ -498,6 +611,8 @@ def main():
     clocks = sampler.stop()
     e2e = None if args.no_e2e else run_e2e(args, dec["probs"], max(3, min(200, args.steps // 10)))
     pre = None if args.no_prefill else run_prefill(args, bf16_tflops, peak_kind, l2_bytes)
+    deq = run_dequant(hbm_gbs)
+    stack = run_stack3b(hbm_gbs)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -534,6 +649,8 @@ def main():
         "gpu_launches": dec["launches_per_step"] * args.steps,
         "e2e": e2e,
         "prefill": pre,
+        "dequant_export": deq,
+        "stack3b_decode": stack,
         "cpu_baseline": cpu,
         "clocks": clocks,
     }

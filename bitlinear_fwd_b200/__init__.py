@@ -31,6 +31,9 @@ _SIGS = {
     "bitlinear_host_workspace_bytes": (_c_sz, [_c_i64, _c_i64, _c_i64]),
     "bitlinear_pack_weights": (ctypes.c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_p, _c_p, _c_p, _c_sz, _c_p]),
     "bitlinear_quant_act": (ctypes.c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_p, _c_p, _c_p]),
+    "bitlinear_dequant_weights": (ctypes.c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_p, _c_p]),
+    "bitlinear_forward_grouped": (ctypes.c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_p, ctypes.c_int, _c_p, _c_p, _c_p,
+                                                 ctypes.c_uint, _c_p, ctypes.c_size_t, _c_p]),
     "bitlinear_forward": (ctypes.c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_i64, _c_p, _c_p, _c_p, _c_p, _c_sz,
                                          _c_p]),
     "bitlinear_forward_ex": (ctypes.c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_i64, _c_p, _c_p, _c_p, ctypes.c_uint,
@@ -148,6 +151,15 @@ def bitlinear_quant_act(x: torch.Tensor):
     return xq, s_x, rs
 
 
+def bitlinear_dequant_weights(packed: torch.Tensor, w_scale: torch.Tensor) -> torch.Tensor:
+    """bf16 export of packed weights: w [N, K] bf16 = u / s_w (zeros +0)."""
+    N, K = packed.shape[0], packed.shape[1] * 4
+    out = torch.empty((N, K), dtype=torch.bfloat16, device=packed.device)
+    _check(lib().bitlinear_dequant_weights(_ptr(packed), N, K, _ptr(w_scale), _ptr(out), _stream(packed.device)),
+           "bitlinear_dequant_weights")
+    return out
+
+
 WEIGHTS_RESIDENT = 1
 
 
@@ -170,6 +182,28 @@ def bitlinear_forward(x: torch.Tensor, packed: torch.Tensor, w_scale: torch.Tens
     else:
         _check(lib().bitlinear_forward(_ptr(x), M, K, _ptr(packed), N, _ptr(w_scale), _ptr(b), _ptr(y),
                                        _ptr(ws), ws.numel(), _stream(x.device)), "bitlinear_forward")
+    return y
+
+
+MAX_GROUPS = 8
+
+
+def bitlinear_forward_grouped(x: torch.Tensor, packed: torch.Tensor, group_rows, w_scales: torch.Tensor,
+                              bias: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                              out: Optional[torch.Tensor] = None, flags: int = 0) -> torch.Tensor:
+    """Layers sharing the input x (q/k/v, gate/up): packed [N, K/4] stacked row-wise,
+    group_rows their row counts, w_scales [G] f32.  Returns y bf16 [M, N], layer g in
+    its own column block."""
+    x = _bits(x)
+    M, K = x.shape
+    N = packed.shape[0]
+    rows = (ctypes.c_int64 * len(group_rows))(*[int(r) for r in group_rows])
+    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    if ws is None:
+        ws = workspace(M, N, K, x.device)
+    _check(lib().bitlinear_forward_grouped(_ptr(x), M, K, _ptr(packed), rows, len(group_rows), _ptr(w_scales),
+                                           _ptr(bias), _ptr(y), flags, _ptr(ws), ws.numel(), _stream(x.device)),
+           "bitlinear_forward_grouped")
     return y
 
 

@@ -76,10 +76,24 @@ int status_of(cudaError_t e) { return e == cudaSuccess ? BITLINEAR_OK : BITLINEA
 // earlier write to the packed weights is complete before they are read --
 // unless BITLINEAR_WEIGHTS_RESIDENT is set, which lets the forward start
 // streaming weights while the previous kernel on the stream finishes.
-int forward_impl(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed_w, int64_t N,
-                 const float* w_scale, const uint16_t* bias, uint16_t* y, int8_t* xq_out, float* sx_out,
-                 int32_t* acc_out, float* y32_out, int engine, unsigned flags, void* ws, size_t ws_bytes,
-                 cudaStream_t stream) {
+static_assert(BITLINEAR_MAX_GROUPS == kMaxGroups, "header and kernels agree on the group limit");
+
+struct Groups {
+  int n;
+  int end[kMaxGroups];
+};
+
+Groups single_group(int64_t N) {
+  Groups g{};
+  g.n = 1;
+  g.end[0] = int(N);
+  return g;
+}
+
+int forward_impl_g(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed_w, int64_t N,
+                   const float* w_scale, const uint16_t* bias, uint16_t* y, int8_t* xq_out, float* sx_out,
+                   int32_t* acc_out, float* y32_out, int engine, unsigned flags, void* ws, size_t ws_bytes,
+                   cudaStream_t stream, const Groups& grp) {
   (void)ws_bytes;
   int sms = 148;
   int st = check_device(&sms);
@@ -108,6 +122,8 @@ int forward_impl(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed_
     d.N = int(N);
     d.K = int(K);
     d.weights_early = resident ? 1 : 0;
+    d.ngroups = grp.n;
+    for (int g = 0; g < kMaxGroups; ++g) d.group_end[g] = grp.end[g];
     return status_of(launch_decode(d, sms, stream));
   }
   float* s_x = reinterpret_cast<float*>(base + L.off_sx);
@@ -130,11 +146,21 @@ int forward_impl(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed_
   a.N = int(N);
   a.K = int(K);
   a.pdl = true;
+  a.ngroups = grp.n;
+  for (int g = 0; g < kMaxGroups; ++g) a.group_end[g] = grp.end[g];
   e = launch_gemm_prefill(a, sms, stream);
   if (e != cudaSuccess) return BITLINEAR_ERR_CUDA;
   if (xq_out) e = cudaMemcpyAsync(xq_out, xq, size_t(M) * size_t(K), cudaMemcpyDeviceToDevice, stream);
   if (e == cudaSuccess && sx_out) e = cudaMemcpyAsync(sx_out, s_x, 4 * size_t(M), cudaMemcpyDeviceToDevice, stream);
   return status_of(e);
+}
+
+int forward_impl(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed_w, int64_t N,
+                 const float* w_scale, const uint16_t* bias, uint16_t* y, int8_t* xq_out, float* sx_out,
+                 int32_t* acc_out, float* y32_out, int engine, unsigned flags, void* ws, size_t ws_bytes,
+                 cudaStream_t stream) {
+  return forward_impl_g(x, M, K, packed_w, N, w_scale, bias, y, xq_out, sx_out, acc_out, y32_out, engine, flags, ws,
+                        ws_bytes, stream, single_group(N));
 }
 
 int check_forward_args(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed_w, int64_t N,
@@ -243,6 +269,29 @@ int bitlinear_forward_ex(const uint16_t* x, int64_t M, int64_t K, const uint8_t*
                       ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
+int bitlinear_forward_grouped(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed_w,
+                              const int64_t* group_rows, int groups, const float* w_scales, const uint16_t* bias,
+                              uint16_t* y, unsigned flags, void* ws, size_t ws_bytes, void* stream) {
+  if (flags & ~static_cast<unsigned>(BITLINEAR_WEIGHTS_RESIDENT)) return BITLINEAR_ERR_SHAPE;
+  if (!group_rows) return BITLINEAR_ERR_NULL;
+  if (groups < 1 || groups > BITLINEAR_MAX_GROUPS) return BITLINEAR_ERR_SHAPE;
+  Groups grp{};
+  grp.n = groups;
+  int64_t N = 0;
+  for (int g = 0; g < groups; ++g) {
+    if (group_rows[g] < 1) return BITLINEAR_ERR_SHAPE;
+    N += group_rows[g];
+    if (N > kMaxMN) return BITLINEAR_ERR_SHAPE;
+    grp.end[g] = int(N);
+  }
+  int st = check_forward_args(x, M, K, packed_w, N, w_scales, bias, y, ws, ws_bytes,
+                              bitlinear_workspace_bytes(M, N, K), false);
+  if (st != BITLINEAR_OK) return st;
+  if (M == 0) return BITLINEAR_OK;
+  return forward_impl_g(x, M, K, packed_w, N, w_scales, bias, y, nullptr, nullptr, nullptr, nullptr, 0, flags, ws,
+                        ws_bytes, static_cast<cudaStream_t>(stream), grp);
+}
+
 int bitlinear_forward_q8(const int8_t* xq, const float* x_scale, const int32_t* xq_rowsum, int64_t M,
                          int64_t K, const uint8_t* packed_w, int64_t N, const float* w_scale,
                          const uint16_t* bias, uint16_t* y, void* ws, size_t ws_bytes, void* stream) {
@@ -273,6 +322,8 @@ int bitlinear_forward_q8(const int8_t* xq, const float* x_scale, const int32_t* 
   a.N = int(N);
   a.K = int(K);
   a.pdl = false;
+  a.ngroups = 1;
+  a.group_end[0] = int(N);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (M > 16) return status_of(launch_gemm_prefill(a, sms, s));
   // the previous operation on the stream is unknown: read the weights only
@@ -294,7 +345,21 @@ int bitlinear_forward_q8(const int8_t* xq, const float* x_scale, const int32_t* 
   d.N = int(N);
   d.K = int(K);
   d.weights_early = 0;
+  d.ngroups = 1;
+  d.group_end[0] = int(N);
   return status_of(launch_decode(d, sms, s));
+}
+
+int bitlinear_dequant_weights(const uint8_t* packed_w, int64_t N, int64_t K, const float* w_scale,
+                              uint16_t* w_bf16, void* stream) {
+  int st = check_shape(1, N, K);
+  if (st != BITLINEAR_OK) return st;
+  if (!packed_w || !w_scale || !w_bf16) return BITLINEAR_ERR_NULL;
+  if (misaligned(packed_w) || misaligned(w_scale) || misaligned(w_bf16)) return BITLINEAR_ERR_ALIGN;
+  int sms = 148;
+  st = check_device(&sms);
+  if (st != BITLINEAR_OK) return st;
+  return status_of(launch_dequant(packed_w, N, K, w_scale, w_bf16, sms, static_cast<cudaStream_t>(stream)));
 }
 
 int bitlinear_forward_debug(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed_w, int64_t N,

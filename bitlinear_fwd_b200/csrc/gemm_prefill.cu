@@ -21,7 +21,8 @@
 //                of four consecutive k) and one tcgen05.st of 32 columns
 //   warps 8..11  epilogue of the previous tile while the MMAs of the next one
 //                run: tcgen05.ld of a row's 128 accumulators, acc - sum_k q
-//                (code offset), y = acc / (s_x s_w) (+ bias), bf16 stores
+//                (code offset), y = acc / (s_x s_w) (+ bias), bf16 stores;
+//                s_w is the scale of the row's group (stacked layers)
 //                (coalesced along weight rows)
 // Barriers: per stage full (TMA bytes landed), ready (A stage written),
 // empty (MMAs done); per accumulator buffer acc_full (tile's MMAs done) and
@@ -50,7 +51,7 @@ constexpr uint32_t kCodeMask = 0x03030303u;
 
 constexpr uint32_t kOffX = 0;
 constexpr uint32_t kOffWp = kOffX + STAGES * kXBytes;
-constexpr uint32_t kOffD = kOffWp + STAGES * kWpBytes;       // s_x * s_w per token [BT]
+constexpr uint32_t kOffD = kOffWp + STAGES * kWpBytes;       // s_x per token [BT]
 constexpr uint32_t kOffRs = kOffD + 4 * BT;                  // row sums per token [BT]
 constexpr uint32_t kOffBar = kOffRs + 4 * BT;
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;        // + barriers, alignment slack
@@ -203,7 +204,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int et = threadIdx.x - 256;             // 0..127
     const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
     pdl_wait_primary();
-    const float s_w = *a.w_scale;
+    float swg[kMaxGroups];                         // s_w of each row group
+#pragma unroll
+    for (int g = 0; g < kMaxGroups; ++g) swg[g] = g < a.ngroups ? a.w_scale[g] : 0.0f;
     int j = 0;
     // The four epilogue warps meet at a named barrier twice per tile; every
     // one of them runs every iteration (a failure only skips work), so the
@@ -211,11 +214,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++j) {
       const int b = j & 1;
       const int n0 = (tile % wtiles) * BW, m0 = (tile / wtiles) * BT;
-      // per-token d = s_x * s_w and row sums of this tile
+      // per-token s_x and row sums of this tile
       asm volatile("bar.sync 1, 128;" ::: "memory");   // previous tile's readers are done
       {
         const int m = m0 + et;
-        d_s[et] = m < a.M ? __fmul_rn(a.s_x[m], s_w) : 1.0f;
+        d_s[et] = m < a.M ? a.s_x[m] : 1.0f;
         rs_s[et] = m < a.M ? a.rowsum[m] : 0;
       }
       asm volatile("bar.sync 1, 128;" ::: "memory");
@@ -230,6 +233,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int n = n0 + 32 * q + lane;
       const bool nv = n < a.N;
       const float bv = (a.bias && nv) ? bf16_bits_to_f32(a.bias[n]) : 0.0f;
+      float s_w = swg[0];                          // this row's group scale
+#pragma unroll
+      for (int g = 1; g < kMaxGroups; ++g)
+        if (g < a.ngroups && n >= a.group_end[g - 1]) s_w = swg[g];
 #pragma unroll 1
       for (int c = 0; c < BT / 32; ++c) {
         uint32_t r[32];
@@ -247,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int mi = 32 * c + i, m = m0 + mi;
           if (m >= a.M) continue;
           const int accv = static_cast<int>(r[i]) - rs_s[mi];
-          float y32 = __fdiv_rn(static_cast<float>(accv), d_s[mi]);
+          float y32 = __fdiv_rn(static_cast<float>(accv), __fmul_rn(d_s[mi], s_w));
           if (a.bias) y32 = __fadd_rn(y32, bv);
           const size_t o = static_cast<size_t>(m) * a.N + n;
           a.y[o] = f32_to_bf16_bits(y32);

@@ -142,7 +142,7 @@ struct SmemTail {
   uint32_t amax[16];                 // absmax per token (bf16 bits)
   int rsum[16];                      // sum of q per token
   float sx[16];                      // s_x per token
-  float sw;
+  float swg[kMaxGroups];             // s_w of each row group
   int issued;                        // loads issued (producer)
   int failed;                        // a wait of this CTA timed out
 };
@@ -222,8 +222,8 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
       const int n = u_begin * kUnitRows + i;
       bias_s[i] = (a.bias && n < N) ? a.bias[n] : static_cast<uint16_t>(0);
     }
+    if (lane < a.ngroups) sm.swg[lane] = a.w_scale[lane];
     if (lane == 0) {
-      sm.sw = *a.w_scale;
       int q = 0;
       for (int r = 0; r < nround && ok; ++r) {
         const bool has3 = kc > 0 && 8 * r < F;       // full chunks of this round, one 3-D load
@@ -515,13 +515,15 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
 
   // ---------------- epilogue: U units x 16 rows x M tokens ----------------
   const int rows = U * kUnitRows;
-  const float s_w = sm.sw;
   for (int idx = threadIdx.x; idx < rows * M; idx += kThreads) {
     const int m = idx / rows, rl = idx - m * rows;
     const int n = u_begin * kUnitRows + rl;
     if (n >= N) continue;
     const int accv = acc_s[rl * NTOK + m] - sm.rsum[m];
-    const float d = __fmul_rn(sm.sx[m], s_w);
+    int gi = 0;                                      // the row's group (scale)
+#pragma unroll
+    for (int g = 0; g + 1 < kMaxGroups; ++g) gi += (g + 1 < a.ngroups && n >= a.group_end[g]) ? 1 : 0;
+    const float d = __fmul_rn(sm.sx[m], sm.swg[gi]);
     float y32 = __fdiv_rn(static_cast<float>(accv), d);
     if (a.bias) y32 = __fadd_rn(y32, bf16_bits_to_f32(bias_s[rl]));
     const size_t o = static_cast<size_t>(m) * N + n;

@@ -36,20 +36,30 @@ cudaError_t launch_pack(const float* w, int64_t N, int64_t K, uint8_t* packed, f
                         float* w_mean, const PackWorkspace& pws, cudaStream_t stream);
 
 // ---- shared forward arguments ----------------------------------------------
+// Rows [group_end[g-1], group_end[g]) of the packed matrix form group g,
+// scaled by w_scale[g] (one group for a plain layer).
+constexpr int kMaxGroups = 8;
+
 struct ForwardArgs {
   const int8_t* xq;       // [M, K]
   const float* s_x;       // [M]
   const int32_t* rowsum;  // [M]
   const uint8_t* packed;  // [N, K/4]
-  const float* w_scale;   // [1]
+  const float* w_scale;   // [ngroups]
   const uint16_t* bias;   // [N] or null
   uint16_t* y;            // [M, N]
   int32_t* acc_out;       // [M, N] or null (debug)
   float* y32_out;         // [M, N] or null (debug)
   uint32_t* status;       // status word
   int M, N, K;
+  int ngroups;
+  int group_end[kMaxGroups];
   bool pdl;               // launched as a programmatic dependent of the act-quant kernel
 };
+
+// ---- bf16 export of packed weights (dequant.cu) ----------------------------
+cudaError_t launch_dequant(const uint8_t* packed, int64_t N, int64_t K, const float* w_scale, uint16_t* w_bf16,
+                           int num_sms, cudaStream_t stream);
 
 // ---- decode engine, M <= 16 (gemv_decode.cu) --------------------------------
 struct DecodeArgs {
@@ -57,7 +67,7 @@ struct DecodeArgs {
   const int8_t* xq;       // int8 [M, K] with s_x when x is null
   const float* s_x;       // [M]
   const uint8_t* packed;  // [N, K/4]
-  const float* w_scale;   // [1]
+  const float* w_scale;   // [ngroups]
   const uint16_t* bias;   // [N] or null
   uint16_t* y;            // [M, N]
   int8_t* xq_out;         // [M, K] or null (debug, quantising path)
@@ -66,6 +76,8 @@ struct DecodeArgs {
   float* y32_out;         // [M, N] or null (debug)
   uint32_t* status;       // status word or null
   int M, N, K;
+  int ngroups;
+  int group_end[kMaxGroups];
   int ring, units_max, kc, tail;  // set by launch_decode
   int weights_early;      // the packed weights, w_scale and bias may be read before the dependency wait
 };

@@ -147,6 +147,26 @@ int bitlinear_forward_ex(const uint16_t* x, int64_t M, int64_t K, const uint8_t*
                          const float* w_scale, const uint16_t* bias, uint16_t* y, unsigned flags, void* ws,
                          size_t ws_bytes, void* stream);
 
+/* Several BitLinear layers that read the same input in one call -- q/k/v,
+ * or gate/up (BitLinear.forward of the Falcon-Edge blog, once per layer):
+ * the input is quantised once and the layers' weights stream through one
+ * launch of the decode engine (M <= 16) or one GEMM (M > 16).
+ *   packed_w    [N, K/4] uint8: the layers' packed matrices stacked row-wise
+ *               (pack layer g into rows [row_g, row_g + group_rows[g]) with
+ *               bitlinear_pack_weights, its scale into w_scales[g])
+ *   group_rows  host array [groups] of row counts, each >= 1; N = their sum
+ *   groups      1 .. BITLINEAR_MAX_GROUPS
+ *   w_scales    [groups] float32 (device), s_w of each layer
+ *   bias        [N] bf16 (the layers' biases stacked) or NULL
+ *   y           [M, N] bf16 out: layer g's outputs are the columns
+ *               [row_g, row_g + group_rows[g])
+ *   flags, ws   as for bitlinear_forward_ex with this N.
+ * Each output equals the one bitlinear_forward gives for that layer alone. */
+#define BITLINEAR_MAX_GROUPS 8
+int bitlinear_forward_grouped(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed_w,
+                              const int64_t* group_rows, int groups, const float* w_scales, const uint16_t* bias,
+                              uint16_t* y, unsigned flags, void* ws, size_t ws_bytes, void* stream);
+
 /* The contraction and epilogue of the forward on activations that
  * bitlinear_quant_act has already quantised (so that several weight
  * matrices that read the same input -- q/k/v, gate/up -- quantise it once).
@@ -157,6 +177,17 @@ int bitlinear_forward_ex(const uint16_t* x, int64_t M, int64_t K, const uint8_t*
 int bitlinear_forward_q8(const int8_t* xq, const float* x_scale, const int32_t* xq_rowsum, int64_t M,
                          int64_t K, const uint8_t* packed_w, int64_t N, const float* w_scale,
                          const uint16_t* bias, uint16_t* y, void* ws, size_t ws_bytes, void* stream);
+
+/* bf16 export of packed ternary weights, for loading them into a plain bf16
+ * linear layer (Falcon-Edge blog, section "Falcon-Edge, a series of universal
+ * models": the state-dict loop param_value = u / param_scale stored as
+ * bfloat16).  w_bf16[n, k] = bf16_rne(float32(u[n, k] / s_w)); zeros are +0.
+ *   packed_w  [N, K/4] uint8 from bitlinear_pack_weights
+ *   w_scale   [1] float32 (device), s_w
+ *   w_bf16    [N, K] bf16 out (16-byte aligned), row-major
+ * Same shape rules as bitlinear_forward; no workspace. */
+int bitlinear_dequant_weights(const uint8_t* packed_w, int64_t N, int64_t K, const float* w_scale,
+                              uint16_t* w_bf16, void* stream);
 
 /* bitlinear_forward with intermediate outputs, for parity tests.  Same
  * kernels; each extra output may be NULL:

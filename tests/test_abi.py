@@ -77,3 +77,21 @@ def test_argument_errors_without_gpu(lib):
     assert lib.bitlinear_forward_debug(16, 32, 256, 16, 512, 16, None, 16, None, None, None, None, 1, 16,
                                        1 << 20, None) == -2               # decode engine needs M <= 16
     assert lib.bitlinear_check_status(None, 0, None) == -1
+    # bf16 export: shape, null and alignment checks come before any device work
+    assert lib.bitlinear_dequant_weights(16, 512, 100, 16, 16, None) == -2
+    assert lib.bitlinear_dequant_weights(16, 0, 256, 16, 16, None) == -2
+    assert lib.bitlinear_dequant_weights(None, 512, 256, 16, 16, None) == -1
+    assert lib.bitlinear_dequant_weights(16, 512, 256, None, 16, None) == -1
+    assert lib.bitlinear_dequant_weights(16, 512, 256, 16, 18, None) == -3
+    # grouped forward: group list checks come first
+    import ctypes
+    rows = (ctypes.c_int64 * 3)(100, 200, 212)
+    bad = (ctypes.c_int64 * 2)(100, 0)
+    g = lib.bitlinear_forward_grouped
+    assert g(16, 8, 256, 16, None, 3, 16, None, 16, 0, 16, 1 << 20, None) == -1    # no group list
+    assert g(16, 8, 256, 16, rows, 0, 16, None, 16, 0, 16, 1 << 20, None) == -2    # no groups
+    assert g(16, 8, 256, 16, rows, 9, 16, None, 16, 0, 16, 1 << 20, None) == -2    # too many groups
+    assert g(16, 8, 256, 16, bad, 2, 16, None, 16, 0, 16, 1 << 20, None) == -2     # empty group
+    assert g(16, 8, 256, 16, rows, 3, None, None, 16, 0, 16, 1 << 20, None) == -1  # no scales
+    assert g(16, 8, 256, 16, rows, 3, 16, None, 16, 2, 16, 1 << 20, None) == -2    # unknown flag
+    assert g(16, 8, 256, 16, rows, 3, 16, None, 16, 0, 16, 16, None) == -4         # workspace too small
