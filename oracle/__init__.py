@@ -38,6 +38,14 @@ design notes):
   it) stores code u+1 in {0,1,2}; row n of the packed matrix is K/16
   little-endian uint32 words; word g holds k = 16g + 4i + j in bits
   8j + 2i .. 8j + 2i + 1 (byte j, bit pair i).  Code 3 is invalid.
+* bf16-faithful mode (``*_bf16`` functions): the listings run on a bf16
+  module.  Every tensor op rounds its result to bf16; PyTorch computes
+  elementwise bf16 ops in float32 and rounds once to bf16.  PyTorch evaluates
+  ``127.0 / t`` as ``t.reciprocal() * 127.0`` (two roundings); the
+  float32 mode reads that formula as one division instead.  The weight scale
+  is the module's bf16 copy of s_w.  ``F.linear`` accumulates the exact
+  integer products and rounds the sum once to bf16.  ``clamp_(min=1e-5)``
+  bounds by bf16(1e-5).
 * The bf16 export of the state-dict loop (``param_value / param_scale``)
   divides in float32 (the dtype of W) and rounds once to bfloat16 (RNE).
   It starts from the packed codes, so a zero is +0: ``round()`` can give
@@ -296,6 +304,55 @@ def forward_grouped(x_bits: np.ndarray, packed: np.ndarray, group_rows, s_ws, bi
         y32[:, off:off + rows], y[:, off:off + rows] = epilogue(acc[:, off:off + rows], s_x, s_w, b)
         off += rows
     assert off == acc.shape[1]
+    return {"q": q, "s_x": s_x, "rowsum": rowsum, "acc": acc, "y32": y32, "y": y}
+
+
+# ---------------------------------------------------------------------------
+# bf16-faithful mode: the listings' dtype semantics on a bf16 module
+# ---------------------------------------------------------------------------
+
+def _bf16(v) -> np.ndarray:
+    """Round float32 values to bf16 (RNE) and widen back to float32."""
+    return bf16_to_f32(f32_to_bf16_rne(np.asarray(v, np.float32)))
+
+
+def act_quant_bf16(x_bits: np.ndarray):
+    """[FE-univ] activation_norm_quant on bf16 tensors, evaluated as PyTorch
+    does: ``127.0 / t`` is ``t.reciprocal() * 127.0``, so scale =
+    bf16(bf16(1 / max(a, bf16(1e-5))) * 127), then q = clamp(round(bf16(x *
+    scale)), -128, 127).
+    Returns (q int8 [M,K], s_x float32 [M] holding bf16 values, rowsum int32)."""
+    x = bf16_to_f32(x_bits)
+    M, K = x.shape
+    if M == 0:
+        return np.zeros((0, K), np.int8), np.zeros(0, np.float32), np.zeros(0, np.int32)
+    a = np.abs(x).max(axis=1)
+    s_x = _bf16(_bf16(F32(1.0) / np.maximum(a, _bf16(CLAMP_MIN))) * F32(QMAX))
+    t = _bf16(x * s_x[:, None])                 # bf16 * bf16 is exact in float32, then one rounding
+    q = np.clip(np.rint(t), -128, 127).astype(np.int8)
+    rowsum = q.astype(np.int64).sum(axis=1).astype(np.int32)
+    return q, s_x.astype(np.float32), rowsum
+
+
+def epilogue_bf16(acc: np.ndarray, s_x: np.ndarray, s_w: np.float32, bias_bits=None):
+    """[FE-univ] BitLinear.forward after F.linear on a bf16 module: y =
+    bf16(acc); d = bf16(bf16(s_w) * s_x); y = bf16(y / d); y = bf16(y + bias).
+    Returns (y32 float32 holding the bf16 values, y bf16 bits)."""
+    y = _bf16(acc.astype(np.float32))
+    d = _bf16(_bf16(np.float32(s_w)) * np.asarray(s_x, np.float32))
+    y = _bf16(y / d[:, None])
+    if bias_bits is not None:
+        y = _bf16(y + bf16_to_f32(bias_bits)[None, :])
+    y = y.astype(np.float32)
+    return y, f32_to_bf16_rne(y)
+
+
+def forward_bf16(x_bits: np.ndarray, packed: np.ndarray, s_w: np.float32, bias_bits=None,
+                 K: int | None = None):
+    """BitLinear.forward with the listings' bf16 dtype semantics."""
+    q, s_x, rowsum = act_quant_bf16(x_bits)
+    acc = contract(q, unpack(packed, K))
+    y32, y = epilogue_bf16(acc, s_x, s_w, bias_bits)
     return {"q": q, "s_x": s_x, "rowsum": rowsum, "acc": acc, "y32": y32, "y": y}
 
 

@@ -434,3 +434,56 @@ def test_grouped_forward_acc_is_one_integer_matmul():
     out = oracle.forward_grouped(xb, oracle.pack(u), [7, 30, 3], [np.float32(1.5), np.float32(2.0), np.float32(0.25)])
     q = oracle.act_quant(xb)[0].astype(np.int64)
     assert np.array_equal(out["acc"], (q @ u.astype(np.int64).T).astype(np.int32))
+
+
+# --------------------------------------------------------------------------
+# bf16-faithful mode: the listings executed by PyTorch on bf16 tensors
+# --------------------------------------------------------------------------
+
+def _listing_on_bf16_module(x, u, s_w, bias):
+    """activation_norm_quant and BitLinear.forward of the Falcon-Edge blog,
+    run by PyTorch (CPU) on a module whose dtype is bfloat16; the weight
+    scale is the module's bf16 copy of s_w."""
+    scale = 127.0 / x.abs().max(dim=-1, keepdim=True).values.clamp_(min=1e-5)
+    xq = (x * scale).round().clamp_(-128, 127)
+    w_quant = torch.tensor(u, dtype=torch.bfloat16)
+    y = torch.nn.functional.linear(xq.to(torch.bfloat16), w_quant)
+    weight_scale = torch.tensor(float(s_w), dtype=torch.float32).to(torch.bfloat16)
+    y = y / (weight_scale * scale)          # post_quant_process(y, weight_scale, input_scale)
+    if bias is not None:
+        y += bias.view(1, -1).expand_as(y)
+    return xq, scale, y
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_bf16_mode_matches_pytorch_bf16_execution(seed):
+    rng = np.random.default_rng(900 + seed)
+    M, K, N = int(rng.integers(1, 9)), int(rng.choice([64, 128, 256])), int(rng.integers(1, 65))
+    x = synth.normal_bf16(300 + seed, 1, (M, K), float(rng.choice([0.01, 1.0, 30.0])))
+    x[0, : K // 2] = 0 if M > 1 else x[0, : K // 2]
+    if M > 2:
+        x[2] = 0                                             # an all-zero row: the clamp decides
+    w = synth.normal_f32(300 + seed, 2, (N, K), 0.02).numpy()
+    packed, s_w, _ = oracle.pack_weights(w)
+    u = oracle.unpack(packed)
+    bias = synth.normal_bf16(300 + seed, 3, (N,), 0.5) if seed % 2 else None
+    xq_t, scale_t, y_t = _listing_on_bf16_module(x, u.astype(np.float32), s_w, bias)
+    out = oracle.forward_bf16(synth.bf16_bits(x), packed, s_w, None if bias is None else synth.bf16_bits(bias))
+    assert np.array_equal(out["q"], xq_t.float().numpy().astype(np.int8))
+    assert np.array_equal(out["s_x"], scale_t.float().numpy()[:, 0])
+    assert np.array_equal(out["y"], synth.bf16_bits(y_t))
+
+
+def test_bf16_mode_differs_from_float32_mode_only_by_rounding():
+    # the two modes read the same pages; they differ only in where rounding
+    # happens, so the outputs agree to within a few bf16 ulps
+    x = synth.normal_bf16(77, 5, (6, 512))
+    w = synth.normal_f32(77, 6, (96, 512), 0.02).numpy()
+    packed, s_w, _ = oracle.pack_weights(w)
+    xb = synth.bf16_bits(x)
+    a = oracle.bf16_to_f32(oracle.forward(xb, packed, s_w)["y"]).astype(np.float64)
+    b = oracle.bf16_to_f32(oracle.forward_bf16(xb, packed, s_w)["y"]).astype(np.float64)
+    # per row, relative to the row's norm (single outputs near zero can move
+    # by more: bf16 rounding of the integer sum and a different s_x)
+    rel = np.linalg.norm(a - b, axis=1) / np.linalg.norm(a, axis=1)
+    assert np.all(rel < 0.02), rel
