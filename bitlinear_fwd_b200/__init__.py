@@ -32,6 +32,9 @@ _SIGS = {
     "bitlinear_pack_weights": (ctypes.c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_p, _c_p, _c_p, _c_sz, _c_p]),
     "bitlinear_quant_act": (ctypes.c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_p, _c_p, _c_p]),
     "bitlinear_dequant_weights": (ctypes.c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_p, _c_p]),
+    "bitlinear_forward_debug_ex": (ctypes.c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_i64, _c_p, _c_p, _c_p, _c_p,
+                                                  _c_p, _c_p, _c_p, ctypes.c_int, ctypes.c_uint, _c_p,
+                                                  ctypes.c_size_t, _c_p]),
     "bitlinear_forward_grouped": (ctypes.c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_p, ctypes.c_int, _c_p, _c_p, _c_p,
                                                  ctypes.c_uint, _c_p, ctypes.c_size_t, _c_p]),
     "bitlinear_forward": (ctypes.c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_i64, _c_p, _c_p, _c_p, _c_p, _c_sz,
@@ -161,6 +164,7 @@ def bitlinear_dequant_weights(packed: torch.Tensor, w_scale: torch.Tensor) -> to
 
 
 WEIGHTS_RESIDENT = 1
+BF16_FAITHFUL = 2
 
 
 def bitlinear_forward(x: torch.Tensor, packed: torch.Tensor, w_scale: torch.Tensor,
@@ -225,8 +229,9 @@ def bitlinear_forward_q8(xq: torch.Tensor, s_x: torch.Tensor, rowsum: torch.Tens
 
 def bitlinear_forward_debug(x: torch.Tensor, packed: torch.Tensor, w_scale: torch.Tensor,
                             bias: Optional[torch.Tensor] = None, engine: int = 0,
-                            ws: Optional[torch.Tensor] = None) -> dict:
-    """Forward with intermediates: y, xq, s_x, acc (int32), y32 (float32)."""
+                            ws: Optional[torch.Tensor] = None, flags: int = 0) -> dict:
+    """Forward with intermediates: y, xq, s_x, acc (int32), y32 (float32).
+    flags=BF16_FAITHFUL calls bitlinear_forward_debug_ex."""
     x = _bits(x)
     M, K = x.shape
     N = packed.shape[0]
@@ -239,9 +244,14 @@ def bitlinear_forward_debug(x: torch.Tensor, packed: torch.Tensor, w_scale: torc
     if ws is None:
         ws = workspace(M, N, K, dev)
     b = None if bias is None else _bits(bias)
-    _check(lib().bitlinear_forward_debug(_ptr(x), M, K, _ptr(packed), N, _ptr(w_scale), _ptr(b), _ptr(y),
-                                         _ptr(xq), _ptr(s_x), _ptr(acc), _ptr(y32), engine, _ptr(ws),
-                                         ws.numel(), _stream(dev)), "bitlinear_forward_debug")
+    if flags:
+        _check(lib().bitlinear_forward_debug_ex(_ptr(x), M, K, _ptr(packed), N, _ptr(w_scale), _ptr(b), _ptr(y),
+                                                _ptr(xq), _ptr(s_x), _ptr(acc), _ptr(y32), engine, flags, _ptr(ws),
+                                                ws.numel(), _stream(dev)), "bitlinear_forward_debug_ex")
+    else:
+        _check(lib().bitlinear_forward_debug(_ptr(x), M, K, _ptr(packed), N, _ptr(w_scale), _ptr(b), _ptr(y),
+                                             _ptr(xq), _ptr(s_x), _ptr(acc), _ptr(y32), engine, _ptr(ws),
+                                             ws.numel(), _stream(dev)), "bitlinear_forward_debug")
     return {"y": y, "xq": xq, "s_x": s_x, "acc": acc, "y32": y32, "ws": ws}
 
 

@@ -1,7 +1,8 @@
 // Per-token activation quantisation (activation_norm_quant of the
 // Falcon-Edge blog, section "Falcon-Edge, a series of universal models"):
 //   s_x = 127 / max(max_k |x|, 1e-5),  q = clamp(round_half_even(x * s_x), -128, 127)
-// in float32, plus the row sum of q that the contraction engines use.
+// in float32, plus the row sum of q that the contraction engines use.  In
+// the bf16-faithful mode every step is rounded as a bf16 module rounds it.
 //
 // One CTA per row.  The row is read once with 16-byte loads and kept in
 // registers between the absmax pass and the quantisation pass (rows of up
@@ -47,7 +48,7 @@ __device__ __forceinline__ int reduce_add_i32(int v, int* red) {
 }
 
 // Quantises 16 bf16 values (two 16-byte vectors) into one 16-byte vector of int8.
-__device__ __forceinline__ uint4 quant16(uint4 lo, uint4 hi, float s, int& sum) {
+__device__ __forceinline__ uint4 quant16(uint4 lo, uint4 hi, float s, int& sum, bool faithful) {
   const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
   uint32_t out[4];
 #pragma unroll
@@ -57,7 +58,8 @@ __device__ __forceinline__ uint4 quant16(uint4 lo, uint4 hi, float s, int& sum) 
     for (int h = 0; h < 4; ++h) {
       const int e = 4 * b + h;  // element 0..15
       const uint32_t bits = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu);
-      const float t = __fmul_rn(bf16_bits_to_f32(bits), s);
+      float t = __fmul_rn(bf16_bits_to_f32(bits), s);
+      if (faithful) t = bf16_round(t);               // the bf16 tensor x * scale
       int q = __float2int_rn(t);
       q = min(127, max(-128, q));
       sum += q;
@@ -73,7 +75,7 @@ __global__ void __launch_bounds__(kThreads) act_quant_kernel(const uint16_t* __r
                                                              int8_t* __restrict__ xq,
                                                              float* __restrict__ s_x,
                                                              int32_t* __restrict__ rowsum,
-                                                             uint32_t* status_clear) {
+                                                             uint32_t* status_clear, bool faithful) {
   pdl_launch_dependents();
   pdl_wait_primary();
   if (status_clear && blockIdx.x == 0 && threadIdx.x == 0) *status_clear = 0u;
@@ -119,18 +121,21 @@ __global__ void __launch_bounds__(kThreads) act_quant_kernel(const uint16_t* __r
   amax = reduce_max_u32(amax, red);
 
   const float a = bf16_bits_to_f32(amax);
-  const float s = __fdiv_rn(127.0f, fmaxf(a, 1e-5f));
+  // float32: 127 / max(a, 1e-5).  bf16 module: PyTorch evaluates 127.0 / t as
+  // t.reciprocal() * 127, each rounded to bf16.
+  const float s = faithful ? bf16_round(__fmul_rn(bf16_round(__fdiv_rn(1.0f, fmaxf(a, bf16_round(1e-5f)))), 127.0f))
+                           : __fdiv_rn(127.0f, fmaxf(a, 1e-5f));
 
   int sum = 0;
   if constexpr (CPT > 0) {
 #pragma unroll
     for (int i = 0; i < CPT; ++i) {
       const int c = threadIdx.x + i * kThreads;
-      if (c < chunks) qr[c] = quant16(cache[2 * i], cache[2 * i + 1], s, sum);
+      if (c < chunks) qr[c] = quant16(cache[2 * i], cache[2 * i + 1], s, sum, faithful);
     }
   } else {
     for (int c = threadIdx.x; c < chunks; c += kThreads)
-      qr[c] = quant16(__ldg(xr + 2 * c), __ldg(xr + 2 * c + 1), s, sum);
+      qr[c] = quant16(__ldg(xr + 2 * c), __ldg(xr + 2 * c + 1), s, sum, faithful);
   }
   sum = reduce_add_i32(sum, reinterpret_cast<int*>(red));
   if (threadIdx.x == 0) {
@@ -143,7 +148,7 @@ __global__ void __launch_bounds__(kThreads) act_quant_kernel(const uint16_t* __r
 
 template <int CPT>
 cudaError_t launch_cpt(const uint16_t* x, int M, int K, int8_t* xq, float* s_x, int32_t* rowsum,
-                       uint32_t* status_clear, bool pdl, cudaStream_t stream) {
+                       uint32_t* status_clear, bool pdl, cudaStream_t stream, bool faithful) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(M, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -154,18 +159,19 @@ cudaError_t launch_cpt(const uint16_t* x, int M, int K, int8_t* xq, float* s_x, 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, act_quant_kernel<CPT>, x, K, xq, s_x, rowsum, status_clear);
+  return cudaLaunchKernelEx(&cfg, act_quant_kernel<CPT>, x, K, xq, s_x, rowsum, status_clear, faithful);
 }
 
 cudaError_t launch_act_quant(const uint16_t* x, int M, int K, int8_t* xq, float* s_x,
-                             int32_t* rowsum, uint32_t* status_clear, bool pdl, cudaStream_t stream) {
+                             int32_t* rowsum, uint32_t* status_clear, bool pdl, cudaStream_t stream,
+                             bool faithful) {
   if (M <= 0) return cudaSuccess;
   const int chunks = K / 16;
-  if (chunks <= kThreads) return launch_cpt<1>(x, M, K, xq, s_x, rowsum, status_clear, pdl, stream);
-  if (chunks <= 2 * kThreads) return launch_cpt<2>(x, M, K, xq, s_x, rowsum, status_clear, pdl, stream);
-  if (chunks <= 4 * kThreads) return launch_cpt<4>(x, M, K, xq, s_x, rowsum, status_clear, pdl, stream);
-  if (chunks <= 8 * kThreads) return launch_cpt<8>(x, M, K, xq, s_x, rowsum, status_clear, pdl, stream);
-  return launch_cpt<0>(x, M, K, xq, s_x, rowsum, status_clear, pdl, stream);
+  if (chunks <= kThreads) return launch_cpt<1>(x, M, K, xq, s_x, rowsum, status_clear, pdl, stream, faithful);
+  if (chunks <= 2 * kThreads) return launch_cpt<2>(x, M, K, xq, s_x, rowsum, status_clear, pdl, stream, faithful);
+  if (chunks <= 4 * kThreads) return launch_cpt<4>(x, M, K, xq, s_x, rowsum, status_clear, pdl, stream, faithful);
+  if (chunks <= 8 * kThreads) return launch_cpt<8>(x, M, K, xq, s_x, rowsum, status_clear, pdl, stream, faithful);
+  return launch_cpt<0>(x, M, K, xq, s_x, rowsum, status_clear, pdl, stream, faithful);
 }
 
 }  // namespace bitlinear

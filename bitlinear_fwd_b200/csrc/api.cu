@@ -102,6 +102,7 @@ int forward_impl_g(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packe
   char* base = static_cast<char*>(ws);
   uint32_t* status = reinterpret_cast<uint32_t*>(base);
   const bool resident = (flags & BITLINEAR_WEIGHTS_RESIDENT) != 0;
+  const bool faithful = (flags & BITLINEAR_BF16_FAITHFUL) != 0;
   const bool decode = engine == 1 || (engine == 0 && M <= 16);
   cudaError_t e;
   if (decode) {
@@ -122,6 +123,7 @@ int forward_impl_g(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packe
     d.N = int(N);
     d.K = int(K);
     d.weights_early = resident ? 1 : 0;
+    d.faithful = faithful ? 1 : 0;
     d.ngroups = grp.n;
     for (int g = 0; g < kMaxGroups; ++g) d.group_end[g] = grp.end[g];
     return status_of(launch_decode(d, sms, stream));
@@ -129,7 +131,7 @@ int forward_impl_g(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packe
   float* s_x = reinterpret_cast<float*>(base + L.off_sx);
   int32_t* rowsum = reinterpret_cast<int32_t*>(base + L.off_rs);
   int8_t* xq = reinterpret_cast<int8_t*>(base + L.off_xq);
-  e = launch_act_quant(x, int(M), int(K), xq, s_x, rowsum, status, resident, stream);
+  e = launch_act_quant(x, int(M), int(K), xq, s_x, rowsum, status, resident, stream, faithful);
   if (e != cudaSuccess) return BITLINEAR_ERR_CUDA;
   ForwardArgs a;
   a.xq = xq;
@@ -146,6 +148,7 @@ int forward_impl_g(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packe
   a.N = int(N);
   a.K = int(K);
   a.pdl = true;
+  a.faithful = faithful;
   a.ngroups = grp.n;
   for (int g = 0; g < kMaxGroups; ++g) a.group_end[g] = grp.end[g];
   e = launch_gemm_prefill(a, sms, stream);
@@ -260,7 +263,7 @@ int bitlinear_forward(const uint16_t* x, int64_t M, int64_t K, const uint8_t* pa
 int bitlinear_forward_ex(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed_w, int64_t N,
                          const float* w_scale, const uint16_t* bias, uint16_t* y, unsigned flags, void* ws,
                          size_t ws_bytes, void* stream) {
-  if (flags & ~static_cast<unsigned>(BITLINEAR_WEIGHTS_RESIDENT)) return BITLINEAR_ERR_SHAPE;
+  if (flags & ~static_cast<unsigned>(BITLINEAR_WEIGHTS_RESIDENT | BITLINEAR_BF16_FAITHFUL)) return BITLINEAR_ERR_SHAPE;
   int st = check_forward_args(x, M, K, packed_w, N, w_scale, bias, y, ws, ws_bytes,
                               bitlinear_workspace_bytes(M, N, K), false);
   if (st != BITLINEAR_OK) return st;
@@ -272,7 +275,7 @@ int bitlinear_forward_ex(const uint16_t* x, int64_t M, int64_t K, const uint8_t*
 int bitlinear_forward_grouped(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed_w,
                               const int64_t* group_rows, int groups, const float* w_scales, const uint16_t* bias,
                               uint16_t* y, unsigned flags, void* ws, size_t ws_bytes, void* stream) {
-  if (flags & ~static_cast<unsigned>(BITLINEAR_WEIGHTS_RESIDENT)) return BITLINEAR_ERR_SHAPE;
+  if (flags & ~static_cast<unsigned>(BITLINEAR_WEIGHTS_RESIDENT | BITLINEAR_BF16_FAITHFUL)) return BITLINEAR_ERR_SHAPE;
   if (!group_rows) return BITLINEAR_ERR_NULL;
   if (groups < 1 || groups > BITLINEAR_MAX_GROUPS) return BITLINEAR_ERR_SHAPE;
   Groups grp{};
@@ -322,6 +325,7 @@ int bitlinear_forward_q8(const int8_t* xq, const float* x_scale, const int32_t* 
   a.N = int(N);
   a.K = int(K);
   a.pdl = false;
+  a.faithful = false;
   a.ngroups = 1;
   a.group_end[0] = int(N);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -345,6 +349,7 @@ int bitlinear_forward_q8(const int8_t* xq, const float* x_scale, const int32_t* 
   d.N = int(N);
   d.K = int(K);
   d.weights_early = 0;
+  d.faithful = 0;
   d.ngroups = 1;
   d.group_end[0] = int(N);
   return status_of(launch_decode(d, sms, s));
@@ -373,6 +378,21 @@ int bitlinear_forward_debug(const uint16_t* x, int64_t M, int64_t K, const uint8
   if (misaligned(xq) || misaligned(x_scale) || misaligned(acc) || misaligned(y32)) return BITLINEAR_ERR_ALIGN;
   if (M == 0) return BITLINEAR_OK;
   return forward_impl(x, M, K, packed_w, N, w_scale, bias, y, xq, x_scale, acc, y32, engine, 0u, ws, ws_bytes,
+                      static_cast<cudaStream_t>(stream));
+}
+
+int bitlinear_forward_debug_ex(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed_w, int64_t N,
+                               const float* w_scale, const uint16_t* bias, uint16_t* y, int8_t* xq,
+                               float* x_scale, int32_t* acc, float* y32, int engine, unsigned flags, void* ws,
+                               size_t ws_bytes, void* stream) {
+  if (flags & ~static_cast<unsigned>(BITLINEAR_BF16_FAITHFUL)) return BITLINEAR_ERR_SHAPE;
+  int st = check_forward_args(x, M, K, packed_w, N, w_scale, bias, y, ws, ws_bytes,
+                              bitlinear_workspace_bytes(M, N, K), false);
+  if (st != BITLINEAR_OK) return st;
+  if (engine < 0 || engine > 2 || (engine == 1 && M > 16)) return BITLINEAR_ERR_SHAPE;
+  if (misaligned(xq) || misaligned(x_scale) || misaligned(acc) || misaligned(y32)) return BITLINEAR_ERR_ALIGN;
+  if (M == 0) return BITLINEAR_OK;
+  return forward_impl(x, M, K, packed_w, N, w_scale, bias, y, xq, x_scale, acc, y32, engine, flags, ws, ws_bytes,
                       static_cast<cudaStream_t>(stream));
 }
 

@@ -246,5 +246,7 @@ __device__ __forceinline__ float bf16_bits_to_f32(uint32_t bits16) {
 __device__ __forceinline__ uint16_t f32_to_bf16_bits(float v) {
   return __bfloat16_as_ushort(__float2bfloat16_rn(v));
 }
+// v rounded to bfloat16 (RNE) and widened back: one bf16 tensor op's result
+__device__ __forceinline__ float bf16_round(float v) { return bf16_bits_to_f32(f32_to_bf16_bits(v)); }
 
 }  // namespace bitlinear

@@ -237,6 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int g = 1; g < kMaxGroups; ++g)
         if (g < a.ngroups && n >= a.group_end[g - 1]) s_w = swg[g];
+      if (a.faithful) s_w = bf16_round(s_w);       // a bf16 module holds s_w in bf16
 #pragma unroll 1
       for (int c = 0; c < BT / 32; ++c) {
         uint32_t r[32];
@@ -254,8 +255,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int mi = 32 * c + i, m = m0 + mi;
           if (m >= a.M) continue;
           const int accv = static_cast<int>(r[i]) - rs_s[mi];
-          float y32 = __fdiv_rn(static_cast<float>(accv), __fmul_rn(d_s[mi], s_w));
-          if (a.bias) y32 = __fadd_rn(y32, bv);
+          float y32;
+          if (!a.faithful) {
+            y32 = __fdiv_rn(static_cast<float>(accv), __fmul_rn(d_s[mi], s_w));
+            if (a.bias) y32 = __fadd_rn(y32, bv);
+          } else {
+            // bf16 module: the sum, the scale product, the quotient and the
+            // bias add are each rounded to bf16
+            y32 = bf16_round(__fdiv_rn(bf16_round(static_cast<float>(accv)), bf16_round(__fmul_rn(s_w, d_s[mi]))));
+            if (a.bias) y32 = bf16_round(__fadd_rn(y32, bv));
+          }
           const size_t o = static_cast<size_t>(m) * a.N + n;
           a.y[o] = f32_to_bf16_bits(y32);
           if (a.acc_out) a.acc_out[o] = accv;

@@ -104,29 +104,43 @@ __device__ __forceinline__ uint32_t absmax16_bits(uint4 lo, uint4 hi) {
 // p = x * s is rounded to float32 first; adding 1.5 * 2^23 then rounds p to an
 // integer with ties to even (the sum lies in [2^23, 2^24), where the float
 // spacing is 1, and the magic constant is even), and the low byte of the sum's
-// bits is q as a two's-complement byte.  |p| <= 127 for finite x because s was
-// formed from the row's absmax, so the [-128, 127] clamp never acts.
-__device__ __forceinline__ uint32_t quant4(uint32_t w01, uint32_t w23, float s) {
-  const float f0 = __uint_as_float(w01 << 16), f1 = __uint_as_float(w01 & 0xFFFF0000u);
-  const float f2 = __uint_as_float(w23 << 16), f3 = __uint_as_float(w23 & 0xFFFF0000u);
-  const uint32_t b0 = __float_as_uint(__fadd_rn(__fmul_rn(f0, s), kRoundMagic));
-  const uint32_t b1 = __float_as_uint(__fadd_rn(__fmul_rn(f1, s), kRoundMagic));
-  const uint32_t b2 = __float_as_uint(__fadd_rn(__fmul_rn(f2, s), kRoundMagic));
-  const uint32_t b3 = __float_as_uint(__fadd_rn(__fmul_rn(f3, s), kRoundMagic));
+// bits is q as a two's-complement byte.  In float32 |p| <= 127 for finite x
+// because s was formed from the row's absmax, so the [-128, 127] clamp never
+// acts; the bf16-faithful path clamps explicitly.
+__device__ __forceinline__ uint32_t quant4(uint32_t w01, uint32_t w23, float s, bool faithful) {
+  float p[4] = {__fmul_rn(__uint_as_float(w01 << 16), s), __fmul_rn(__uint_as_float(w01 & 0xFFFF0000u), s),
+                __fmul_rn(__uint_as_float(w23 << 16), s), __fmul_rn(__uint_as_float(w23 & 0xFFFF0000u), s)};
+  if (faithful) {
+    // the bf16 tensor x * scale; here the scale can exceed 127 / absmax by a
+    // few bf16 ulps, so the product can round to 128 and the clamp acts
+#pragma unroll
+    for (int e = 0; e < 4; ++e) p[e] = fminf(fmaxf(bf16_round(p[e]), -128.0f), 127.0f);
+  }
+  const uint32_t b0 = __float_as_uint(__fadd_rn(p[0], kRoundMagic));
+  const uint32_t b1 = __float_as_uint(__fadd_rn(p[1], kRoundMagic));
+  const uint32_t b2 = __float_as_uint(__fadd_rn(p[2], kRoundMagic));
+  const uint32_t b3 = __float_as_uint(__fadd_rn(p[3], kRoundMagic));
   return __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
 }
 
-__device__ __forceinline__ uint4 quant16(uint4 lo, uint4 hi, float s, int& sum) {
+__device__ __forceinline__ uint4 quant16(uint4 lo, uint4 hi, float s, int& sum, bool faithful) {
   uint4 q;
-  q.x = quant4(lo.x, lo.y, s);
-  q.y = quant4(lo.z, lo.w, s);
-  q.z = quant4(hi.x, hi.y, s);
-  q.w = quant4(hi.z, hi.w, s);
+  q.x = quant4(lo.x, lo.y, s, faithful);
+  q.y = quant4(lo.z, lo.w, s, faithful);
+  q.z = quant4(hi.x, hi.y, s, faithful);
+  q.w = quant4(hi.z, hi.w, s, faithful);
   sum = __dp4a(static_cast<int>(q.x), 0x01010101, sum);
   sum = __dp4a(static_cast<int>(q.y), 0x01010101, sum);
   sum = __dp4a(static_cast<int>(q.z), 0x01010101, sum);
   sum = __dp4a(static_cast<int>(q.w), 0x01010101, sum);
   return q;
+}
+
+// s_x from the row's absmax a: 127 / max(a, 1e-5) in float32, or, on a bf16
+// module, PyTorch's evaluation of 127.0 / t: bf16(bf16(1 / t) * 127)
+__device__ __forceinline__ float act_scale(float a, bool faithful) {
+  return faithful ? bf16_round(__fmul_rn(bf16_round(__fdiv_rn(1.0f, fmaxf(a, bf16_round(1e-5f)))), 127.0f))
+                  : __fdiv_rn(127.0f, fmaxf(a, 1e-5f));
 }
 
 __device__ __forceinline__ int bytesum16(uint4 v, int sum) {
@@ -294,10 +308,10 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
 #pragma unroll
       for (int j = 0; j < NT; ++j) {
         const int m = min(warp / P + j * mstep, M - 1);
-        sxr[j] = __fdiv_rn(127.0f, fmaxf(bf16_bits_to_f32(sm.amax[m]), 1e-5f));
+        sxr[j] = act_scale(bf16_bits_to_f32(sm.amax[m]), a.faithful);
       }
       if (threadIdx.x < M) {
-        const float sxv = __fdiv_rn(127.0f, fmaxf(bf16_bits_to_f32(sm.amax[threadIdx.x]), 1e-5f));
+        const float sxv = act_scale(bf16_bits_to_f32(sm.amax[threadIdx.x]), a.faithful);
         sm.sx[threadIdx.x] = sxv;
         if (blockIdx.x == 0 && a.sx_out) a.sx_out[threadIdx.x] = sxv;
       }
@@ -311,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
         const int ch = part * 32 + lane + (i - j * C) * 32 * P;
         if (i < NT * C && m < M && ch < cpr) {
           int ps = 0;
-          const uint4 qv = quant16(v[i][0], v[i][1], j ? sxr[NT - 1] : sxr[0], ps);
+          const uint4 qv = quant16(v[i][0], v[i][1], j ? sxr[NT - 1] : sxr[0], ps, a.faithful);
           if (j) sum[NT - 1] += ps;
           else sum[0] += ps;
           *reinterpret_cast<uint4*>(xs + m * S + 16 * xs_chunk(ch)) = qv;
@@ -348,7 +362,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
       }
       consumer_sync();
       if (threadIdx.x < M) {
-        const float sxv = __fdiv_rn(127.0f, fmaxf(bf16_bits_to_f32(sm.amax[threadIdx.x]), 1e-5f));
+        const float sxv = act_scale(bf16_bits_to_f32(sm.amax[threadIdx.x]), a.faithful);
         sm.sx[threadIdx.x] = sxv;
         if (blockIdx.x == 0 && a.sx_out) a.sx_out[threadIdx.x] = sxv;
       }
@@ -384,7 +398,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
             for (int j = 0; j < kQB; ++j) {
               const int ch = ch0 + j * 32 * P;
               if (ch < ccpr) {
-                const uint4 qv = quant16(v[j][0], v[j][1], sxm, sum);
+                const uint4 qv = quant16(v[j][0], v[j][1], sxm, sum, a.faithful);
                 if (blockIdx.x == 0 && a.xq_out) *reinterpret_cast<uint4*>(a.xq_out + roff + 16 * ch) = qv;
                 *reinterpret_cast<uint4*>(xrow + 16 * xs_chunk(ch)) = qv;
               }
@@ -523,9 +537,18 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
     int gi = 0;                                      // the row's group (scale)
 #pragma unroll
     for (int g = 0; g + 1 < kMaxGroups; ++g) gi += (g + 1 < a.ngroups && n >= a.group_end[g]) ? 1 : 0;
-    const float d = __fmul_rn(sm.sx[m], sm.swg[gi]);
-    float y32 = __fdiv_rn(static_cast<float>(accv), d);
-    if (a.bias) y32 = __fadd_rn(y32, bf16_bits_to_f32(bias_s[rl]));
+    float y32;
+    if (!a.faithful) {
+      const float d = __fmul_rn(sm.sx[m], sm.swg[gi]);
+      y32 = __fdiv_rn(static_cast<float>(accv), d);
+      if (a.bias) y32 = __fadd_rn(y32, bf16_bits_to_f32(bias_s[rl]));
+    } else {
+      // bf16 module: F.linear's sum, the scale product, the quotient and the
+      // bias add are each a bf16 tensor
+      const float d = bf16_round(__fmul_rn(bf16_round(sm.swg[gi]), sm.sx[m]));
+      y32 = bf16_round(__fdiv_rn(bf16_round(static_cast<float>(accv)), d));
+      if (a.bias) y32 = bf16_round(__fadd_rn(y32, bf16_bits_to_f32(bias_s[rl])));
+    }
     const size_t o = static_cast<size_t>(m) * N + n;
     a.y[o] = f32_to_bf16_bits(y32);
     if (a.acc_out) a.acc_out[o] = accv;

@@ -20,8 +20,11 @@ bool encode_3d_u8(CUtensorMap* map, const void* base, const uint64_t dims[3], co
 // ---- activation quantisation (act_quant.cu) --------------------------------
 // pdl: launch as a programmatic dependent of the previous kernel on the stream
 // (the kernel waits for it before touching memory).
+// faithful: the bf16-module rounding of every step (scale = bf16(bf16(1/a) * 127),
+// q = round(bf16(x * scale))) instead of float32 arithmetic
 cudaError_t launch_act_quant(const uint16_t* x, int M, int K, int8_t* xq, float* s_x,
-                             int32_t* rowsum, uint32_t* status_clear, bool pdl, cudaStream_t stream);
+                             int32_t* rowsum, uint32_t* status_clear, bool pdl, cudaStream_t stream,
+                             bool faithful = false);
 
 // ---- weight absmean + ternarise + pack (pack.cu) ----------------------------
 // Workspace layout used by the pack kernels.
@@ -55,6 +58,7 @@ struct ForwardArgs {
   int ngroups;
   int group_end[kMaxGroups];
   bool pdl;               // launched as a programmatic dependent of the act-quant kernel
+  bool faithful;          // bf16-module epilogue: every step rounded to bf16
 };
 
 // ---- bf16 export of packed weights (dequant.cu) ----------------------------
@@ -78,6 +82,7 @@ struct DecodeArgs {
   int M, N, K;
   int ngroups;
   int group_end[kMaxGroups];
+  int faithful;           // bf16-module rounding of the quantisation and the epilogue
   int ring, units_max, kc, tail;  // set by launch_decode
   int weights_early;      // the packed weights, w_scale and bias may be read before the dependency wait
 };

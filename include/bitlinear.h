@@ -142,6 +142,15 @@ int bitlinear_forward(const uint16_t* x, int64_t M, int64_t K, const uint8_t* pa
  *   launch), which overlaps consecutive layers.  Never set it when the
  *   previous operation on the stream writes packed_w, w_scale or bias. */
 
+#define BITLINEAR_BF16_FAITHFUL 2u
+/*   Compute as the listings do on a bfloat16 module (Falcon-Edge blog,
+ *   section "Falcon-Edge, a series of universal models", activation_norm_quant
+ *   and BitLinear.forward): every tensor op rounds to bf16, s_x =
+ *   bf16(bf16(1 / max(a, 1e-5)) * 127) (PyTorch's evaluation of 127.0 / t),
+ *   q = round(bf16(x * s_x)), y = bf16(bf16(acc) / bf16(bf16(s_w) * s_x)),
+ *   then bf16(y + bias).  Without it, every step is float32 with one rounding
+ *   to bf16 at the end. */
+
 /* bitlinear_forward with flags (0 = identical to bitlinear_forward). */
 int bitlinear_forward_ex(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed_w, int64_t N,
                          const float* w_scale, const uint16_t* bias, uint16_t* y, unsigned flags, void* ws,
@@ -177,6 +186,12 @@ int bitlinear_forward_grouped(const uint16_t* x, int64_t M, int64_t K, const uin
 int bitlinear_forward_q8(const int8_t* xq, const float* x_scale, const int32_t* xq_rowsum, int64_t M,
                          int64_t K, const uint8_t* packed_w, int64_t N, const float* w_scale,
                          const uint16_t* bias, uint16_t* y, void* ws, size_t ws_bytes, void* stream);
+
+/* bitlinear_forward_debug with flags (BITLINEAR_BF16_FAITHFUL or 0). */
+int bitlinear_forward_debug_ex(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed_w,
+                               int64_t N, const float* w_scale, const uint16_t* bias, uint16_t* y,
+                               int8_t* xq, float* x_scale, int32_t* acc, float* y32, int engine,
+                               unsigned flags, void* ws, size_t ws_bytes, void* stream);
 
 /* bf16 export of packed ternary weights, for loading them into a plain bf16
  * linear layer (Falcon-Edge blog, section "Falcon-Edge, a series of universal

@@ -93,5 +93,10 @@ def test_argument_errors_without_gpu(lib):
     assert g(16, 8, 256, 16, rows, 9, 16, None, 16, 0, 16, 1 << 20, None) == -2    # too many groups
     assert g(16, 8, 256, 16, bad, 2, 16, None, 16, 0, 16, 1 << 20, None) == -2     # empty group
     assert g(16, 8, 256, 16, rows, 3, None, None, 16, 0, 16, 1 << 20, None) == -1  # no scales
-    assert g(16, 8, 256, 16, rows, 3, 16, None, 16, 2, 16, 1 << 20, None) == -2    # unknown flag
+    assert g(16, 8, 256, 16, rows, 3, 16, None, 16, 4, 16, 1 << 20, None) == -2    # unknown flag
     assert g(16, 8, 256, 16, rows, 3, 16, None, 16, 0, 16, 16, None) == -4         # workspace too small
+    # debug with flags: only the bf16-faithful flag is accepted
+    assert lib.bitlinear_forward_debug_ex(16, 8, 256, 16, 512, 16, None, 16, None, None, None, None, 0, 1, 16,
+                                          1 << 20, None) == -2
+    assert lib.bitlinear_forward_debug_ex(None, 8, 256, 16, 512, 16, None, 16, None, None, None, None, 0, 2, 16,
+                                          1 << 20, None) == -1
