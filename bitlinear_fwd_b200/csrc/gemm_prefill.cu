@@ -207,6 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float swg[kMaxGroups];                         // s_w of each row group
 #pragma unroll
     for (int g = 0; g < kMaxGroups; ++g) swg[g] = g < a.ngroups ? a.w_scale[g] : 0.0f;
+    const bool simple = a.ngroups == 1 && !a.faithful;
     int j = 0;
     // The four epilogue warps meet at a named barrier twice per tile; every
     // one of them runs every iteration (a failure only skips work), so the
@@ -217,8 +218,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // per-token s_x and row sums of this tile
       asm volatile("bar.sync 1, 128;" ::: "memory");   // previous tile's readers are done
       {
+        // one float32 layer: d = s_x * s_w per token; otherwise s_x (the
+        // row's scale enters per element)
         const int m = m0 + et;
-        d_s[et] = m < a.M ? a.s_x[m] : 1.0f;
+        d_s[et] = m < a.M ? (simple ? __fmul_rn(a.s_x[m], swg[0]) : a.s_x[m]) : 1.0f;
         rs_s[et] = m < a.M ? a.rowsum[m] : 0;
       }
       asm volatile("bar.sync 1, 128;" ::: "memory");
@@ -250,25 +253,44 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) mbar_arrive(&acc_empty[b]);
         }
         if (!nv) continue;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int mi = 32 * c + i, m = m0 + mi;
-          if (m >= a.M) continue;
-          const int accv = static_cast<int>(r[i]) - rs_s[mi];
-          float y32;
-          if (!a.faithful) {
-            y32 = __fdiv_rn(static_cast<float>(accv), __fmul_rn(d_s[mi], s_w));
-            if (a.bias) y32 = __fadd_rn(y32, bv);
-          } else {
-            // bf16 module: the sum, the scale product, the quotient and the
-            // bias add are each rounded to bf16
-            y32 = bf16_round(__fdiv_rn(bf16_round(static_cast<float>(accv)), bf16_round(__fmul_rn(s_w, d_s[mi]))));
-            if (a.bias) y32 = bf16_round(__fadd_rn(y32, bv));
-          }
-          const size_t o = static_cast<size_t>(m) * a.N + n;
+        auto emit = [&](int mi, int accv, float y32) {
+          const size_t o = static_cast<size_t>(m0 + mi) * a.N + n;
           a.y[o] = f32_to_bf16_bits(y32);
           if (a.acc_out) a.acc_out[o] = accv;
           if (a.y32_out) a.y32_out[o] = y32;
+        };
+        if (simple) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int mi = 32 * c + i;
+            if (m0 + mi >= a.M) continue;
+            const int accv = static_cast<int>(r[i]) - rs_s[mi];
+            float y32 = __fdiv_rn(static_cast<float>(accv), d_s[mi]);
+            if (a.bias) y32 = __fadd_rn(y32, bv);
+            emit(mi, accv, y32);
+          }
+        } else if (!a.faithful) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int mi = 32 * c + i;
+            if (m0 + mi >= a.M) continue;
+            const int accv = static_cast<int>(r[i]) - rs_s[mi];
+            float y32 = __fdiv_rn(static_cast<float>(accv), __fmul_rn(d_s[mi], s_w));
+            if (a.bias) y32 = __fadd_rn(y32, bv);
+            emit(mi, accv, y32);
+          }
+        } else {
+          // bf16 module: the sum, the scale product, the quotient and the
+          // bias add are each rounded to bf16
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int mi = 32 * c + i;
+            if (m0 + mi >= a.M) continue;
+            const int accv = static_cast<int>(r[i]) - rs_s[mi];
+            float y32 = bf16_round(__fdiv_rn(bf16_round(static_cast<float>(accv)), bf16_round(__fmul_rn(s_w, d_s[mi]))));
+            if (a.bias) y32 = bf16_round(__fadd_rn(y32, bv));
+            emit(mi, accv, y32);
+          }
         }
       }
     }
