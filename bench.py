@@ -11,15 +11,18 @@ three times the L2 so that every step streams them from DRAM.  A step is
 captured once as a CUDA graph per weight copy and replayed.
 
 Also on the line:
-  roofline      the decode contraction kernel alone (launched through
-                bitlinear_forward_q8 between CUDA events on its stream):
-                algorithmic bytes per launch / mean launch time, against the
-                measured HBM copy bandwidth
+  roofline      the decode kernel (the whole forward is that one kernel):
+                algorithmic bytes per launch / mean launch time over the timed
+                graph replays, against the measured HBM copy bandwidth
   prefill       int8 TOPS of the prefill workload (M in {512, 2048, 8192},
                 (K, N) = (3200, 8640) and (8640, 3200)), the same way, with
                 the tcgen05 GEMM's own roofline against the int8 peak
-  e2e           the decode metric through bitlinear_forward_host: host bf16
-                activations copied in and outputs copied back every call
+  e2e           the decode metric through bitlinear_forward_host_async: host
+                bf16 activations copied in and outputs copied back every call,
+                the step's six calls enqueued and synchronised once
+  dequant_export, stack3b_decode
+                the bf16 export kernel's GB/s, and the 3B-class 26-layer
+                projection stack at M=1 with and without grouped calls
   cpu_baseline  the CPU oracle on a bounded sample of the decode workload
   clocks        nvidia-smi samples taken while the workload ran
 
@@ -335,8 +338,12 @@ def run_e2e(args, probs, steps):
     wss = [bl.workspace(p.M, p.N, p.K, "cuda", host=True) for p in probs]
 
     def step(r):
+        # the step's six calls are enqueued (host x in, host y out), then the
+        # step waits for its results
         for p, x, y, ws in zip(probs, xs, ys, wss):
-            bl.bitlinear_forward_host(x, p.packed[r % len(p.packed)], p.s_w, p.bias, y_host=y, ws=ws)
+            bl.bitlinear_forward_host_async(x, p.packed[r % len(p.packed)], p.s_w, p.bias, y_host=y, ws=ws,
+                                            flags=bl.WEIGHTS_RESIDENT)
+        torch.cuda.current_stream().synchronize()
 
     for i in range(3):
         step(i)
@@ -353,7 +360,7 @@ def run_e2e(args, probs, steps):
     return {"value": round(whole_job_gbs(bytes_step, steps, ms, world_size()), 2), "unit": "GB/s",
             "h2d_bytes_per_step": sum(2 * p.M * p.K for p in probs),
             "d2h_bytes_per_step": sum(2 * p.M * p.N for p in probs),
-            "api": "bitlinear_forward_host (pinned host x in, host y out, synchronous per call)"}
+            "api": "bitlinear_forward_host_async (pinned host x in, host y out), one stream sync per step"}
 
 
 def run_prefill(args, bf16_tflops, peak_kind, l2_bytes):

@@ -32,6 +32,8 @@ _SIGS = {
     "bitlinear_pack_weights": (ctypes.c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_p, _c_p, _c_p, _c_sz, _c_p]),
     "bitlinear_quant_act": (ctypes.c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_p, _c_p, _c_p]),
     "bitlinear_dequant_weights": (ctypes.c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_p, _c_p]),
+    "bitlinear_forward_host_async": (ctypes.c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_i64, _c_p, _c_p, _c_p,
+                                                    ctypes.c_uint, _c_p, ctypes.c_size_t, _c_p]),
     "bitlinear_forward_debug_ex": (ctypes.c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_i64, _c_p, _c_p, _c_p, _c_p,
                                                   _c_p, _c_p, _c_p, ctypes.c_int, ctypes.c_uint, _c_p,
                                                   ctypes.c_size_t, _c_p]),
@@ -271,6 +273,26 @@ def bitlinear_forward_host(x_host: torch.Tensor, packed: torch.Tensor, w_scale: 
     _check(lib().bitlinear_forward_host(_ptr(x_host), M, K, _ptr(packed), N, _ptr(w_scale), _ptr(b),
                                         _ptr(y_host), _ptr(ws), ws.numel(), _stream(dev)),
            "bitlinear_forward_host")
+    return y_host
+
+
+def bitlinear_forward_host_async(x_host: torch.Tensor, packed: torch.Tensor, w_scale: torch.Tensor,
+                                 bias: Optional[torch.Tensor] = None, y_host: Optional[torch.Tensor] = None,
+                                 ws: Optional[torch.Tensor] = None, flags: int = 0) -> torch.Tensor:
+    """Stream-ordered host-to-host forward: enqueues the copies and kernels and
+    returns; y_host is valid once the current stream is synchronised."""
+    x_host = _bits(x_host)
+    M, K = x_host.shape
+    N = packed.shape[0]
+    dev = packed.device
+    if y_host is None:
+        y_host = torch.empty((M, N), dtype=torch.bfloat16, pin_memory=True)
+    if ws is None:
+        ws = workspace(M, N, K, dev, host=True)
+    b = None if bias is None else _bits(bias)
+    _check(lib().bitlinear_forward_host_async(_ptr(x_host), M, K, _ptr(packed), N, _ptr(w_scale), _ptr(b),
+                                              _ptr(y_host), flags, _ptr(ws), ws.numel(), _stream(dev)),
+           "bitlinear_forward_host_async")
     return y_host
 
 

@@ -396,26 +396,42 @@ int bitlinear_forward_debug_ex(const uint16_t* x, int64_t M, int64_t K, const ui
                       static_cast<cudaStream_t>(stream));
 }
 
-int bitlinear_forward_host(const uint16_t* x_host, int64_t M, int64_t K, const uint8_t* packed_w, int64_t N,
-                           const float* w_scale, const uint16_t* bias, uint16_t* y_host, void* ws,
-                           size_t ws_bytes, void* stream) {
+namespace {
+int forward_host_impl(const uint16_t* x_host, int64_t M, int64_t K, const uint8_t* packed_w, int64_t N,
+                      const float* w_scale, const uint16_t* bias, uint16_t* y_host, unsigned flags, void* ws,
+                      size_t ws_bytes, cudaStream_t s, bool sync) {
   int st = check_forward_args(x_host, M, K, packed_w, N, w_scale, bias, y_host, ws, ws_bytes,
                               bitlinear_host_workspace_bytes(M, N, K), true);
   if (st != BITLINEAR_OK) return st;
   if (M == 0) return BITLINEAR_OK;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   const FwdLayout L = fwd_layout(M, N, K);
   char* base = static_cast<char*>(ws);
   uint16_t* xd = reinterpret_cast<uint16_t*>(base + L.off_xh);
   uint16_t* yd = reinterpret_cast<uint16_t*>(base + L.off_yh);
   if (cudaMemcpyAsync(xd, x_host, 2 * size_t(M) * size_t(K), cudaMemcpyHostToDevice, s) != cudaSuccess)
     return BITLINEAR_ERR_CUDA;
-  st = forward_impl(xd, M, K, packed_w, N, w_scale, bias, yd, nullptr, nullptr, nullptr, nullptr, 0, 0u, ws,
+  st = forward_impl(xd, M, K, packed_w, N, w_scale, bias, yd, nullptr, nullptr, nullptr, nullptr, 0, flags, ws,
                     ws_bytes, s);
   if (st != BITLINEAR_OK) return st;
   if (cudaMemcpyAsync(y_host, yd, 2 * size_t(M) * size_t(N), cudaMemcpyDeviceToHost, s) != cudaSuccess)
     return BITLINEAR_ERR_CUDA;
-  return status_of(cudaStreamSynchronize(s));
+  return sync ? status_of(cudaStreamSynchronize(s)) : BITLINEAR_OK;
+}
+}  // namespace
+
+int bitlinear_forward_host(const uint16_t* x_host, int64_t M, int64_t K, const uint8_t* packed_w, int64_t N,
+                           const float* w_scale, const uint16_t* bias, uint16_t* y_host, void* ws,
+                           size_t ws_bytes, void* stream) {
+  return forward_host_impl(x_host, M, K, packed_w, N, w_scale, bias, y_host, 0u, ws, ws_bytes,
+                           static_cast<cudaStream_t>(stream), true);
+}
+
+int bitlinear_forward_host_async(const uint16_t* x_host, int64_t M, int64_t K, const uint8_t* packed_w, int64_t N,
+                                 const float* w_scale, const uint16_t* bias, uint16_t* y_host, unsigned flags,
+                                 void* ws, size_t ws_bytes, void* stream) {
+  if (flags & ~static_cast<unsigned>(BITLINEAR_WEIGHTS_RESIDENT | BITLINEAR_BF16_FAITHFUL)) return BITLINEAR_ERR_SHAPE;
+  return forward_host_impl(x_host, M, K, packed_w, N, w_scale, bias, y_host, flags, ws, ws_bytes,
+                           static_cast<cudaStream_t>(stream), false);
 }
 
 int bitlinear_check_status(const void* ws, size_t ws_bytes, void* stream) {

@@ -225,6 +225,18 @@ int bitlinear_forward_host(const uint16_t* x_host, int64_t M, int64_t K, const u
                            int64_t N, const float* w_scale, const uint16_t* bias,
                            uint16_t* y_host, void* ws, size_t ws_bytes, void* stream);
 
+/* bitlinear_forward_host without the final synchronisation, with flags:
+ * the copies and kernels are only enqueued on `stream`.  y_host holds the
+ * result once the stream reaches that point (synchronise it, or an event
+ * recorded after the call).  x_host must stay unchanged until then.  With
+ * pinned host memory the copies are asynchronous, so consecutive calls
+ * overlap their copies with the previous calls' kernels.  Pageable memory
+ * falls back to synchronous copies.  Each call in flight needs its own
+ * workspace. */
+int bitlinear_forward_host_async(const uint16_t* x_host, int64_t M, int64_t K, const uint8_t* packed_w,
+                                 int64_t N, const float* w_scale, const uint16_t* bias, uint16_t* y_host,
+                                 unsigned flags, void* ws, size_t ws_bytes, void* stream);
+
 /* bitlinear_forward for callers that cannot allocate device memory (code
  * running inside someone else's CUDA-graph capture, server plugins given no
  * allocator, paths that must never allocate).  It takes no workspace: the

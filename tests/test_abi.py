@@ -100,3 +100,6 @@ def test_argument_errors_without_gpu(lib):
                                           1 << 20, None) == -2
     assert lib.bitlinear_forward_debug_ex(None, 8, 256, 16, 512, 16, None, 16, None, None, None, None, 0, 2, 16,
                                           1 << 20, None) == -1
+    # stream-ordered host forward: flag check first, then the host argument checks
+    assert lib.bitlinear_forward_host_async(16, 8, 256, 16, 512, 16, None, 16, 4, 16, 1 << 20, None) == -2
+    assert lib.bitlinear_forward_host_async(None, 8, 256, 16, 512, 16, None, 16, 0, 16, 1 << 20, None) == -1

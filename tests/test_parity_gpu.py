@@ -159,6 +159,14 @@ def test_forward_host_matches_device():
     y_dev = bl.bitlinear_forward(x.cuda(), packed, s_w, b).cpu()
     y_host = bl.bitlinear_forward_host(x.pin_memory(), packed, s_w, b)
     assert torch.equal(y_dev.view(torch.int16), y_host.view(torch.int16))
+    # the stream-ordered variant: several calls in flight, each with its own
+    # workspace and output, one synchronisation at the end
+    xs = [synth.normal_bf16(55, i, tuple(x.shape)).pin_memory() for i in range(3)]
+    outs = [bl.bitlinear_forward_host_async(xi, packed, s_w, b, flags=bl.WEIGHTS_RESIDENT) for xi in xs]
+    torch.cuda.current_stream().synchronize()
+    for xi, yi in zip(xs, outs):
+        want = bl.bitlinear_forward(xi.cuda(), packed, s_w, b).cpu()
+        assert torch.equal(yi.view(torch.int16), want.view(torch.int16))
 
 
 @pytest.mark.parametrize("M", [4, 16, 40])
