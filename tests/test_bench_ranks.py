@@ -74,3 +74,26 @@ def test_single_process_needs_no_process_group():
     assert bench.world_size() == 1
     assert bench.elapsed_max_over_ranks(3.5) == 3.5
     assert bench.whole_job_gbs(2e9, 10, 1000.0, 1) == pytest.approx(20.0)
+
+
+def test_reference_arm_prints_one_contract_line(capsys):
+    # --impl reference on one process: the CPU oracle timed on the decode
+    # sweep, printed as the reference arm's JSON line
+    sys.path.insert(0, ROOT)
+    import json
+    import bench
+
+    class A:
+        steps, gpus = 1, 1
+
+    assert bench.reference_arm(A) == 0
+    lines = [l for l in capsys.readouterr().out.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["unit"] == "GB/s" and d["higher_is_better"] is True
+    assert d["value"] > 0 and d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
+    assert "workload" in d["config"]
