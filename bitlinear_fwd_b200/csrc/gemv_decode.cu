@@ -21,7 +21,10 @@
 //   * The consumer warps form each token's absmax over the row, s_x =
 //     127 / max(absmax, 1e-5) in float32, and q = round_half_even(x s_x) as
 //     int8 into shared memory, one 4096-k round at a time, with the sum of q
-//     per token.  Pre-quantised int8 input is copied in instead.
+//     per token.  For M <= 4 and K <= 4096 each lane's share of x is read
+//     once and held in registers between the two steps; otherwise x is read
+//     again for the quantising step.  Pre-quantised int8 input is copied in
+//     instead.
 //   * In round r warp w takes sub-box w (k = 4096r + 512w ..) of every unit
 //     of the CTA, so it loads its x fragment once per round and reuses it for
 //     all units.  Per sub-box a thread
@@ -32,7 +35,9 @@
 //     4^i sum(c q); the fields are combined with exact shifts and added to the
 //     unit's int32 sums in shared memory.
 //   * Epilogue: acc = sum(c q) - sum(q) = sum(u q); y = acc / (s_x s_w)
-//     (+ bias) -> bf16.
+//     (+ bias) -> bf16, with s_w the scale of the row's layer when several
+//     layers are stacked.  The bf16-faithful mode rounds the scale, the
+//     products, the sum and the quotient to bf16 as a bf16 module does.
 // Rows beyond N and k beyond K are zero-filled by TMA (code 0), so they add
 // nothing whatever the x bytes there are.
 //
