@@ -309,13 +309,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 cudaError_t launch_gemm_prefill(const ForwardArgs& a, int num_sms, cudaStream_t stream) {
   if (a.M <= 0) return cudaSuccess;
-  static bool attr_done = false;
-  if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kSmemBytes));
-    if (e != cudaSuccess) return e;
-    attr_done = true;
-  }
+  static unsigned long long attr_done = 0;        // one bit per device
+  cudaError_t ea = set_smem_attr_once(gemm_prefill_kernel, static_cast<int>(kSmemBytes), &attr_done);
+  if (ea != cudaSuccess) return ea;
   CUtensorMap tm_x, tm_w;
   if (!encode_2d_u8(&tm_x, a.xq, a.K, a.M, a.K, BK, BT, CU_TENSOR_MAP_SWIZZLE_128B)) return cudaErrorInvalidValue;
   if (!encode_2d_u8(&tm_w, a.packed, a.K / 4, a.N, a.K / 4, BK / 4, BW, CU_TENSOR_MAP_SWIZZLE_NONE))

@@ -565,12 +565,9 @@ template <int NT>
 cudaError_t launch_nt(const CUtensorMap& tm3, const CUtensorMap& tm2, const DecodeArgs& a, const DecodePlan& p,
                       cudaStream_t stream) {
   auto kern = decode_kernel<NT>;
-  static bool attr_done = false;
-  if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-    if (e != cudaSuccess) return e;
-    attr_done = true;
-  }
+  static unsigned long long attr_done = 0;        // one bit per device
+  cudaError_t ea = set_smem_attr_once(kern, 227 * 1024, &attr_done);
+  if (ea != cudaSuccess) return ea;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.grid, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);

@@ -65,6 +65,20 @@ struct ForwardArgs {
 cudaError_t launch_dequant(const uint8_t* packed, int64_t N, int64_t K, const float* w_scale, uint16_t* w_bf16,
                            int num_sms, cudaStream_t stream);
 
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per kernel and
+// device (the attribute belongs to the device that is current at the call)
+template <typename Kern>
+cudaError_t set_smem_attr_once(Kern kern, int bytes, unsigned long long* done_mask) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (__atomic_load_n(done_mask, __ATOMIC_ACQUIRE) & bit) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) __atomic_fetch_or(done_mask, bit, __ATOMIC_RELEASE);
+  return e;
+}
+
 // ---- decode engine, M <= 16 (gemv_decode.cu) --------------------------------
 struct DecodeArgs {
   const uint16_t* x;      // bf16 [M, K], quantised inside the kernel; or null
