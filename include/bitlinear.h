@@ -22,6 +22,8 @@
  *   - the contraction is exact in int32 (|acc| <= 127*K);
  *   - d = s_x*s_w (float32), y32 = float(acc) / d (float32, correctly
  *     rounded), y32 += float(bias) if a bias is given, y = bf16_rne(y32).
+ *   The flag BITLINEAR_BF16_FAITHFUL switches to the rounding of a bf16
+ *   module instead (see its definition below).
  *
  * Conventions for every entry point:
  *   - Shapes: x is [M, K] row-major, W is [N, K] (nn.Linear [out, in]),
@@ -31,7 +33,9 @@
  *   - Every pointer argument is a DEVICE pointer unless its name ends in
  *     _host.  Device pointers must be 16-byte aligned (BITLINEAR_ERR_ALIGN
  *     otherwise).  All buffers are owned by the caller; the library
- *     allocates nothing and keeps no state between calls.
+ *     allocates nothing and keeps no data between calls (it caches
+ *     per-device facts: compute capability, SM count, kernel attributes;
+ *     bitlinear_forward_noalloc has its own fixed scratch array).
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Work
  *     is enqueued on it and the call returns without synchronising, except
  *     where stated.  Calls on different streams with distinct workspaces
