@@ -19,11 +19,13 @@
 //   warps 4..7   weight unpack: thread = weight row; its 32 packed bytes become
 //                32 registers of codes c = u + 1 (one word -> four registers
 //                of four consecutive k) and one tcgen05.st of 32 columns
-//   warps 8..11  epilogue of the previous tile while the MMAs of the next one
-//                run: tcgen05.ld of a row's 128 accumulators, acc - sum_k q
-//                (code offset), y = acc / (s_x s_w) (+ bias), bf16 stores;
-//                s_w is the scale of the row's group (stacked layers)
-//                (coalesced along weight rows)
+//   warps 8..15  epilogue of the previous tile while the MMAs of the next one
+//                run; warps w and w + 4 share a lane quarter of tensor memory
+//                and take one half of the tile's tokens each: tcgen05.ld of a
+//                row's 64 accumulators, acc - sum_k q (code offset),
+//                y = acc / (s_x s_w) (+ bias), bf16 stores (coalesced along
+//                weight rows); s_w is the scale of the row's group (stacked
+//                layers)
 // Barriers: per stage full (TMA bytes landed), ready (A stage written),
 // empty (MMAs done); per accumulator buffer acc_full (tile's MMAs done) and
 // acc_empty (epilogue has read it).  Shared memory carries only x and the
@@ -42,7 +44,9 @@ constexpr int BW = 128;                      // weight rows per tile (MMA M)
 constexpr int BT = 128;                      // tokens per tile (MMA N)
 constexpr int BK = 128;                      // k per block
 constexpr int STAGES = 6;
-constexpr int kThreads = 384;
+constexpr int kThreads = 512;
+constexpr int kEpiWarps = 8;                // two per tensor-memory lane quarter
+constexpr int kEpiCols = BT / 2;            // tokens of a tile per epilogue warp
 constexpr uint32_t kXBytes = BT * BK;        // 16 KB x tile per stage
 constexpr uint32_t kWpBytes = BW * BK / 4;   // 4 KB packed weights per stage
 constexpr uint32_t kACols = BK / 4;          // tensor-memory columns of one A stage
@@ -85,7 +89,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 4);
+      mbar_init(&acc_empty[b], kEpiWarps);
     }
     mbar_init(drain, 1);
     *failed = 0;
@@ -201,7 +205,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp >= 8) {
     // ---------------- epilogue ----------------
     const int q = warp & 3;
-    const int et = threadIdx.x - 256;             // 0..127
+    const int et = threadIdx.x - 256;             // 0..255
+    const int half = (warp - 8) >> 2;             // which half of the tile's tokens
     const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
     pdl_wait_primary();
     float swg[kMaxGroups];                         // s_w of each row group
@@ -216,15 +221,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int b = j & 1;
       const int n0 = (tile % wtiles) * BW, m0 = (tile / wtiles) * BT;
       // per-token s_x and row sums of this tile
-      asm volatile("bar.sync 1, 128;" ::: "memory");   // previous tile's readers are done
-      {
+      asm volatile("bar.sync 1, 256;" ::: "memory");   // previous tile's readers are done
+      if (et < BT) {
         // one float32 layer: d = s_x * s_w per token; otherwise s_x (the
         // row's scale enters per element)
         const int m = m0 + et;
         d_s[et] = m < a.M ? (simple ? __fmul_rn(a.s_x[m], swg[0]) : a.s_x[m]) : 1.0f;
         rs_s[et] = m < a.M ? a.rowsum[m] : 0;
       }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
+      asm volatile("bar.sync 1, 256;" ::: "memory");
       bool ok = !__any_sync(0xffffffffu, *failed != 0);
       if (ok) ok = mbar_wait(&acc_full[b], (j >> 1) & 1, wait_ns);
       ok = __all_sync(0xffffffffu, ok);             // warp-uniform decision
@@ -242,11 +247,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (g < a.ngroups && n >= a.group_end[g - 1]) s_w = swg[g];
       if (a.faithful) s_w = bf16_round(s_w);       // a bf16 module holds s_w in bf16
 #pragma unroll 1
-      for (int c = 0; c < BT / 32; ++c) {
+      for (int c = half * (kEpiCols / 32); c < (half + 1) * (kEpiCols / 32); ++c) {
         uint32_t r[32];
         tmem_ld_32x32b_x32(tmem_base + b * BT + lane_base + 32 * c, r);
         tmem_wait_ld();
-        if (c == BT / 32 - 1) {
+        if (c == (half + 1) * (kEpiCols / 32) - 1) {
           // the whole accumulator is in registers: hand the buffer back
           tc_fence_before();
           __syncwarp();
