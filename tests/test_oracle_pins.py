@@ -7,6 +7,9 @@ forms and invariants.  Sources: the Falcon-Edge blog (section "Falcon-Edge,
 a series of universal models": activation_norm_quant, _weight_quant,
 BitLinear) and the 2-bit storage remark in the Hacker News comments of
 "BitNet: inference framework for 1-bit LLMs" (GeekNews).
+
+Every pin runs twice: against the numpy oracle and against the C++ oracle
+(``oracle.cpp``), two independent restatements of the same pages.
 """
 
 import itertools
@@ -19,11 +22,23 @@ import numpy as np
 import pytest
 import torch
 
-import oracle
+import oracle as numpy_oracle
 import synth
+from oracle import cpp as cpp_oracle
 from tests.exact import f32_exact, nearest_bf16_bits, nearest_f32
 
 RNG = np.random.default_rng(20260101)
+
+ORACLES = {"numpy": numpy_oracle, "cpp": cpp_oracle}
+oracle = numpy_oracle          # the oracle under test; set per test below
+
+
+@pytest.fixture(params=sorted(ORACLES), autouse=True)
+def which_oracle(request):
+    global oracle
+    saved, oracle = oracle, ORACLES[request.param]
+    yield request.param
+    oracle = saved
 
 
 def bits_of_bf16(values):
@@ -334,7 +349,16 @@ def test_bf16_conversions():
 # The pins catch planted mistakes (mutations planted in the oracle, on CPU)
 # --------------------------------------------------------------------------
 
-def test_pins_catch_planted_mistakes(golden_dir, monkeypatch):
+def test_pins_catch_planted_mistakes(golden_dir, monkeypatch, tmp_path, which_oracle):
+    if which_oracle == "cpp":
+        # the same three mistakes, compiled into copies of the C++ oracle
+        for mistake in (1, 2, 3):
+            with cpp_oracle.planted(mistake, str(tmp_path)):
+                with pytest.raises(AssertionError):
+                    check_hand_worked(golden_dir)
+                    test_pack_layout_fixture(golden_dir)
+        check_hand_worked(golden_dir)
+        return
     orig_act, orig_epi, orig_pack = oracle.act_quant, oracle.epilogue, oracle.pack
 
     def act_floor(xb):                      # floor instead of round
