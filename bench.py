@@ -23,7 +23,9 @@ Also on the line:
   dequant_export, stack3b_decode
                 the bf16 export kernel's GB/s, and the 3B-class 26-layer
                 projection stack at M=1 with and without grouped calls
-  cpu_baseline  the CPU oracle on a bounded sample of the decode workload
+  cpu_baseline  the numpy CPU oracle on a bounded sample of the decode
+                workload, with the plain C++ oracle timed beside it
+                (cpu_baseline.cpp_oracle, one thread)
   clocks        nvidia-smi samples taken while the workload ran
 
 With --gpus N > 1 (under torchrun) every rank runs the same workload on its
@@ -501,11 +503,15 @@ def run_dequant(hbm_gbs, reps=20):
 # ---------------------------------------------------------------------------
 
 class OracleDecode:
-    """The CPU oracle on the decode workload (all six problems, every weight
-    row).  Inputs are generated and packed by the oracle once, untimed."""
+    """A CPU oracle on the decode workload (all six problems, every weight
+    row): the numpy oracle, or with ``impl="cpp"`` the plain C++ one.
+    Inputs are generated and packed by that oracle once, untimed."""
 
-    def __init__(self):
-        import oracle
+    def __init__(self, impl="numpy"):
+        if impl == "cpp":
+            from oracle import cpp as oracle
+        else:
+            import oracle
         self.oracle = oracle
         try:
             from threadpoolctl import threadpool_info
@@ -522,9 +528,16 @@ class OracleDecode:
             packed, s_w, _ = wcache[key]
             self.items.append((synth.bf16_bits(c.x()), packed, s_w, synth.bf16_bits(c.bias()),
                                decode_bytes(c.M, c.N, c.K)))
-        self.desc = ("oracle.forward (act quant, unpack, exact contraction, epilogue) on the 6 decode problems "
-                     "with every weight row, packing untimed; numpy elementwise steps single-threaded, "
-                     f"float64 matmul on {self.blas} BLAS threads")
+        if impl == "cpp":
+            self.cores = 1
+            self.desc = ("the C++ oracle's forward (plain loops: act quant, unpack, int64 contraction, "
+                         "epilogue) on the 6 decode problems with every weight row, packing untimed; "
+                         "one thread")
+        else:
+            self.cores = self.blas
+            self.desc = ("oracle.forward (act quant, unpack, exact contraction, epilogue) on the 6 decode "
+                         "problems with every weight row, packing untimed; numpy elementwise steps "
+                         f"single-threaded, float64 matmul on {self.blas} BLAS threads")
 
     def step(self):
         """One pass over the workload; returns (bytes, seconds)."""
@@ -535,6 +548,26 @@ class OracleDecode:
             s += time.perf_counter() - t0
             b += nbytes
         return b, s
+
+
+def timed_oracle(impl, budget_s, max_passes=8):
+    """Passes of one CPU oracle over the decode workload until ``budget_s``
+    seconds of oracle time; a cpu_baseline-style dict."""
+    od = OracleDecode(impl)
+    b, s, n = 0, 0.0, 0
+    while s < budget_s and n < max_passes:
+        bb, ss = od.step()
+        b, s, n = b + bb, s + ss, n + 1
+    return {"value": round(b / s / 1e9, 4), "unit": "GB/s", "cores": od.cores, "kind": "oracle",
+            "sample": f"{n} passes ({s:.1f} s) of " + od.desc}
+
+
+def cpp_oracle_baseline(budget_s=5.0):
+    """The C++ oracle timed beside the numpy one; never fails the line."""
+    try:
+        return timed_oracle("cpp", budget_s)
+    except Exception as e:                      # e.g. no C++ compiler on the host
+        return {"unavailable": f"{type(e).__name__}: {e}"}
 
 
 def reference_arm(args):
@@ -558,8 +591,9 @@ def reference_arm(args):
             "config": {"workload": "decode GEMV sweep: M in {1,4,16}, (K,N) in {(4096,4096),(4096,11008)}; "
                                    "the CPU oracle, the only reference implementation of this method",
                        "parallelism": "rank 0 host cores"},
-            "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": od.blas, "kind": "oracle",
-                             "sample": f"{steps} passes of " + od.desc},
+            "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": od.cores, "kind": "oracle",
+                             "sample": f"{steps} passes of " + od.desc,
+                             "cpp_oracle": cpp_oracle_baseline()},
             "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -623,13 +657,8 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
-        od = OracleDecode()
-        b, s, n = 0, 0.0, 0
-        while s < 10.0 and n < 8:
-            bb, ss = od.step()
-            b, s, n = b + bb, s + ss, n + 1
-        cpu = {"value": round(b / s / 1e9, 4), "unit": "GB/s", "cores": od.blas, "kind": "oracle",
-               "sample": f"{n} passes ({s:.1f} s) of " + od.desc}
+        cpu = timed_oracle("numpy", 10.0)
+        cpu["cpp_oracle"] = cpp_oracle_baseline()
 
     line = {
         "metric": "BitLinear decode GB/s (% of HBM peak); prefill int8 TOPS (% TC peak)",

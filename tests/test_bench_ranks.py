@@ -97,3 +97,7 @@ def test_reference_arm_prints_one_contract_line(capsys):
     assert d["value"] > 0 and d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
     assert "workload" in d["config"]
+    # the plain C++ oracle timed beside the numpy one, on one thread
+    cpp = d["cpu_baseline"]["cpp_oracle"]
+    assert "unavailable" not in cpp, cpp
+    assert cpp["value"] > 0 and cpp["cores"] == 1 and cpp["kind"] == "oracle" and cpp["unit"] == "GB/s"
