@@ -23,6 +23,8 @@ Also on the line:
   dequant_export, stack3b_decode
                 the bf16 export kernel's GB/s, and the 3B-class 26-layer
                 projection stack at M=1 with and without grouped calls
+  pack          weight ternarisation and packing timed alone on the GPU
+                (28672 x 8192), and both CPU oracles' packing beside it
   cpu_baseline  the numpy CPU oracle on a bounded sample of the decode
                 workload, with the plain C++ oracle timed beside it
                 (cpu_baseline.cpp_oracle, one thread)
@@ -500,6 +502,77 @@ def run_dequant(hbm_gbs, reps=20):
             "frac": round(gbs / hbm_gbs, 4), "note": "output 470 MB > L2, each launch streams it to DRAM"}
 
 
+def pack_bytes(N, K):
+    """Algorithmic bytes of one weight packing: W read twice (the mean must be
+    complete before any weight is ternarised, and these W are larger than
+    L2), the 2-bit codes written, the scale and the mean."""
+    return 2 * 4 * N * K + N * K // 4 + 8
+
+
+def run_pack(hbm_gbs, reps=10):
+    """Weight ternarisation and packing timed alone (bitlinear_pack_weights:
+    absmean bins, finalize, ternarise-and-pack, three kernels) on the
+    100B-class gate shape, 28672 x 8192 fp32 (940 MB, larger than L2), CUDA
+    events over ``reps`` calls on the current stream."""
+    import bitlinear_fwd_b200 as bl
+    N, K = 28672, 8192
+    g = torch.Generator(device="cuda").manual_seed(12)
+    w = torch.randn((N, K), device="cuda", generator=g).mul_(0.01)
+    packed = torch.empty((N, K // 4), dtype=torch.uint8, device="cuda")
+    s_w = torch.empty(1, dtype=torch.float32, device="cuda")
+    mean = torch.empty(1, dtype=torch.float32, device="cuda")
+    ws = torch.empty(bl.pack_workspace_bytes(N, K), dtype=torch.uint8, device="cuda")
+    lib, st = bl.lib(), torch.cuda.current_stream().cuda_stream
+    call = lambda: lib.bitlinear_pack_weights(w.data_ptr(), N, K, packed.data_ptr(), s_w.data_ptr(),
+                                              mean.data_ptr(), ws.data_ptr(), ws.numel(), st)
+    for _ in range(3):
+        assert call() == 0
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        call()
+    e1.record()
+    e1.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / reps
+    nbytes = pack_bytes(N, K)
+    gbs = nbytes / (us * 1e-6) / 1e9
+    del w, packed, ws
+    return {"kernels": "absmean_bins_kernel + absmean_finalize_kernel + ternarise_pack_kernel",
+            "shape": [N, K], "us_per_call": round(us, 1), "bytes_per_call": nbytes,
+            "achieved": round(gbs, 1), "unit": "GB/s", "peak": hbm_gbs, "frac": round(gbs / hbm_gbs, 4),
+            "note": "once per weight matrix, outside the forward; bytes = 8 B/weight (W read twice) "
+                    "+ 0.25 B/weight written"}
+
+
+def oracle_pack_baseline(budget_s=6.0):
+    """Both CPU oracles' pack_weights on the decode sweep's 11008 x 4096
+    weights, bytes counted as for the GPU."""
+    out = {}
+    w = None
+    for impl in ("numpy", "cpp"):
+        try:
+            if impl == "cpp":
+                from oracle import cpp as orc
+            else:
+                import oracle as orc
+            if w is None:
+                c = [c for c in wl.workload2() if c.N == 11008][0]
+                w = c.w().numpy()
+            N, K = w.shape
+            s, n = 0.0, 0
+            while s < budget_s / 2 and n < 4:
+                t0 = time.perf_counter()
+                orc.pack_weights(w)
+                s += time.perf_counter() - t0
+                n += 1
+            out[impl] = {"value": round(pack_bytes(N, K) * n / s / 1e9, 3), "unit": "GB/s",
+                         "cores": 1, "sample": f"{n} calls ({s:.1f} s) of pack_weights on [{N}, {K}] fp32"}
+        except Exception as e:
+            out[impl] = {"unavailable": f"{type(e).__name__}: {e}"}
+    return out
+
+
 # ---------------------------------------------------------------------------
 
 class OracleDecode:
@@ -654,11 +727,16 @@ def main():
     pre = None if args.no_prefill else run_prefill(args, bf16_tflops, peak_kind, l2_bytes)
     deq = run_dequant(hbm_gbs)
     stack = run_stack3b(hbm_gbs)
+    try:
+        pack = {"gpu": run_pack(hbm_gbs)}
+    except Exception as e:
+        pack = {"gpu": {"unavailable": f"{type(e).__name__}: {e}"}}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         cpu = timed_oracle("numpy", 10.0)
         cpu["cpp_oracle"] = cpp_oracle_baseline()
+        pack["cpu_oracle"] = oracle_pack_baseline()
 
     line = {
         "metric": "BitLinear decode GB/s (% of HBM peak); prefill int8 TOPS (% TC peak)",
@@ -687,6 +765,7 @@ def main():
         "prefill": pre,
         "dequant_export": deq,
         "stack3b_decode": stack,
+        "pack": pack,
         "cpu_baseline": cpu,
         "clocks": clocks,
     }
