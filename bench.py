@@ -23,6 +23,8 @@ Also on the line:
   dequant_export, stack3b_decode
                 the bf16 export kernel's GB/s, and the 3B-class 26-layer
                 projection stack at M=1 with and without grouped calls
+  ffn100b_stack the 100B-class FFN stack (13 layers, 2.29 GB of packed
+                weights) at M in {1, 8, 64, 512}: tokens/s per stack pass
   pack          weight ternarisation and packing timed alone on the GPU
                 (28672 x 8192), and both CPU oracles' packing beside it
   cpu_baseline  the numpy CPU oracle on a bounded sample of the decode
@@ -502,6 +504,69 @@ def run_dequant(hbm_gbs, reps=20):
             "frac": round(gbs / hbm_gbs, 4), "note": "output 470 MB > L2, each launch streams it to DRAM"}
 
 
+def run_ffn100b(hbm_gbs, int8_tops, Ms=(1, 8, 64, 512), layers=13, reps=10):
+    """The 100B-class FFN stack: hidden 8192, FFN 28672; per layer gate and
+    up (8192 -> 28672, the same input) and down (28672 -> 8192); 13 layers
+    of independent weights (2.29 GB packed, far above L2).  One
+    bitlinear_forward per projection (3 launches per layer), weights
+    resident, one CUDA graph per pass of the whole stack.  Reports the
+    equivalent tokens/s of the stack, and the weight stream (GB/s, M <= 8:
+    the decode engine) or int8 TOPS (M >= 64: the prefill engine) against
+    its roofline."""
+    import bitlinear_fwd_b200 as bl
+    H, F = 8192, 28672
+    gen = torch.Generator(device="cuda").manual_seed(31)
+    lay = [{"gate": _random_packed(F, H, gen), "up": _random_packed(F, H, gen),
+            "down": _random_packed(H, F, gen), "s": torch.full((1,), 80.0, device="cuda")}
+           for _ in range(layers)]
+    wbytes = layers * 3 * F * H // 4
+    R = bl.WEIGHTS_RESIDENT
+    out = {"workload": f"100B-class FFN stack: {layers} layers x (gate, up 8192->28672; down 28672->8192), "
+                       "random valid 2-bit codes, no bias",
+           "layers": layers, "weights_bytes_per_pass": wbytes, "launches_per_pass": 3 * layers, "per_M": []}
+    for M in Ms:
+        x = torch.randn((M, H), device="cuda", generator=gen).to(torch.bfloat16)
+        xd = torch.randn((M, F), device="cuda", generator=gen).to(torch.bfloat16)
+        yg = torch.empty((M, F), dtype=torch.bfloat16, device="cuda")
+        yu = torch.empty((M, F), dtype=torch.bfloat16, device="cuda")
+        yd = torch.empty((M, H), dtype=torch.bfloat16, device="cuda")
+        ws = bl.workspace(M, F, F, "cuda")
+
+        def stack():
+            for L in lay:
+                bl.bitlinear_forward(x, L["gate"], L["s"], ws=ws, out=yg, flags=R)
+                bl.bitlinear_forward(x, L["up"], L["s"], ws=ws, out=yu, flags=R)
+                bl.bitlinear_forward(xd, L["down"], L["s"], ws=ws, out=yd, flags=R)
+
+        stack()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            stack()
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            g.replay()
+        e1.record()
+        e1.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / reps
+        ops = layers * 3 * 2 * M * F * H
+        row = {"M": M, "us_per_pass": round(us, 1), "tokens_per_s": round(M / (us * 1e-6), 1)}
+        if M <= 16:
+            gbs = wbytes / (us * 1e-6) / 1e9
+            row.update({"bound": "hbm", "weights_gbs": round(gbs, 1), "frac": round(gbs / hbm_gbs, 4)})
+        else:
+            tops = ops / (us * 1e-6) / 1e12
+            row.update({"bound": "tensor", "tops": round(tops, 1), "frac": round(tops / int8_tops, 4)})
+        out["per_M"].append(row)
+        del g, x, xd, yg, yu, yd, ws
+    del lay
+    return out
+
+
 def pack_bytes(N, K):
     """Algorithmic bytes of one weight packing: W read twice (the mean must be
     complete before any weight is ternarised, and these W are larger than
@@ -737,6 +802,10 @@ def main():
         cpu = timed_oracle("numpy", 10.0)
         cpu["cpp_oracle"] = cpp_oracle_baseline()
         pack["cpu_oracle"] = oracle_pack_baseline()
+    try:
+        ffn = run_ffn100b(hbm_gbs, bf16_tflops * INT8_OVER_BF16)
+    except Exception as e:
+        ffn = {"unavailable": f"{type(e).__name__}: {e}"}
 
     line = {
         "metric": "BitLinear decode GB/s (% of HBM peak); prefill int8 TOPS (% TC peak)",
@@ -766,6 +835,7 @@ def main():
         "dequant_export": deq,
         "stack3b_decode": stack,
         "pack": pack,
+        "ffn100b_stack": ffn,
         "cpu_baseline": cpu,
         "clocks": clocks,
     }
