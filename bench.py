@@ -23,6 +23,8 @@ Also on the line:
   dequant_export, stack3b_decode
                 the bf16 export kernel's GB/s, and the 3B-class 26-layer
                 projection stack at M=1 with and without grouped calls
+  stack3b_prefill the same 3B-class stack at M=2048 (prefill engine), with
+                int8 TOPS
   ffn100b_stack the 100B-class FFN stack (13 layers, 2.29 GB of packed
                 weights) at M in {1, 8, 64, 512}: tokens/s per stack pass
   pack          weight ternarisation and packing timed alone on the GPU
@@ -404,14 +406,15 @@ def _random_packed(N, K, gen):
     return lut[torch.randint(0, 81, (N, K // 4), device="cuda", generator=gen)]
 
 
-def run_stack3b(hbm_gbs, M=1, layers=26, reps=20):
+def run_stack3b(hbm_gbs, M=1, layers=26, reps=20, int8_tops=None):
     """The 3B-class decoder projection stack at M tokens: per layer q/k/v
     (3200 -> 3 x 3200), o (3200 -> 3200), gate/up (3200 -> 2 x 8640), down
     (8640 -> 3200); 26 layers of independent weights (806 MB packed).
     Timed two ways: one bitlinear_forward per projection (7 launches per
     layer) and with the shared-input groups fused (q/k/v and gate/up through
     bitlinear_forward_grouped: 4 launches per layer).  Weights resident,
-    replayed as one CUDA graph per pass."""
+    replayed as one CUDA graph per pass.  With M > 16 (the prefill engine)
+    and ``int8_tops`` given, int8 TOPS against that peak are added."""
     import bitlinear_fwd_b200 as bl
     H, F = 3200, 8640
     gen = torch.Generator(device="cuda").manual_seed(21)
@@ -470,7 +473,11 @@ def run_stack3b(hbm_gbs, M=1, layers=26, reps=20):
         out[name] = {"us_per_pass": round(us, 1), "tokens_per_s": round(M / (us * 1e-6), 1),
                      "weights_gbs": round(wbytes / (us * 1e-6) / 1e9, 1),
                      "frac_of_hbm": round(wbytes / (us * 1e-6) / 1e9 / hbm_gbs, 4),
-                     "launches_per_pass": launches * layers}
+                     "launches_per_pass": launches * layers * (2 if M > 16 else 1)}   # act quant + GEMM
+        if M > 16 and int8_tops:
+            ops = 2 * M * layers * (3 * H * H + H * H + 2 * F * H + H * F)
+            tops = ops / (us * 1e-6) / 1e12
+            out[name].update({"tops": round(tops, 1), "frac_of_int8": round(tops / int8_tops, 4)})
         del g
     out["weights_bytes_per_pass"] = wbytes
     return out
@@ -523,7 +530,8 @@ def run_ffn100b(hbm_gbs, int8_tops, Ms=(1, 8, 64, 512), layers=13, reps=10):
     R = bl.WEIGHTS_RESIDENT
     out = {"workload": f"100B-class FFN stack: {layers} layers x (gate, up 8192->28672; down 28672->8192), "
                        "random valid 2-bit codes, no bias",
-           "layers": layers, "weights_bytes_per_pass": wbytes, "launches_per_pass": 3 * layers, "per_M": []}
+           "layers": layers, "weights_bytes_per_pass": wbytes, "calls_per_pass": 3 * layers,
+           "per_M": []}
     for M in Ms:
         x = torch.randn((M, H), device="cuda", generator=gen).to(torch.bfloat16)
         xd = torch.randn((M, F), device="cuda", generator=gen).to(torch.bfloat16)
@@ -554,7 +562,8 @@ def run_ffn100b(hbm_gbs, int8_tops, Ms=(1, 8, 64, 512), layers=13, reps=10):
         e1.synchronize()
         us = e0.elapsed_time(e1) * 1e3 / reps
         ops = layers * 3 * 2 * M * F * H
-        row = {"M": M, "us_per_pass": round(us, 1), "tokens_per_s": round(M / (us * 1e-6), 1)}
+        row = {"M": M, "us_per_pass": round(us, 1), "tokens_per_s": round(M / (us * 1e-6), 1),
+               "launches_per_pass": 3 * layers * (2 if M > 16 else 1)}
         if M <= 16:
             gbs = wbytes / (us * 1e-6) / 1e9
             row.update({"bound": "hbm", "weights_gbs": round(gbs, 1), "frac": round(gbs / hbm_gbs, 4)})
@@ -806,6 +815,10 @@ def main():
         ffn = run_ffn100b(hbm_gbs, bf16_tflops * INT8_OVER_BF16)
     except Exception as e:
         ffn = {"unavailable": f"{type(e).__name__}: {e}"}
+    try:
+        stack_pre = run_stack3b(hbm_gbs, M=2048, reps=5, int8_tops=bf16_tflops * INT8_OVER_BF16)
+    except Exception as e:
+        stack_pre = {"unavailable": f"{type(e).__name__}: {e}"}
 
     line = {
         "metric": "BitLinear decode GB/s (% of HBM peak); prefill int8 TOPS (% TC peak)",
@@ -836,6 +849,7 @@ def main():
         "stack3b_decode": stack,
         "pack": pack,
         "ffn100b_stack": ffn,
+        "stack3b_prefill": stack_pre,
         "cpu_baseline": cpu,
         "clocks": clocks,
     }
