@@ -1,6 +1,9 @@
 """Host-only checks of the C ABI: the library loads, exports every function
 that include/bitlinear.h declares, answers size queries, and rejects bad
-arguments before touching the GPU (no compute call is made here)."""
+arguments before touching the GPU.  On a machine without a GPU, valid
+arguments are also shown to pass every host check and stop at the device
+check; that test is skipped wherever a GPU is visible, because its fake
+pointers would then reach a kernel launch."""
 
 import ctypes
 import os
@@ -103,3 +106,79 @@ def test_argument_errors_without_gpu(lib):
     # stream-ordered host forward: flag check first, then the host argument checks
     assert lib.bitlinear_forward_host_async(16, 8, 256, 16, 512, 16, None, 16, 4, 16, 1 << 20, None) == -2
     assert lib.bitlinear_forward_host_async(None, 8, 256, 16, 512, 16, None, 16, 0, 16, 1 << 20, None) == -1
+
+
+def test_more_argument_errors_without_gpu(lib):
+    """Every entry point rejects bad shapes, NULL and misaligned pointers and
+    short workspaces on the host, before any CUDA call."""
+    # sizes beyond the documented limits
+    assert _fwd(lib, N=(1 << 23) + 1) == -2
+    assert _fwd(lib, K=(1 << 19) + 64) == -2
+    assert _fwd(lib, M=(1 << 23) + 1) == -2
+    assert lib.bitlinear_pack_weights(16, 1 << 23, 1 << 19, 16, 16, None, 16, 4096, None) == -2   # N*K >= 2^40
+    # misaligned scale, workspace and output
+    assert _fwd(lib, s=20) == -3
+    assert _fwd(lib, ws=24) == -3
+    assert _fwd(lib, y=18) == -3
+    # M == 0 is a valid empty call that touches nothing
+    assert _fwd(lib, M=0) == 0
+    # flags
+    assert lib.bitlinear_forward_ex(16, 8, 256, 16, 512, 16, None, 16, 4, 16, 1 << 20, None) == -2
+    # pre-quantised activations
+    q8 = lib.bitlinear_forward_q8
+    assert q8(None, 16, 16, 8, 256, 16, 512, 16, None, 16, 16, 256, None) == -1
+    assert q8(16, 16, None, 8, 256, 16, 512, 16, None, 16, 16, 256, None) == -1
+    assert q8(16, 18, 16, 8, 256, 16, 512, 16, None, 16, 16, 256, None) == -3
+    assert q8(16, 16, 16, 8, 100, 16, 512, 16, None, 16, 16, 256, None) == -2
+    assert q8(16, 16, 16, 8, 256, 16, 512, 16, None, 16, 16, 128, None) == -4
+    assert q8(16, 16, 16, 0, 256, 16, 512, 16, None, 16, 16, 256, None) == 0
+    # host buffers: no alignment rule for host x and y, but a larger workspace
+    dev_ws = bl.workspace_bytes(8, 512, 256)
+    host = lib.bitlinear_forward_host
+    assert host(16, 8, 256, 16, 512, 16, None, 16, 16, dev_ws, None) == -4
+    assert host(16, 8, 256, 16, 512, 16, None, None, 16, 1 << 20, None) == -1
+    assert host(16, 8, 256, 18, 512, 16, None, 16, 16, 1 << 20, None) == -3     # packed weights are on the device
+    # the no-allocation forward: its fixed scratch bounds M*K
+    na = lib.bitlinear_forward_noalloc
+    assert na(16, 64, 1 << 19, 16, 512, 16, None, 16, None) == -4
+    assert na(16, 8, 100, 16, 512, 16, None, 16, None) == -2
+    # quantisation alone
+    assert lib.bitlinear_quant_act(None, 4, 256, 16, 16, None, None) == -1
+    assert lib.bitlinear_quant_act(16, 4, 256, 16, 18, None, None) == -3
+
+
+def _no_cuda_device():
+    import torch
+    return not torch.cuda.is_available() and torch.cuda.device_count() == 0
+
+
+@pytest.mark.skipif(not _no_cuda_device(),
+                    reason="the fake pointers of this test would reach a kernel launch on a GPU")
+def test_valid_arguments_pass_every_host_check(lib):
+    """Valid arguments get through every host check of each entry point and
+    stop only at the device check (no GPU here: BITLINEAR_ERR_CUDA or
+    BITLINEAR_ERR_DEVICE), so the checks reject nothing the header allows."""
+    no_device = (-5, -7)
+    rows = (ctypes.c_int64 * 3)(100, 200, 212)
+    host_ws = bl.host_workspace_bytes(8, 512, 256)
+    calls = {
+        "forward": _fwd(lib),
+        "forward_ex resident": lib.bitlinear_forward_ex(16, 8, 256, 16, 512, 16, None, 16, 1, 16, 1 << 20, None),
+        "forward_ex both flags": lib.bitlinear_forward_ex(16, 8, 256, 16, 512, 16, 32, 16, 3, 16, 1 << 20, None),
+        "forward M=16": _fwd(lib, M=16),
+        "forward M=17": _fwd(lib, M=17),
+        "grouped": lib.bitlinear_forward_grouped(16, 8, 256, 16, rows, 3, 16, None, 16, 2, 16, 1 << 20, None),
+        "q8": lib.bitlinear_forward_q8(16, 16, 16, 8, 256, 16, 512, 16, None, 16, 16, 256, None),
+        "debug engine 1": lib.bitlinear_forward_debug(16, 16, 256, 16, 512, 16, None, 16, None, None, None,
+                                                      None, 1, 16, 1 << 20, None),
+        "debug_ex engine 2": lib.bitlinear_forward_debug_ex(16, 8, 256, 16, 512, 16, None, 16, 16, 16, 16, 16,
+                                                            2, 2, 16, 1 << 20, None),
+        "host": lib.bitlinear_forward_host(18, 8, 256, 16, 512, 16, None, 18, 16, host_ws, None),
+        "host_async": lib.bitlinear_forward_host_async(18, 8, 256, 16, 512, 16, None, 18, 3, 16, host_ws, None),
+        "noalloc": lib.bitlinear_forward_noalloc(16, 8, 256, 16, 512, 16, None, 16, None),
+        "pack": lib.bitlinear_pack_weights(16, 512, 256, 16, 16, 16, 16, 4096, None),
+        "quant_act": lib.bitlinear_quant_act(16, 4, 256, 16, 16, 16, None),
+        "dequant": lib.bitlinear_dequant_weights(16, 512, 256, 16, 16, None),
+    }
+    wrong = {k: v for k, v in calls.items() if v not in no_device}
+    assert not wrong, wrong
