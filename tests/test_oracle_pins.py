@@ -144,6 +144,26 @@ def test_act_quant_invariants():
         assert np.array_equal(sk, (s_x * np.float32(2.0 ** -k)).astype(np.float32))
 
 
+def test_act_quant_approximates_x():
+    """The int8 activations approximate x (the blog's x ~ x_quant / x_scale):
+    q = round(fl(x * s_x)) with |fl(x * s_x)| <= 127 + ulp, so
+    |x * s_x - q| <= 1/2 + 127 * 2^-24 for every element, in exact
+    arithmetic (float64 holds x * s_x exactly: 8 + 24 significant bits)."""
+    for seed, dist in ((11, "normal"), (12, "student"), (13, "outliers")):
+        if dist == "normal":
+            x = synth.normal_bf16(seed, 1, (9, 512), 3.0)
+        elif dist == "student":
+            x = synth.student_t4_bf16(seed, 1, (9, 512))
+        else:
+            x = synth.normal_with_outliers_bf16(seed, 1, (9, 512))
+        q, s_x, _ = oracle.act_quant(synth.bf16_bits(x))
+        xs = x.double().numpy() * s_x.astype(np.float64)[:, None]
+        err = np.abs(xs - q.astype(np.float64))
+        assert np.all(err <= 0.5 + 127 * 2.0 ** -24), err.max()
+        # and the bound is not vacuous: errors fill most of [0, 1/2]
+        assert err.max() > 0.45
+
+
 # --------------------------------------------------------------------------
 # Step 2: absmean scale, ternarisation, packing
 # --------------------------------------------------------------------------
