@@ -87,7 +87,6 @@ def test_argument_errors_without_gpu(lib):
     assert lib.bitlinear_dequant_weights(16, 512, 256, None, 16, None) == -1
     assert lib.bitlinear_dequant_weights(16, 512, 256, 16, 18, None) == -3
     # grouped forward: group list checks come first
-    import ctypes
     rows = (ctypes.c_int64 * 3)(100, 200, 212)
     bad = (ctypes.c_int64 * 2)(100, 0)
     g = lib.bitlinear_forward_grouped
