@@ -31,7 +31,8 @@ Also on the line:
                 (28672 x 8192), and both CPU oracles' packing beside it
   cpu_baseline  the numpy CPU oracle on a bounded sample of the decode
                 workload, with the plain C++ oracle timed beside it
-                (cpu_baseline.cpp_oracle, one thread)
+                (cpu_baseline.cpp_oracle, one thread), and bounded samples of the
+                prefill, 3B-stack and 100B-FFN workloads (cpu_baseline.per_workload)
   clocks        nvidia-smi samples taken while the workload ran
 
 With --gpus N > 1 (under torchrun) every rank runs the same workload on its
@@ -709,6 +710,60 @@ def timed_oracle(impl, budget_s, max_passes=8):
             "sample": f"{n} passes ({s:.1f} s) of " + od.desc}
 
 
+def oracle_workloads_baseline():
+    """The numpy oracle beyond the decode sweep, one bounded sample each:
+    workload 3 at M=512 (K=3200, N=8640); one layer of workload 4 at M=1
+    (7 projections; the 26-layer figure is extrapolated); the gate
+    projection of workload 5 at M=8 (random valid 2-bit codes, since the
+    forward's cost does not depend on their values; the 39-projection stack
+    figure is extrapolated).  Packing is untimed."""
+    import oracle
+    out = []
+
+    def timed(fn, reps=1, warm=True):
+        if warm:
+            fn()
+        t0 = time.perf_counter()
+        for _ in range(reps):
+            fn()
+        return (time.perf_counter() - t0) / reps
+
+    try:
+        c = [c for c in wl.workload3() if c.M == 512 and c.K == 3200][0]
+        packed, s_w, _ = oracle.pack_weights(c.w().numpy())
+        xb = synth.bf16_bits(c.x())
+        t = timed(lambda: oracle.forward(xb, packed, s_w))
+        out.append({"workload": "prefill M=512, K=3200, N=8640 (workload 3)", "s_per_call": round(t, 3),
+                    "value": round(2 * c.M * c.N * c.K / t / 1e12, 5), "unit": "TOPS"})
+    except Exception as e:
+        out.append({"workload": "prefill M=512", "unavailable": f"{type(e).__name__}: {e}"})
+    try:
+        calls = []
+        for c in wl.workload4(1, layers=[0]):
+            packed, s_w, _ = oracle.pack_weights(c.w().numpy())
+            calls.append((synth.bf16_bits(c.x()), packed, s_w))
+        t = timed(lambda: [oracle.forward(xb, p, s) for xb, p, s in calls])
+        out.append({"workload": "3B-class stack at M=1 (workload 4): one layer of 7 projections timed, "
+                                "26 layers extrapolated", "s_per_layer": round(t, 3),
+                    "value": round(1.0 / (26 * t), 4), "unit": "tokens/s (extrapolated)"})
+    except Exception as e:
+        out.append({"workload": "3B-class stack", "unavailable": f"{type(e).__name__}: {e}"})
+    try:
+        N, K, M = 28672, 8192, 8
+        rng = np.random.default_rng(5)
+        lut = np.array([a | (b << 2) | (c << 4) | (d << 6) for a in range(3) for b in range(3)
+                        for c in range(3) for d in range(3)], dtype=np.uint8)
+        packed = lut[rng.integers(0, 81, (N, K // 4))]
+        xb = synth.bf16_bits(synth.normal_bf16(wl.seed_of(5), 10_000, (M, K)))
+        t = timed(lambda: oracle.forward(xb, packed, np.float32(80.0)), warm=False)
+        out.append({"workload": "100B-class FFN (workload 5): one gate projection at M=8 timed, the "
+                                "13-layer stack (39 projections) extrapolated", "s_per_call": round(t, 3),
+                    "value": round(M / (39 * t), 5), "unit": "tokens/s (extrapolated)"})
+    except Exception as e:
+        out.append({"workload": "100B-class FFN", "unavailable": f"{type(e).__name__}: {e}"})
+    return out
+
+
 def cpp_oracle_baseline(budget_s=5.0):
     """The C++ oracle timed beside the numpy one; never fails the line."""
     try:
@@ -810,6 +865,7 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu:
         cpu = timed_oracle("numpy", 10.0)
         cpu["cpp_oracle"] = cpp_oracle_baseline()
+        cpu["per_workload"] = oracle_workloads_baseline()
         pack["cpu_oracle"] = oracle_pack_baseline()
     try:
         ffn = run_ffn100b(hbm_gbs, bf16_tflops * INT8_OVER_BF16)
