@@ -22,12 +22,15 @@
  *   - the contraction is exact in int32 (|acc| <= 127*K);
  *   - d = s_x*s_w (float32), y32 = float(acc) / d (float32, correctly
  *     rounded), y32 += float(bias) if a bias is given, y = bf16_rne(y32).
+ *     float(acc) is exact while |acc| < 2^24 (always for K <= 132104), and
+ *     rounds to nearest even beyond that.
  *   The flag BITLINEAR_BF16_FAITHFUL switches to the rounding of a bf16
  *   module instead (see its definition below).
  *
  * Conventions for every entry point:
  *   - Shapes: x is [M, K] row-major, W is [N, K] (nn.Linear [out, in]),
- *     y is [M, N].  K must be a positive multiple of 64; M >= 0, N >= 1.
+ *     y is [M, N].  K must be a positive multiple of 64 and at most 2^19;
+ *     0 <= M <= 2^23 and 1 <= N <= 2^23 (BITLINEAR_ERR_SHAPE otherwise).
  *     M == 0 is a no-op that returns BITLINEAR_OK.
  *   - bf16 values travel as their uint16_t bit patterns.
  *   - Every pointer argument is a DEVICE pointer unless its name ends in
