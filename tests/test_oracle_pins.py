@@ -358,6 +358,25 @@ def test_epilogue_exact_rational():
             assert int(y[m, n]) == nearest_bf16_bits(want)
 
 
+def test_epilogue_large_accumulators_round_once():
+    # beyond 2^24 (K > 132104) float(acc) is the float32 nearest to acc (ties
+    # to even), then the division rounds once more
+    acc = np.array([[(1 << 24) + 1, (1 << 24) + 3, -((1 << 25) + 2), (1 << 25) + 6, 127 * (1 << 19)]],
+                   dtype=np.int32)
+    s_x = np.array([3.5], np.float32)
+    s_w = np.float32(21.25)
+    y32, y = oracle.epilogue(acc, s_x, s_w)
+    d = nearest_f32(f32_exact(s_x[0]) * f32_exact(s_w))
+    for n in range(acc.shape[1]):
+        a = nearest_f32(Fraction(int(acc[0, n])))
+        want = nearest_f32(Fraction(float(a)) / Fraction(float(d)))
+        assert y32[0, n] == want, n
+        assert int(y[0, n]) == nearest_bf16_bits(want)
+    # the ties: 2^24 + 1 -> 2^24 (even), 2^24 + 3 -> 2^24 + 4
+    assert nearest_f32(Fraction((1 << 24) + 1)) == np.float32(1 << 24)
+    assert nearest_f32(Fraction((1 << 24) + 3)) == np.float32((1 << 24) + 4)
+
+
 def test_bf16_conversions():
     v = np.array([1.0, -2.5, 3.0e-39, 65504.0, 1.00390625, 1.005859375], np.float32)
     b = oracle.f32_to_bf16_rne(v)
