@@ -5,7 +5,8 @@ activation_norm_quant of the Falcon-Edge blog (section "Falcon-Edge, a
 series of universal models") scales each token by 127 / max(|x|, 1e-5).
 These rows reach the parts of that formula that ordinary activations do
 not:
-- a row scaled by 1e30, so s_x is about 1e-28;
+- a row scaled by 1e30, so s_x is about 1e-28, and a row near the bf16
+  maximum, whose 1 / absmax is subnormal (the bf16-faithful scale);
 - a row of bf16 subnormals, and a row of tiny normal values, both below the
   clamp, so s_x = 127 / 1e-5;
 - a single huge outlier in an otherwise ordinary row, so every other value
@@ -29,8 +30,8 @@ K, N = 256, 160
 
 
 def extreme_rows() -> np.ndarray:
-    """Six extreme rows, float32 values that bf16 holds exactly or rounds."""
-    base = synth.normal_bf16(4200, 1, (6, K)).float().numpy()
+    """Seven extreme rows, float32 values that bf16 holds exactly or rounds."""
+    base = synth.normal_bf16(4200, 1, (7, K)).float().numpy()
     x = base.copy()
     x[0] = base[0] * np.float32(1e30)
     x[1] = base[1] * np.float32(2.0 ** -130)            # bf16 subnormals
@@ -38,6 +39,7 @@ def extreme_rows() -> np.ndarray:
     x[3, 7] = np.float32(1e30)                           # one outlier
     x[4] = np.float32(-0.0)
     x[5] = np.resize(np.array([127.0, 2.5, 3.5, -0.5, 0.5, -2.5, 1.5, -63.5], np.float32), K)
+    x[6] = base[6] / np.abs(base[6]).max() * np.float32(2e38)
     return x
 
 
@@ -45,9 +47,9 @@ def make_x(M: int) -> torch.Tensor:
     rows = extreme_rows()
     ordinary = synth.normal_bf16(4201, M, (M, K)).float().numpy()
     x = ordinary.copy()
-    slots = range(M) if M <= 6 else range(0, M, 3)      # every third row past six
+    slots = range(M) if M <= 7 else range(0, M, 2)      # every second row past seven
     for j, i in enumerate(slots):
-        x[i] = rows[j % 6]
+        x[i] = rows[j % 7]
     return torch.from_numpy(x).to(torch.bfloat16)
 
 
@@ -57,7 +59,7 @@ def oracle_out(x, packed, s_w, bias, faithful):
     return f(xb, packed, np.float32(s_w), None if bias is None else synth.bf16_bits(bias))
 
 
-CASES = [(6, 1), (16, 1), (6, 2), (40, 2)]      # (M, engine): 1 decode, 2 prefill
+CASES = [(7, 1), (16, 1), (7, 2), (40, 2)]      # (M, engine): 1 decode, 2 prefill
 
 
 @pytest.mark.parametrize("faithful", [False, True], ids=["float32", "bf16_faithful"])

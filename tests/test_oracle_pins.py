@@ -537,6 +537,34 @@ def test_bf16_mode_matches_pytorch_bf16_execution(seed):
     assert np.array_equal(out["y"], synth.bf16_bits(y_t))
 
 
+def test_bf16_mode_matches_pytorch_on_extreme_rows():
+    # the listings on a bf16 module, run by PyTorch, for rows at the edges of
+    # bf16: a 1e30 row, a row near the bf16 maximum (1 / absmax is subnormal),
+    # a subnormal row and a tiny row (both below the clamp), one huge
+    # outlier, -0.0, .5 ties
+    K, N = 128, 48
+    base = synth.normal_bf16(4300, 1, (7, K)).float()
+    x = base.clone()
+    x[0] = base[0] * 1e30
+    x[1] = base[1] * 2.0 ** -130
+    x[2] = base[2] * 1e-7
+    x[3, 5] = 1e30
+    x[4] = -0.0
+    x[5] = torch.tensor([127.0, 2.5, 3.5, -0.5, 0.5, -2.5, 1.5, -63.5] * (K // 8))
+    x[6] = base[6] / base[6].abs().max() * 2e38
+    x = x.to(torch.bfloat16)
+    assert 0 < 1.0 / float(x[6].float().abs().max()) < 1.1754944e-38      # a subnormal reciprocal
+    w = synth.normal_f32(4300, 2, (N, K), 0.02).numpy()
+    packed, s_w, _ = oracle.pack_weights(w)
+    u = oracle.unpack(packed)
+    bias = synth.normal_bf16(4300, 3, (N,), 0.5)
+    xq_t, scale_t, y_t = _listing_on_bf16_module(x, u.astype(np.float32), s_w, bias)
+    out = oracle.forward_bf16(synth.bf16_bits(x), packed, s_w, synth.bf16_bits(bias))
+    assert np.array_equal(out["q"], xq_t.float().numpy().astype(np.int8))
+    assert np.array_equal(out["s_x"], scale_t.float().numpy()[:, 0])
+    assert np.array_equal(out["y"], synth.bf16_bits(y_t))
+
+
 def test_bf16_mode_differs_from_float32_mode_only_by_rounding():
     # the two modes read the same pages; they differ only in where rounding
     # happens, so the outputs agree to within a few bf16 ulps
