@@ -142,6 +142,17 @@ def test_deterministic_repeat():
         assert torch.equal(o[2].view(torch.int16), outs[0][2].view(torch.int16))
 
 
+def test_deterministic_repeat_prefill():
+    # the persistent tcgen05 GEMM has a static tile schedule and exact int32
+    # sums: three runs give the same bytes (races would show up here)
+    c = [c for c in _W3 if c.M == 2048 and c.K == 3200][0]
+    x, w = c.x().cuda(), c.w().cuda()
+    packed, s_w, _ = bl.bitlinear_pack_weights(w)
+    ys = [bl.bitlinear_forward(x, packed, s_w).cpu() for _ in range(3)]
+    for y in ys[1:]:
+        assert torch.equal(y.view(torch.int16), ys[0].view(torch.int16))
+
+
 def test_quant_act_standalone():
     x = synth.student_t4_bf16(80, 1, (300, 3200))
     xq, s_x, rs = bl.bitlinear_quant_act(x.cuda())
