@@ -51,6 +51,8 @@ _SIGS = {
                                               _c_sz, _c_p]),
     "bitlinear_check_status": (ctypes.c_int, [_c_p, _c_sz, _c_p]),
     "bitlinear_forward_noalloc": (ctypes.c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_i64, _c_p, _c_p, _c_p, _c_p]),
+    "bitlinear_noalloc_check_status": (ctypes.c_int, [_c_p]),
+    "bitlinear_test_force_timeout": (ctypes.c_int, [ctypes.c_int]),
 }
 
 _lib = None
@@ -104,6 +106,65 @@ def _bits(t: torch.Tensor) -> torch.Tensor:
     return t.contiguous()
 
 
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype, shape=None, device=None, min_numel: int = 0) -> None:
+    """Host-side check of one tensor argument: dtype, exact shape, device and
+    contiguity, so that a wrong argument raises here instead of making a
+    kernel read or write out of bounds."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.numel() < min_numel:
+        raise ValueError(f"{name} needs at least {min_numel} elements, got {t.numel()}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _check_forward(x: torch.Tensor, packed: torch.Tensor, w_scale: torch.Tensor, bias, out, ws,
+                   n_scales: int = 1, x_on_host: bool = False) -> tuple:
+    """The arguments shared by the forward entry points, checked on the host
+    before anything is enqueued: dtypes (TypeError), then shapes and layout
+    (BitLinearError BITLINEAR_ERR_SHAPE for K, ValueError otherwise), then
+    devices (ValueError).  Returns (M, N, K)."""
+    lib()                                        # a missing library is reported first
+    if x.dim() != 2:
+        raise ValueError(f"x must be 2-D [M, K], got {tuple(x.shape)}")
+    M, K = x.shape
+    if K % 64 != 0 or K <= 0:
+        raise BitLinearError(-2, f"K = {K} must be a positive multiple of 64")
+    if packed.dim() != 2:
+        raise ValueError(f"packed must be 2-D [N, K/4], got {tuple(packed.shape)}")
+    N = packed.shape[0]
+    _need(packed, "packed", torch.uint8, (N, K // 4))
+    _need(w_scale, "w_scale", torch.float32, None, min_numel=n_scales)
+    if bias is not None:
+        _need(bias, "bias", torch.bfloat16, (N,))
+    if out is not None:
+        _need(out, "y_host" if x_on_host else "out", torch.bfloat16, (M, N))
+    if ws is not None:
+        _need(ws, "ws", torch.uint8)
+    dev = packed.device
+    if dev.type != "cuda":
+        raise ValueError(f"packed must be on a CUDA device, got {dev}")
+    if x_on_host:
+        if x.device.type != "cpu":
+            raise ValueError("x_host must be a host (CPU) tensor")
+        if out is not None and out.device.type != "cpu":
+            raise ValueError("y_host must be a host (CPU) tensor")
+    else:
+        for t, name in ((x, "x"), (out, "out")):
+            if t is not None and t.device != dev:
+                raise ValueError(f"{name} is on {t.device}, packed on {dev}")
+    for t, name in ((w_scale, "w_scale"), (bias, "bias"), (ws, "ws")):
+        if t is not None and t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, packed on {dev}")
+    return M, N, K
+
+
 def packed_bytes(N: int, K: int) -> int:
     return int(lib().bitlinear_packed_bytes(N, K))
 
@@ -133,7 +194,11 @@ def bitlinear_pack_weights(w: torch.Tensor, ws: Optional[torch.Tensor] = None):
     w = w.contiguous()
     if w.dtype != torch.float32 or w.dim() != 2:
         raise TypeError("w must be a float32 [N, K] tensor")
+    if w.device.type != "cuda":
+        raise ValueError("w must be on a CUDA device")
     N, K = w.shape
+    if ws is not None:
+        _need(ws, "ws", torch.uint8, None, w.device, min_numel=pack_workspace_bytes(N, K))
     packed = torch.empty((N, K // 4), dtype=torch.uint8, device=w.device)
     w_scale = torch.empty(1, dtype=torch.float32, device=w.device)
     w_mean = torch.empty(1, dtype=torch.float32, device=w.device)
@@ -147,6 +212,8 @@ def bitlinear_pack_weights(w: torch.Tensor, ws: Optional[torch.Tensor] = None):
 def bitlinear_quant_act(x: torch.Tensor):
     """activation_norm_quant.  x: bf16 [M, K].  Returns (xq int8, s_x f32, rowsum i32)."""
     x = _bits(x)
+    if x.dim() != 2 or x.device.type != "cuda":
+        raise ValueError("x must be a 2-D CUDA tensor [M, K]")
     M, K = x.shape
     xq = torch.empty((M, K), dtype=torch.int8, device=x.device)
     s_x = torch.empty(M, dtype=torch.float32, device=x.device)
@@ -158,7 +225,14 @@ def bitlinear_quant_act(x: torch.Tensor):
 
 def bitlinear_dequant_weights(packed: torch.Tensor, w_scale: torch.Tensor) -> torch.Tensor:
     """bf16 export of packed weights: w [N, K] bf16 = u / s_w (zeros +0)."""
+    lib()
+    if packed.dim() != 2:
+        raise ValueError("packed must be 2-D [N, K/4]")
+    if packed.device.type != "cuda":
+        raise ValueError("packed must be on a CUDA device")
     N, K = packed.shape[0], packed.shape[1] * 4
+    _need(packed, "packed", torch.uint8, (N, K // 4))
+    _need(w_scale, "w_scale", torch.float32, None, packed.device, min_numel=1)
     out = torch.empty((N, K), dtype=torch.bfloat16, device=packed.device)
     _check(lib().bitlinear_dequant_weights(_ptr(packed), N, K, _ptr(w_scale), _ptr(out), _stream(packed.device)),
            "bitlinear_dequant_weights")
@@ -175,8 +249,7 @@ def bitlinear_forward(x: torch.Tensor, packed: torch.Tensor, w_scale: torch.Tens
     """BitLinear.forward: y bf16 [M, N] from x bf16 [M, K] and packed weights.
     flags=WEIGHTS_RESIDENT calls bitlinear_forward_ex (see the C header)."""
     x = _bits(x)
-    M, K = x.shape
-    N = packed.shape[0]
+    M, N, K = _check_forward(x, packed, w_scale, bias, out, ws)
     y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     if ws is None:
         ws = workspace(M, N, K, x.device)
@@ -201,8 +274,9 @@ def bitlinear_forward_grouped(x: torch.Tensor, packed: torch.Tensor, group_rows,
     group_rows their row counts, w_scales [G] f32.  Returns y bf16 [M, N], layer g in
     its own column block."""
     x = _bits(x)
-    M, K = x.shape
-    N = packed.shape[0]
+    M, N, K = _check_forward(x, packed, w_scales, bias, out, ws, n_scales=len(group_rows))
+    if sum(int(r) for r in group_rows) != N:
+        raise ValueError(f"group_rows sum to {sum(int(r) for r in group_rows)}, packed has {N} rows")
     rows = (ctypes.c_int64 * len(group_rows))(*[int(r) for r in group_rows])
     y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     if ws is None:
@@ -217,8 +291,17 @@ def bitlinear_forward_q8(xq: torch.Tensor, s_x: torch.Tensor, rowsum: torch.Tens
                          w_scale: torch.Tensor, bias: Optional[torch.Tensor] = None,
                          ws: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Contraction + epilogue on activations from bitlinear_quant_act."""
+    if xq.dim() != 2:
+        raise ValueError("xq must be 2-D [M, K]")
     M, K = xq.shape
+    _need(xq, "xq", torch.int8, (M, K))
+    _need(s_x, "s_x", torch.float32, (M,))
+    _need(rowsum, "rowsum", torch.int32, (M,))
     N = packed.shape[0]
+    _check_forward(xq, packed, w_scale, bias, out, ws)
+    for t, name in ((s_x, "s_x"), (rowsum, "rowsum")):
+        if t.device != packed.device:
+            raise ValueError(f"{name} is on {t.device}, packed on {packed.device}")
     y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=xq.device)
     if ws is None:
         ws = torch.zeros(256, dtype=torch.uint8, device=xq.device)
@@ -235,8 +318,7 @@ def bitlinear_forward_debug(x: torch.Tensor, packed: torch.Tensor, w_scale: torc
     """Forward with intermediates: y, xq, s_x, acc (int32), y32 (float32).
     flags=BF16_FAITHFUL calls bitlinear_forward_debug_ex."""
     x = _bits(x)
-    M, K = x.shape
-    N = packed.shape[0]
+    M, N, K = _check_forward(x, packed, w_scale, bias, None, ws)
     dev = x.device
     y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     xq = torch.empty((M, K), dtype=torch.int8, device=dev)
@@ -262,8 +344,7 @@ def bitlinear_forward_host(x_host: torch.Tensor, packed: torch.Tensor, w_scale: 
                            ws: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Forward from host activations to a host output (synchronous)."""
     x_host = _bits(x_host)
-    M, K = x_host.shape
-    N = packed.shape[0]
+    M, N, K = _check_forward(x_host, packed, w_scale, bias, y_host, ws, x_on_host=True)
     dev = packed.device
     if y_host is None:
         y_host = torch.empty((M, N), dtype=torch.bfloat16, pin_memory=True)
@@ -282,8 +363,7 @@ def bitlinear_forward_host_async(x_host: torch.Tensor, packed: torch.Tensor, w_s
     """Stream-ordered host-to-host forward: enqueues the copies and kernels and
     returns; y_host is valid once the current stream is synchronised."""
     x_host = _bits(x_host)
-    M, K = x_host.shape
-    N = packed.shape[0]
+    M, N, K = _check_forward(x_host, packed, w_scale, bias, y_host, ws, x_on_host=True)
     dev = packed.device
     if y_host is None:
         y_host = torch.empty((M, N), dtype=torch.bfloat16, pin_memory=True)
@@ -301,8 +381,7 @@ def bitlinear_forward_noalloc(x: torch.Tensor, packed: torch.Tensor, w_scale: to
     """bitlinear_forward with the library's fixed device scratch instead of a
     workspace (for callers that cannot allocate; see the C header)."""
     x = _bits(x)
-    M, K = x.shape
-    N = packed.shape[0]
+    M, N, K = _check_forward(x, packed, w_scale, bias, out, None)
     y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     b = None if bias is None else _bits(bias)
     _check(lib().bitlinear_forward_noalloc(_ptr(x), M, K, _ptr(packed), N, _ptr(w_scale), _ptr(b), _ptr(y),
@@ -313,3 +392,16 @@ def bitlinear_forward_noalloc(x: torch.Tensor, packed: torch.Tensor, w_scale: to
 def bitlinear_check_status(ws: torch.Tensor) -> int:
     """Status of the most recent call that used workspace ws (synchronises)."""
     return int(lib().bitlinear_check_status(_ptr(ws), ws.numel(), _stream(ws.device)))
+
+
+def bitlinear_noalloc_check_status(device=None) -> int:
+    """Status of the noalloc calls on the current device since the last
+    reset (synchronises the current stream)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    return int(lib().bitlinear_noalloc_check_status(_stream(dev)))
+
+
+def bitlinear_test_force_timeout(on: bool) -> bool:
+    """Test hook: while on, every forward's kernels take one wait that runs out
+    (1 ms) and report BITLINEAR_ERR_TIMEOUT.  Returns the previous setting."""
+    return bool(lib().bitlinear_test_force_timeout(1 if on else 0))
