@@ -4,6 +4,8 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "../../include/bitlinear.h"
 #include "kernels.h"
 
@@ -58,6 +60,21 @@ int check_device(int* sms) {
   if (sms) *sms = d.sms;
   return d.checked == 1 ? BITLINEAR_OK : BITLINEAR_ERR_DEVICE;
 }
+
+}  // namespace
+
+// The current device is a B200 (sm_100): BITLINEAR_OK, BITLINEAR_ERR_DEVICE
+// or BITLINEAR_ERR_CUDA.  Used by entry points defined in other files.
+int bitlinear::current_device_status() { return check_device(nullptr); }
+
+// Forced-timeout test hook (bitlinear_test_force_timeout): while it is on,
+// every launch gets the short main-loop wait limit and one wait on a barrier
+// that nothing signals.
+static std::atomic<int> g_force_timeout{0};
+uint64_t bitlinear::launch_wait_ns() { return g_force_timeout.load() ? kTestWaitLimitNs : kWaitLimitNs; }
+int bitlinear::launch_stall() { return g_force_timeout.load() ? 1 : 0; }
+
+namespace {
 
 int check_shape(int64_t M, int64_t N, int64_t K) {
   if (M < 0 || M > kMaxMN || N < 1 || N > kMaxMN || K < 64 || K > kMaxK || (K % 64) != 0)
@@ -126,6 +143,8 @@ int forward_impl_g(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packe
     d.faithful = faithful ? 1 : 0;
     d.ngroups = grp.n;
     for (int g = 0; g < kMaxGroups; ++g) d.group_end[g] = grp.end[g];
+    d.wait_ns = launch_wait_ns();
+    d.stall = launch_stall();
     return status_of(launch_decode(d, sms, stream));
   }
   float* s_x = reinterpret_cast<float*>(base + L.off_sx);
@@ -151,6 +170,8 @@ int forward_impl_g(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packe
   a.faithful = faithful;
   a.ngroups = grp.n;
   for (int g = 0; g < kMaxGroups; ++g) a.group_end[g] = grp.end[g];
+  a.wait_ns = launch_wait_ns();
+  a.stall = launch_stall();
   e = launch_gemm_prefill(a, sms, stream);
   if (e != cudaSuccess) return BITLINEAR_ERR_CUDA;
   if (xq_out) e = cudaMemcpyAsync(xq_out, xq, size_t(M) * size_t(K), cudaMemcpyDeviceToDevice, stream);
@@ -223,7 +244,7 @@ size_t bitlinear_host_workspace_bytes(int64_t M, int64_t N, int64_t K) {
 
 int bitlinear_pack_weights(const float* w, int64_t N, int64_t K, uint8_t* packed, float* w_scale,
                            float* w_mean, void* ws, size_t ws_bytes, void* stream) {
-  if (N < 1 || K < 64 || (K % 64) != 0 || N > kMaxMN || K > kMaxK || N * K >= (int64_t(1) << 40))
+  if (N < 1 || K < 64 || (K % 64) != 0 || N > kMaxMN || K > kMaxK || N * K >= (int64_t(1) << 39))
     return BITLINEAR_ERR_SHAPE;
   if (!w || !packed || !w_scale) return BITLINEAR_ERR_NULL;
   if (misaligned(w) || misaligned(packed) || misaligned(w_scale) || misaligned(w_mean))
@@ -328,6 +349,8 @@ int bitlinear_forward_q8(const int8_t* xq, const float* x_scale, const int32_t* 
   a.faithful = false;
   a.ngroups = 1;
   a.group_end[0] = int(N);
+  a.wait_ns = launch_wait_ns();
+  a.stall = launch_stall();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (M > 16) return status_of(launch_gemm_prefill(a, sms, s));
   // the previous operation on the stream is unknown: read the weights only
@@ -352,6 +375,8 @@ int bitlinear_forward_q8(const int8_t* xq, const float* x_scale, const int32_t* 
   d.faithful = 0;
   d.ngroups = 1;
   d.group_end[0] = int(N);
+  d.wait_ns = a.wait_ns;
+  d.stall = a.stall;
   return status_of(launch_decode(d, sms, s));
 }
 
@@ -432,6 +457,10 @@ int bitlinear_forward_host_async(const uint16_t* x_host, int64_t M, int64_t K, c
   if (flags & ~static_cast<unsigned>(BITLINEAR_WEIGHTS_RESIDENT | BITLINEAR_BF16_FAITHFUL)) return BITLINEAR_ERR_SHAPE;
   return forward_host_impl(x_host, M, K, packed_w, N, w_scale, bias, y_host, flags, ws, ws_bytes,
                            static_cast<cudaStream_t>(stream), false);
+}
+
+int bitlinear_test_force_timeout(int on) {
+  return g_force_timeout.exchange(on ? 1 : 0);
 }
 
 int bitlinear_check_status(const void* ws, size_t ws_bytes, void* stream) {

@@ -9,6 +9,9 @@
 
 namespace bitlinear {
 
+// ---- device check (api.cu): BITLINEAR_OK when the current GPU is sm_100 ----
+int current_device_status();
+
 // ---- TMA tensor maps (tensor_map.cu) ---------------------------------------
 bool encode_2d_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
                   uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle);
@@ -31,8 +34,12 @@ cudaError_t launch_act_quant(const uint16_t* x, int M, int K, int8_t* xq, float*
 struct PackWorkspace {
   uint32_t* status;   // 1 word
   float* mean;        // 1 float
-  uint64_t* bins;     // 256 exponent bins
+  uint64_t* bins;     // kAbsmeanBins exponent bins
 };
+// Exponent bins of the exact absmean sum: bin e holds a sum of 24-bit
+// significands of weight 2^(max(e,1) - 150); the window sums' chunks reach
+// exponents up to 254 - 36 + 72 = 290.
+constexpr int kAbsmeanBins = 320;
 constexpr size_t kPackWsBytes = 4096;
 PackWorkspace pack_workspace(void* ws);
 cudaError_t launch_pack(const float* w, int64_t N, int64_t K, uint8_t* packed, float* w_scale,
@@ -59,6 +66,8 @@ struct ForwardArgs {
   int group_end[kMaxGroups];
   bool pdl;               // launched as a programmatic dependent of the act-quant kernel
   bool faithful;          // bf16-module epilogue: every step rounded to bf16
+  uint64_t wait_ns;       // limit of the main-loop waits (drains keep kWaitLimitNs)
+  int stall;              // test hook: first wait on a barrier nothing signals
 };
 
 // ---- bf16 export of packed weights (dequant.cu) ----------------------------
@@ -99,7 +108,17 @@ struct DecodeArgs {
   int faithful;           // bf16-module rounding of the quantisation and the epilogue
   int ring, units_max, kc, tail;  // set by launch_decode
   int weights_early;      // the packed weights, w_scale and bias may be read before the dependency wait
+  uint64_t wait_ns;       // limit of the main-loop waits (drains keep kWaitLimitNs)
+  int stall;              // test hook: first wait on a barrier nothing signals
 };
+
+// Main-loop wait limits: the default, and the short one used while the
+// forced-timeout test hook is on.
+constexpr uint64_t kTestWaitLimitNs = 1000ull * 1000ull;   // 1 ms
+// Wait limit and stall flag for the next launch (the forced-timeout test hook
+// of api.cu).
+uint64_t launch_wait_ns();
+int launch_stall();
 struct DecodePlan {
   int grid, units_max, ring, kc, tail;
   size_t slot_bytes, smem;

@@ -54,9 +54,24 @@ extern "C" int bitlinear_forward_noalloc(const uint16_t* x, int64_t M, int64_t K
   const size_t need = bitlinear_workspace_bytes(M, N, K);
   if (need == 0) return BITLINEAR_ERR_SHAPE;
   if (need > BITLINEAR_NOALLOC_SCRATCH_BYTES) return BITLINEAR_ERR_WORKSPACE;   // beyond the fixed scratch
+  // the device check comes first: on a GPU the library has no code for, the
+  // symbol lookup below would fail with a less telling error
+  int st = bitlinear::current_device_status();
+  if (st != BITLINEAR_OK) return st;
   void* scratch = nullptr;
-  const int st = scratch_for_current_device(&scratch);
+  st = scratch_for_current_device(&scratch);
   if (st != BITLINEAR_OK) return st;
   return bitlinear_forward(x, M, K, packed_w, N, w_scale, bias, y, scratch, BITLINEAR_NOALLOC_SCRATCH_BYTES,
                            stream);
+}
+
+// The status word lives at the start of the scratch array, as in any
+// workspace; this reads and clears it for the current device.
+extern "C" int bitlinear_noalloc_check_status(void* stream) {
+  int st = bitlinear::current_device_status();
+  if (st != BITLINEAR_OK) return st;
+  void* scratch = nullptr;
+  st = scratch_for_current_device(&scratch);
+  if (st != BITLINEAR_OK) return st;
+  return bitlinear_check_status(scratch, BITLINEAR_NOALLOC_SCRATCH_BYTES, stream);
 }

@@ -110,7 +110,8 @@ size_t bitlinear_host_workspace_bytes(int64_t M, int64_t N, int64_t K);
  *   w_mean   [1] float32 out, the exactly rounded mean |w|; may be NULL
  *   ws       workspace of bitlinear_pack_workspace_bytes bytes; its
  *            contents on entry do not matter
- * N * K must be below 2^40. */
+ * N * K must be below 2^39 (the exact sum's 64-bit exponent bins stay
+ * below 2^64; no GPU holds a float32 tensor of that size). */
 int bitlinear_pack_weights(const float* w, int64_t N, int64_t K, uint8_t* packed,
                            float* w_scale, float* w_mean, void* ws, size_t ws_bytes,
                            void* stream);
@@ -259,11 +260,23 @@ int bitlinear_forward_host_async(const uint16_t* x_host, int64_t M, int64_t K, c
  *     other.  Serialise them, e.g. on one stream.
  *   - The first call on a device looks up the array's device address on that
  *     device (make the device current first); make that first call before
- *     any stream capture.
+ *     any stream capture.  The address is cached for the device's primary
+ *     context: do not use this entry point after a cudaDeviceReset in the
+ *     same process.
+ *   - A device-side wait that gives up is recorded in the scratch array's
+ *     status word; read it with bitlinear_noalloc_check_status.
  *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call. */
 #define BITLINEAR_NOALLOC_SCRATCH_BYTES (16u << 20)
 int bitlinear_forward_noalloc(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed_w, int64_t N,
                               const float* w_scale, const uint16_t* bias, uint16_t* y, void* stream);
+
+/* bitlinear_check_status for the fixed scratch array of
+ * bitlinear_forward_noalloc on the current device: reads and clears its
+ * status word (synchronises `stream`).  Returns BITLINEAR_OK, or
+ * BITLINEAR_ERR_TIMEOUT if a device-side bounded wait of a noalloc call gave
+ * up since the last reset (each noalloc call resets it when it starts).  The
+ * paper has no counterpart to this entry point either. */
+int bitlinear_noalloc_check_status(void* stream);
 
 /* Reads and clears the status word of a workspace (synchronises
  * `stream`).  bitlinear_pack_weights, bitlinear_forward, _debug and _host
@@ -271,6 +284,19 @@ int bitlinear_forward_noalloc(const uint16_t* x, int64_t M, int64_t K, const uin
  * BITLINEAR_OK, or BITLINEAR_ERR_TIMEOUT if a device-side bounded wait gave
  * up since the last reset.  `ws_bytes` is the size the calls were given. */
 int bitlinear_check_status(const void* ws, size_t ws_bytes, void* stream);
+
+/* Test hook for the failure path of the device-side waits.  While it is on
+ * (on != 0), every forward launched by this process -- bitlinear_forward and
+ * its variants, both engines -- makes one wait on a barrier that nothing
+ * signals, with a 1 ms limit instead of the usual 1 s for its main-loop
+ * waits.  That wait gives up, the kernel stops its main loop, lets every copy
+ * and tensor-core operation already started finish (those drains keep the
+ * 1 s limit), sets BITLINEAR_ERR_TIMEOUT in the status word and exits; y is
+ * then left unspecified.  No fault, trap or hang is involved: the context
+ * stays usable and the next forward after switching the hook off is normal.
+ * Process-wide and not meant for production use.  Returns the previous
+ * setting (0 or 1). */
+int bitlinear_test_force_timeout(int on);
 
 #ifdef __cplusplus
 }

@@ -114,7 +114,8 @@ def test_more_argument_errors_without_gpu(lib):
     assert _fwd(lib, N=(1 << 23) + 1) == -2
     assert _fwd(lib, K=(1 << 19) + 64) == -2
     assert _fwd(lib, M=(1 << 23) + 1) == -2
-    assert lib.bitlinear_pack_weights(16, 1 << 23, 1 << 19, 16, 16, None, 16, 4096, None) == -2   # N*K >= 2^40
+    assert lib.bitlinear_pack_weights(16, 1 << 23, 1 << 19, 16, 16, None, 16, 4096, None) == -2   # N*K >= 2^39
+    assert lib.bitlinear_pack_weights(16, 1 << 20, 1 << 19, 16, 16, None, 16, 4096, None) == -2   # N*K = 2^39
     # misaligned scale, workspace and output
     assert _fwd(lib, s=20) == -3
     assert _fwd(lib, ws=24) == -3
@@ -175,6 +176,7 @@ def test_valid_arguments_pass_every_host_check(lib):
         "host": lib.bitlinear_forward_host(18, 8, 256, 16, 512, 16, None, 18, 16, host_ws, None),
         "host_async": lib.bitlinear_forward_host_async(18, 8, 256, 16, 512, 16, None, 18, 3, 16, host_ws, None),
         "noalloc": lib.bitlinear_forward_noalloc(16, 8, 256, 16, 512, 16, None, 16, None),
+        "noalloc status": lib.bitlinear_noalloc_check_status(None),
         "pack": lib.bitlinear_pack_weights(16, 512, 256, 16, 16, 16, 16, 4096, None),
         "quant_act": lib.bitlinear_quant_act(16, 4, 256, 16, 16, 16, None),
         "dequant": lib.bitlinear_dequant_weights(16, 512, 256, 16, 16, None),

@@ -39,10 +39,15 @@ def test_noalloc_matches_forward_twice(M, N, K, with_bias):
         x = synth.normal_bf16(91 + call, M * K, (M, K)).cuda()
         want = bl.bitlinear_forward(x, packed, s_w, bias)
         y = torch.full((M, N), -1.0, dtype=torch.bfloat16, device="cuda")
+        torch.cuda.synchronize()
+        free_before = torch.cuda.mem_get_info()[0]
         assert _noalloc(x, packed, s_w, bias, y) == 0
         torch.cuda.synchronize()
+        if call == 1:                          # its kernels are loaded by now: no device memory taken
+            assert torch.cuda.mem_get_info()[0] == free_before
         # same tolerance as the other parity tests: bit-exact bf16 output
         assert torch.equal(y.view(torch.int16), want.view(torch.int16)), f"call {call} differs"
+        assert bl.bitlinear_noalloc_check_status() == 0
 
 
 def test_noalloc_rejects_sizes_beyond_scratch():
@@ -55,3 +60,26 @@ def test_noalloc_rejects_sizes_beyond_scratch():
                                               ctypes.c_void_p(packed.data_ptr()), N,
                                               ctypes.c_void_p(s_w.data_ptr()), None,
                                               ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(st)) == -4
+
+
+@pytest.mark.parametrize("M", [4, 40])
+def test_noalloc_reports_a_timeout(M):
+    """A device-side wait that gives up inside a noalloc call is visible to
+    the caller through bitlinear_noalloc_check_status (the status word sits in
+    the fixed scratch, which the caller cannot name); the next call is normal."""
+    N, K = 512, 1024
+    w = synth.normal_f32(95, N + K, (N, K), 0.02).cuda()
+    packed, s_w, _ = bl.bitlinear_pack_weights(w)
+    x = synth.normal_bf16(96, M * K, (M, K)).cuda()
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    bl.bitlinear_test_force_timeout(True)
+    try:
+        assert _noalloc(x, packed, s_w, None, y) == 0
+        assert bl.bitlinear_noalloc_check_status() == -6
+    finally:
+        bl.bitlinear_test_force_timeout(False)
+    assert _noalloc(x, packed, s_w, None, y) == 0
+    assert bl.bitlinear_noalloc_check_status() == 0
+    want = bl.bitlinear_forward(x, packed, s_w)
+    torch.cuda.synchronize()
+    assert torch.equal(y.view(torch.int16), want.view(torch.int16))
