@@ -53,6 +53,14 @@ _SIGS = {
     "bitlinear_forward_noalloc": (ctypes.c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_i64, _c_p, _c_p, _c_p, _c_p]),
     "bitlinear_noalloc_check_status": (ctypes.c_int, [_c_p]),
     "bitlinear_test_force_timeout": (ctypes.c_int, [ctypes.c_int]),
+    "bitlinear_absmean_bins": (ctypes.c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_p]),
+    "bitlinear_pack_weights_from_bins": (ctypes.c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_i64, _c_p, _c_p, _c_p, _c_p,
+                                                        _c_sz, _c_p]),
+    "bitlinear_act_absmax": (ctypes.c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_p]),
+    "bitlinear_forward_partial": (ctypes.c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_p, _c_i64, _c_p, ctypes.c_uint,
+                                                 _c_p, _c_sz, _c_p]),
+    "bitlinear_epilogue_sum": (ctypes.c_int, [_c_p, ctypes.c_int, _c_i64, _c_i64, _c_p, _c_p, _c_p, _c_p, _c_p,
+                                              ctypes.c_uint, _c_p]),
 }
 
 _lib = None
@@ -405,3 +413,102 @@ def bitlinear_test_force_timeout(on: bool) -> bool:
     """Test hook: while on, every forward's kernels take one wait that runs out
     (1 ms) and report BITLINEAR_ERR_TIMEOUT.  Returns the previous setting."""
     return bool(lib().bitlinear_test_force_timeout(1 if on else 0))
+
+
+# ---- tensor-parallel K-split pieces (see the C header) ----------------------
+
+ABSMEAN_BINS = 320
+MAX_PARTS = 8
+
+
+def bitlinear_absmean_bins(w: torch.Tensor) -> torch.Tensor:
+    """Exact exponent bins of sum |w| over this shard: uint64 [320] as int64
+    (two's complement); the bins of several shards add."""
+    lib()
+    if w.dim() != 2:
+        raise ValueError("w must be 2-D [N, K]")
+    _need(w, "w", torch.float32)
+    if w.device.type != "cuda":
+        raise ValueError("w must be on a CUDA device")
+    N, K = w.shape
+    bins = torch.empty(ABSMEAN_BINS, dtype=torch.int64, device=w.device)
+    _check(lib().bitlinear_absmean_bins(_ptr(w), N, K, _ptr(bins), _stream(w.device)), "bitlinear_absmean_bins")
+    return bins
+
+
+def bitlinear_pack_weights_from_bins(w: torch.Tensor, bins: torch.Tensor, n_total: int,
+                                     ws: Optional[torch.Tensor] = None):
+    """Pack one shard with s_w from the summed bins of all shards.
+    Returns (packed, w_scale, w_mean) as bitlinear_pack_weights does."""
+    lib()
+    if w.dim() != 2:
+        raise ValueError("w must be 2-D [N, K]")
+    _need(w, "w", torch.float32)
+    _need(bins, "bins", torch.int64, (ABSMEAN_BINS,), w.device)
+    if w.device.type != "cuda":
+        raise ValueError("w must be on a CUDA device")
+    N, K = w.shape
+    packed = torch.empty((N, K // 4), dtype=torch.uint8, device=w.device)
+    w_scale = torch.empty(1, dtype=torch.float32, device=w.device)
+    w_mean = torch.empty(1, dtype=torch.float32, device=w.device)
+    if ws is None:
+        ws = torch.empty(pack_workspace_bytes(N, K), dtype=torch.uint8, device=w.device)
+    _check(lib().bitlinear_pack_weights_from_bins(_ptr(w), N, K, _ptr(bins), int(n_total), _ptr(packed),
+                                                  _ptr(w_scale), _ptr(w_mean), _ptr(ws), ws.numel(),
+                                                  _stream(w.device)), "bitlinear_pack_weights_from_bins")
+    return packed, w_scale, w_mean
+
+
+def bitlinear_act_absmax(x: torch.Tensor) -> torch.Tensor:
+    """Each token's absmax over this K-shard of x, float32 [M]."""
+    x = _bits(x)
+    if x.dim() != 2 or x.device.type != "cuda":
+        raise ValueError("x must be a 2-D CUDA tensor [M, K]")
+    M, K = x.shape
+    out = torch.empty(M, dtype=torch.float32, device=x.device)
+    _check(lib().bitlinear_act_absmax(_ptr(x), M, K, _ptr(out), _stream(x.device)), "bitlinear_act_absmax")
+    return out
+
+
+def bitlinear_forward_partial(x: torch.Tensor, absmax: torch.Tensor, packed: torch.Tensor,
+                              ws: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                              flags: int = 0) -> torch.Tensor:
+    """int32 [M, N] partial sums of one K-shard, quantised with the whole
+    row's absmax."""
+    x = _bits(x)
+    M, N, K = _check_forward(x, packed, absmax, None, None, ws)
+    _need(absmax, "absmax", torch.float32, (M,), packed.device)
+    acc = out if out is not None else torch.empty((M, N), dtype=torch.int32, device=x.device)
+    _need(acc, "out", torch.int32, (M, N), packed.device)
+    if ws is None:
+        ws = workspace(M, N, K, x.device)
+    _check(lib().bitlinear_forward_partial(_ptr(x), M, K, _ptr(absmax), _ptr(packed), N, _ptr(acc), flags,
+                                           _ptr(ws), ws.numel(), _stream(x.device)), "bitlinear_forward_partial")
+    return acc
+
+
+def bitlinear_epilogue_sum(partials, absmax: torch.Tensor, w_scale: torch.Tensor,
+                           bias: Optional[torch.Tensor] = None, flags: int = 0, acc_out: Optional[torch.Tensor] = None,
+                           out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """y bf16 [M, N] from int32 partial sums (a tensor or a list of them, all
+    [M, N]), the tokens' absmax over the whole K, s_w and the bias."""
+    lib()
+    parts = [partials] if isinstance(partials, torch.Tensor) else list(partials)
+    if not 1 <= len(parts) <= MAX_PARTS:
+        raise ValueError(f"1 .. {MAX_PARTS} partial sums")
+    M, N = parts[0].shape
+    dev = parts[0].device
+    for p in parts:
+        _need(p, "partial", torch.int32, (M, N))
+    _need(absmax, "absmax", torch.float32, (M,), dev)
+    _need(w_scale, "w_scale", torch.float32, None, dev, min_numel=1)
+    if bias is not None:
+        _need(bias, "bias", torch.bfloat16, (N,), dev)
+    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    _need(y, "out", torch.bfloat16, (M, N), dev)
+    if acc_out is not None:
+        _need(acc_out, "acc_out", torch.int32, (M, N), dev)
+    arr = (ctypes.c_void_p * len(parts))(*[p.data_ptr() for p in parts])
+    _check(lib().bitlinear_epilogue_sum(arr, len(parts), M, N, _ptr(absmax), _ptr(w_scale), _ptr(bias), _ptr(y),
+                                        _ptr(acc_out), flags, _stream(dev)), "bitlinear_epilogue_sum")
+    return y

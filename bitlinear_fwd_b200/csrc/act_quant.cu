@@ -75,7 +75,8 @@ __global__ void __launch_bounds__(kThreads) act_quant_kernel(const uint16_t* __r
                                                              int8_t* __restrict__ xq,
                                                              float* __restrict__ s_x,
                                                              int32_t* __restrict__ rowsum,
-                                                             uint32_t* status_clear, bool faithful) {
+                                                             uint32_t* status_clear, bool faithful,
+                                                             const float* __restrict__ absmax_in) {
   pdl_launch_dependents();
   pdl_wait_primary();
   if (status_clear && blockIdx.x == 0 && threadIdx.x == 0) *status_clear = 0u;
@@ -120,7 +121,8 @@ __global__ void __launch_bounds__(kThreads) act_quant_kernel(const uint16_t* __r
   amax = max(amax & 0xFFFFu, amax >> 16);
   amax = reduce_max_u32(amax, red);
 
-  const float a = bf16_bits_to_f32(amax);
+  // a K-shard takes the absmax of the whole row, all-reduced over the shards
+  const float a = absmax_in ? absmax_in[row] : bf16_bits_to_f32(amax);
   // float32: 127 / max(a, 1e-5).  bf16 module: PyTorch evaluates 127.0 / t as
   // t.reciprocal() * 127, each rounded to bf16.
   const float s = faithful ? bf16_round(__fmul_rn(bf16_round(__fdiv_rn(1.0f, fmaxf(a, bf16_round(1e-5f)))), 127.0f))
@@ -144,11 +146,36 @@ __global__ void __launch_bounds__(kThreads) act_quant_kernel(const uint16_t* __r
   }
 }
 
+// Per-token absmax over this x (one K-shard of the row), as float32: the
+// partial reduction of activation_norm_quant that an all-reduce MAX completes.
+__global__ void __launch_bounds__(kThreads) act_absmax_kernel(const uint16_t* __restrict__ x, int K,
+                                                              float* __restrict__ absmax) {
+  pdl_wait_primary();
+  __shared__ uint32_t red[kThreads / 32];
+  const int row = blockIdx.x;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<size_t>(row) * K);
+  uint32_t amax = 0;
+  for (int c = threadIdx.x; c < (K >> 3); c += kThreads) {
+    const uint4 a = __ldg(xr + c);
+    amax = absmax_pair(amax, a.x); amax = absmax_pair(amax, a.y);
+    amax = absmax_pair(amax, a.z); amax = absmax_pair(amax, a.w);
+  }
+  amax = max(amax & 0xFFFFu, amax >> 16);
+  amax = reduce_max_u32(amax, red);
+  if (threadIdx.x == 0) absmax[row] = bf16_bits_to_f32(amax);
+}
+
 }  // namespace
+
+cudaError_t launch_act_absmax(const uint16_t* x, int M, int K, float* absmax, cudaStream_t stream) {
+  if (M <= 0) return cudaSuccess;
+  act_absmax_kernel<<<M, kThreads, 0, stream>>>(x, K, absmax);
+  return cudaGetLastError();
+}
 
 template <int CPT>
 cudaError_t launch_cpt(const uint16_t* x, int M, int K, int8_t* xq, float* s_x, int32_t* rowsum,
-                       uint32_t* status_clear, bool pdl, cudaStream_t stream, bool faithful) {
+                       uint32_t* status_clear, bool pdl, cudaStream_t stream, bool faithful, const float* absmax_in) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(M, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -159,19 +186,20 @@ cudaError_t launch_cpt(const uint16_t* x, int M, int K, int8_t* xq, float* s_x, 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, act_quant_kernel<CPT>, x, K, xq, s_x, rowsum, status_clear, faithful);
+  return cudaLaunchKernelEx(&cfg, act_quant_kernel<CPT>, x, K, xq, s_x, rowsum, status_clear, faithful, absmax_in);
 }
 
 cudaError_t launch_act_quant(const uint16_t* x, int M, int K, int8_t* xq, float* s_x,
                              int32_t* rowsum, uint32_t* status_clear, bool pdl, cudaStream_t stream,
-                             bool faithful) {
+                             bool faithful, const float* absmax_in) {
   if (M <= 0) return cudaSuccess;
   const int chunks = K / 16;
-  if (chunks <= kThreads) return launch_cpt<1>(x, M, K, xq, s_x, rowsum, status_clear, pdl, stream, faithful);
-  if (chunks <= 2 * kThreads) return launch_cpt<2>(x, M, K, xq, s_x, rowsum, status_clear, pdl, stream, faithful);
-  if (chunks <= 4 * kThreads) return launch_cpt<4>(x, M, K, xq, s_x, rowsum, status_clear, pdl, stream, faithful);
-  if (chunks <= 8 * kThreads) return launch_cpt<8>(x, M, K, xq, s_x, rowsum, status_clear, pdl, stream, faithful);
-  return launch_cpt<0>(x, M, K, xq, s_x, rowsum, status_clear, pdl, stream, faithful);
+  const float* am = absmax_in;
+  if (chunks <= kThreads) return launch_cpt<1>(x, M, K, xq, s_x, rowsum, status_clear, pdl, stream, faithful, am);
+  if (chunks <= 2 * kThreads) return launch_cpt<2>(x, M, K, xq, s_x, rowsum, status_clear, pdl, stream, faithful, am);
+  if (chunks <= 4 * kThreads) return launch_cpt<4>(x, M, K, xq, s_x, rowsum, status_clear, pdl, stream, faithful, am);
+  if (chunks <= 8 * kThreads) return launch_cpt<8>(x, M, K, xq, s_x, rowsum, status_clear, pdl, stream, faithful, am);
+  return launch_cpt<0>(x, M, K, xq, s_x, rowsum, status_clear, pdl, stream, faithful, am);
 }
 
 }  // namespace bitlinear

@@ -459,6 +459,153 @@ int bitlinear_forward_host_async(const uint16_t* x_host, int64_t M, int64_t K, c
                            static_cast<cudaStream_t>(stream), false);
 }
 
+// ---- tensor-parallel K-split pieces -----------------------------------------
+
+static_assert(BITLINEAR_ABSMEAN_BINS == kAbsmeanBins, "header and kernels agree on the bin count");
+static_assert(BITLINEAR_MAX_PARTS == kMaxParts, "header and kernels agree on the partial-sum limit");
+
+int bitlinear_absmean_bins(const float* w, int64_t N, int64_t K, uint64_t* bins, void* stream) {
+  if (N < 1 || K < 64 || (K % 64) != 0 || N > kMaxMN || K > kMaxK || N * K >= (int64_t(1) << 39))
+    return BITLINEAR_ERR_SHAPE;
+  if (!w || !bins) return BITLINEAR_ERR_NULL;
+  if (misaligned(w) || misaligned(bins)) return BITLINEAR_ERR_ALIGN;
+  int st = check_device(nullptr);
+  if (st != BITLINEAR_OK) return st;
+  return status_of(launch_absmean_bins(w, N, K, bins, static_cast<cudaStream_t>(stream)));
+}
+
+int bitlinear_pack_weights_from_bins(const float* w, int64_t N, int64_t K, const uint64_t* bins, int64_t n_total,
+                                     uint8_t* packed, float* w_scale, float* w_mean, void* ws, size_t ws_bytes,
+                                     void* stream) {
+  if (N < 1 || K < 64 || (K % 64) != 0 || N > kMaxMN || K > kMaxK || N * K >= (int64_t(1) << 39))
+    return BITLINEAR_ERR_SHAPE;
+  if (n_total < N * K || n_total >= (int64_t(1) << 39)) return BITLINEAR_ERR_SHAPE;
+  if (!w || !bins || !packed || !w_scale) return BITLINEAR_ERR_NULL;
+  if (misaligned(w) || misaligned(bins) || misaligned(packed) || misaligned(w_scale) || misaligned(w_mean))
+    return BITLINEAR_ERR_ALIGN;
+  if (!ws || ws_bytes < kPackWsBytes) return BITLINEAR_ERR_WORKSPACE;
+  if (misaligned(ws)) return BITLINEAR_ERR_ALIGN;
+  int st = check_device(nullptr);
+  if (st != BITLINEAR_OK) return st;
+  return status_of(launch_pack_from_bins(w, N, K, bins, n_total, packed, w_scale, w_mean, pack_workspace(ws),
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+int bitlinear_act_absmax(const uint16_t* x, int64_t M, int64_t K, float* absmax, void* stream) {
+  if (M < 0 || M > kMaxMN || K < 64 || K > kMaxK || (K % 64) != 0) return BITLINEAR_ERR_SHAPE;
+  if (M == 0) return BITLINEAR_OK;
+  if (!x || !absmax) return BITLINEAR_ERR_NULL;
+  if (misaligned(x) || misaligned(absmax)) return BITLINEAR_ERR_ALIGN;
+  int st = check_device(nullptr);
+  if (st != BITLINEAR_OK) return st;
+  return status_of(launch_act_absmax(x, int(M), int(K), absmax, static_cast<cudaStream_t>(stream)));
+}
+
+int bitlinear_forward_partial(const uint16_t* x, int64_t M, int64_t K, const float* absmax, const uint8_t* packed_w,
+                              int64_t N, int32_t* acc, unsigned flags, void* ws, size_t ws_bytes, void* stream) {
+  if (flags & ~static_cast<unsigned>(BITLINEAR_BF16_FAITHFUL)) return BITLINEAR_ERR_SHAPE;
+  int st = check_shape(M, N, K);
+  if (st != BITLINEAR_OK) return st;
+  if (!x || !absmax || !packed_w || !acc) return BITLINEAR_ERR_NULL;
+  if (misaligned(x) || misaligned(absmax) || misaligned(packed_w) || misaligned(acc)) return BITLINEAR_ERR_ALIGN;
+  if (!ws || ws_bytes < bitlinear_workspace_bytes(M, N, K)) return BITLINEAR_ERR_WORKSPACE;
+  if (misaligned(ws)) return BITLINEAR_ERR_ALIGN;
+  if (M == 0) return BITLINEAR_OK;
+  int sms = 148;
+  st = check_device(&sms);
+  if (st != BITLINEAR_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const FwdLayout L = fwd_layout(M, N, K);
+  char* base = static_cast<char*>(ws);
+  uint32_t* status = reinterpret_cast<uint32_t*>(base);
+  float* s_x = reinterpret_cast<float*>(base + L.off_sx);
+  int32_t* rowsum = reinterpret_cast<int32_t*>(base + L.off_rs);
+  int8_t* xq = reinterpret_cast<int8_t*>(base + L.off_xq);
+  // this shard's x, quantised with the scale of the whole row
+  const bool faithful = (flags & BITLINEAR_BF16_FAITHFUL) != 0;
+  if (launch_act_quant(x, int(M), int(K), xq, s_x, rowsum, status, false, s, faithful, absmax) != cudaSuccess)
+    return BITLINEAR_ERR_CUDA;
+  // the contraction alone: exact int32 partial sums, no bf16 output
+  if (M > 16) {
+    ForwardArgs a;
+    a.xq = xq;
+    a.s_x = s_x;
+    a.rowsum = rowsum;
+    a.packed = packed_w;
+    a.w_scale = s_x;              // any finite scale: the quotient is not stored
+    a.bias = nullptr;
+    a.y = nullptr;
+    a.acc_out = acc;
+    a.y32_out = nullptr;
+    a.status = status;
+    a.M = int(M);
+    a.N = int(N);
+    a.K = int(K);
+    a.pdl = true;
+    a.faithful = false;
+    a.ngroups = 1;
+    a.group_end[0] = int(N);
+    a.wait_ns = launch_wait_ns();
+    a.stall = launch_stall();
+    return status_of(launch_gemm_prefill(a, sms, s));
+  }
+  DecodeArgs d;
+  d.x = nullptr;
+  d.xq = xq;
+  d.s_x = s_x;
+  d.packed = packed_w;
+  d.w_scale = s_x;
+  d.bias = nullptr;
+  d.y = nullptr;
+  d.xq_out = nullptr;
+  d.sx_out = nullptr;
+  d.acc_out = acc;
+  d.y32_out = nullptr;
+  d.status = status;
+  d.M = int(M);
+  d.N = int(N);
+  d.K = int(K);
+  d.weights_early = 0;
+  d.faithful = 0;
+  d.ngroups = 1;
+  d.group_end[0] = int(N);
+  d.wait_ns = launch_wait_ns();
+  d.stall = launch_stall();
+  return status_of(launch_decode(d, sms, s));
+}
+
+int bitlinear_epilogue_sum(const int32_t* const* partials, int nparts, int64_t M, int64_t N, const float* absmax,
+                           const float* w_scale, const uint16_t* bias, uint16_t* y, int32_t* acc_out,
+                           unsigned flags, void* stream) {
+  if (flags & ~static_cast<unsigned>(BITLINEAR_BF16_FAITHFUL)) return BITLINEAR_ERR_SHAPE;
+  if (M < 0 || M > kMaxMN || N < 1 || N > kMaxMN) return BITLINEAR_ERR_SHAPE;
+  if (nparts < 1 || nparts > BITLINEAR_MAX_PARTS) return BITLINEAR_ERR_SHAPE;
+  if (!partials) return BITLINEAR_ERR_NULL;
+  if (M == 0) return BITLINEAR_OK;
+  EpilogueArgs a{};
+  for (int r = 0; r < nparts; ++r) {
+    if (!partials[r]) return BITLINEAR_ERR_NULL;
+    if (misaligned(partials[r])) return BITLINEAR_ERR_ALIGN;
+    a.part[r] = partials[r];
+  }
+  if (!absmax || !w_scale || !y) return BITLINEAR_ERR_NULL;
+  if (misaligned(absmax) || misaligned(w_scale) || misaligned(bias) || misaligned(y) || misaligned(acc_out))
+    return BITLINEAR_ERR_ALIGN;
+  int sms = 148;
+  int st = check_device(&sms);
+  if (st != BITLINEAR_OK) return st;
+  a.nparts = nparts;
+  a.absmax = absmax;
+  a.w_scale = w_scale;
+  a.bias = bias;
+  a.y = y;
+  a.acc_out = acc_out;
+  a.M = M;
+  a.N = N;
+  a.faithful = (flags & BITLINEAR_BF16_FAITHFUL) ? 1 : 0;
+  return status_of(launch_epilogue(a, sms, static_cast<cudaStream_t>(stream)));
+}
+
 int bitlinear_test_force_timeout(int on) {
   return g_force_timeout.exchange(on ? 1 : 0);
 }

@@ -59,10 +59,15 @@ constexpr uint32_t kOffD = kOffWp + STAGES * kWpBytes;       // s_x per token [B
 constexpr uint32_t kOffRs = kOffD + 4 * BT;                  // row sums per token [BT]
 constexpr uint32_t kOffBar = kOffRs + 4 * BT;
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;        // + barriers, alignment slack
+// tcgen05.alloc of all 512 columns waits until the columns are free, with no
+// time limit.  It never waits here because two CTAs of this kernel cannot
+// share an SM (their shared memory exceeds the SM's 228 KB), and no other
+// kernel of the library uses tensor memory.
+static_assert(2 * kSmemBytes > 228 * 1024, "one GEMM CTA per SM keeps the 512-column allocation uncontended");
 
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_prefill_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
-                        const ForwardArgs a, uint64_t wait_ns) {
+                        const ForwardArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kOffBar);
@@ -73,6 +78,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* drain = acc_empty + 2;            // every issued MMA has completed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* failed = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* drain_bad = failed + 1;       // a drain gave up: MMAs may still run
+  uint64_t* stall_bar = reinterpret_cast<uint64_t*>(smem + kOffBar + 224);   // never signalled (test hook)
+  const uint64_t wait_ns = a.wait_ns;
   float* d_s = reinterpret_cast<float*>(smem + kOffD);
   int* rs_s = reinterpret_cast<int*>(smem + kOffRs);
 
@@ -92,7 +100,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&acc_empty[b], kEpiWarps);
     }
     mbar_init(drain, 1);
+    mbar_init(stall_bar, 1);
     *failed = 0;
+    *drain_bad = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_x);
     tma_prefetch_desc(&tm_w);
@@ -130,10 +140,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(smem + kOffX + s * kXBytes, &tm_x, &full[s], kb * BK, m0);
         }
       }
-      // drain: the last copy issued into each stage has landed
+      // drain: the last copy issued into each stage has landed.  The drain
+      // keeps the fixed limit whatever the main loop's limit is, so that no
+      // copy is still writing shared memory when the CTA exits.
       for (int s = 0; s < STAGES; ++s) {
         const int cnt = g > s ? (g - 1 - s) / STAGES + 1 : 0;
-        if (cnt > 0 && !mbar_wait(&full[s], (cnt - 1) & 1, wait_ns)) *failed = 1;
+        if (cnt > 0 && !mbar_wait(&full[s], (cnt - 1) & 1, kWaitLimitNs)) {
+          *failed = 1;
+          *drain_bad = 1;
+        }
       }
     }
   } else if (warp == 1) {
@@ -141,6 +156,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---------------- MMA issuer ----------------
       constexpr uint32_t idesc = umma_idesc_i8(BW, BT, true, true);
       int g = 0, j = 0;
+      // forced-timeout test: a wait that nothing completes runs out, and the
+      // CTA takes the same path as after any wait that gives up
+      if (a.stall && !mbar_wait(stall_bar, 0, wait_ns)) *failed = 1;
       for (int tile = blockIdx.x; tile < ntiles && !*failed; tile += gridDim.x, ++j) {
         const int b = j & 1;
         // the epilogue has read this buffer's previous tile (fresh barriers pass parity 1)
@@ -168,8 +186,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_commit(&acc_full[b]);                // the tile's accumulator is complete
       }
       // every MMA issued above has completed before tensor memory is freed
+      // (fixed limit, as for the copies)
       umma_commit(drain);
-      if (!mbar_wait(drain, 0, wait_ns)) *failed = 1;
+      if (!mbar_wait(drain, 0, kWaitLimitNs)) {
+        *failed = 1;
+        *drain_bad = 1;
+      }
     }
   } else if (warp >= 4 && warp < 8) {
     // ---------------- weight unpack into tensor memory ----------------
@@ -214,9 +236,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int g = 0; g < kMaxGroups; ++g) swg[g] = g < a.ngroups ? a.w_scale[g] : 0.0f;
     const bool simple = a.ngroups == 1 && !a.faithful;
     int j = 0;
-    // The four epilogue warps meet at a named barrier twice per tile; every
+    // The eight epilogue warps meet at a named barrier twice per tile; every
     // one of them runs every iteration (a failure only skips work), so the
-    // barrier always gets its 128 threads.
+    // barrier always gets its 256 threads.
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++j) {
       const int b = j & 1;
       const int n0 = (tile % wtiles) * BW, m0 = (tile / wtiles) * BT;
@@ -260,7 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!nv) continue;
         auto emit = [&](int mi, int accv, float y32) {
           const size_t o = static_cast<size_t>(m0 + mi) * a.N + n;
-          a.y[o] = f32_to_bf16_bits(y32);
+          if (a.y) a.y[o] = f32_to_bf16_bits(y32);
           if (a.acc_out) a.acc_out[o] = accv;
           if (a.y32_out) a.y32_out[o] = y32;
         };
@@ -304,7 +326,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0 && *failed) report_status(a.status, kStatusTimeout);
-  if (warp == 2) {
+  // Tensor memory is freed only when every MMA is known to have completed;
+  // after a drain that gave up (never seen: it needs MMAs or copies stuck
+  // for a whole second) the CTA exits without freeing it rather than free
+  // it under a running MMA.
+  if (warp == 2 && !*drain_bad) {
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
   }
@@ -332,7 +358,7 @@ cudaError_t launch_gemm_prefill(const ForwardArgs& a, int num_sms, cudaStream_t 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = a.pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, gemm_prefill_kernel, tm_x, tm_w, a, kWaitLimitNs);
+  return cudaLaunchKernelEx(&cfg, gemm_prefill_kernel, tm_x, tm_w, a);
 }
 
 }  // namespace bitlinear

@@ -158,6 +158,7 @@ __device__ __forceinline__ int bytesum16(uint4 v, int sum) {
 struct SmemTail {
   uint64_t full[kMaxRing];
   uint64_t empty[kMaxRing];
+  uint64_t stall;                    // never signalled (forced-timeout test hook)
   uint32_t amax[16];                 // absmax per token (bf16 bits)
   int rsum[16];                      // sum of q per token
   float sx[16];                      // s_x per token
@@ -218,6 +219,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
       mbar_init(&sm.full[s], 1);
       mbar_init(&sm.empty[s], kConsumerWarps);
     }
+    mbar_init(&sm.stall, 1);
     fence_mbar_init();
     if (kc > 0) tma_prefetch_desc(&tm3);
     if (a.tail) tma_prefetch_desc(&tm2);
@@ -250,7 +252,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
         const uint32_t bytes = (has3 ? kc * kSubBytes : 0) + (hast ? kSubBytes : 0);
         for (int u = 0; u < U; ++u, ++q) {
           const int s = q % ring;
-          if (q >= ring && !mbar_wait(&sm.empty[s], ((q / ring) - 1) & 1, kWaitLimitNs)) {
+          if (q >= ring && !mbar_wait(&sm.empty[s], ((q / ring) - 1) & 1, a.wait_ns)) {
             ok = false;
             break;
           }
@@ -376,6 +378,9 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
     }
     consumer_sync();
 
+    // forced-timeout test: a wait that nothing completes runs out, and the
+    // CTA takes the same path as after any wait that gives up
+    if (a.stall && !mbar_wait(&sm.stall, 0, a.wait_ns)) ok = false;
     const int r0 = mma_row_to_box(g);                // sub-box rows r0 and r0 + 8
     for (int r = 0; r < nround; ++r) {
       const int c0 = r * kChunkK;
@@ -459,7 +464,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
         // every consumer warp waits for every load (also when it has no
         // sub-box in it): its arrival on the empty barrier must not run ahead
         // of the slot's phases
-        if (ok && !mbar_wait(&sm.full[s], (q / ring) & 1, kWaitLimitNs)) ok = false;
+        if (ok && !mbar_wait(&sm.full[s], (q / ring) & 1, a.wait_ns)) ok = false;
         if (!ok) break;
         int acc[4][NT][4];
 #pragma unroll
@@ -555,7 +560,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
       if (a.bias) y32 = bf16_round(__fadd_rn(y32, bf16_bits_to_f32(bias_s[rl])));
     }
     const size_t o = static_cast<size_t>(m) * N + n;
-    a.y[o] = f32_to_bf16_bits(y32);
+    if (a.y) a.y[o] = f32_to_bf16_bits(y32);
     if (a.acc_out) a.acc_out[o] = accv;
     if (a.y32_out) a.y32_out[o] = y32;
   }

@@ -25,9 +25,13 @@ bool encode_3d_u8(CUtensorMap* map, const void* base, const uint64_t dims[3], co
 // (the kernel waits for it before touching memory).
 // faithful: the bf16-module rounding of every step (scale = bf16(bf16(1/a) * 127),
 // q = round(bf16(x * scale))) instead of float32 arithmetic
+// absmax_in: the tokens' absmax over the whole row when x is one K-shard of
+// it (null: the kernel forms it from x)
 cudaError_t launch_act_quant(const uint16_t* x, int M, int K, int8_t* xq, float* s_x,
                              int32_t* rowsum, uint32_t* status_clear, bool pdl, cudaStream_t stream,
-                             bool faithful = false);
+                             bool faithful = false, const float* absmax_in = nullptr);
+// float32 max_k |x[m, k]| of each token over this x
+cudaError_t launch_act_absmax(const uint16_t* x, int M, int K, float* absmax, cudaStream_t stream);
 
 // ---- weight absmean + ternarise + pack (pack.cu) ----------------------------
 // Workspace layout used by the pack kernels.
@@ -44,6 +48,29 @@ constexpr size_t kPackWsBytes = 4096;
 PackWorkspace pack_workspace(void* ws);
 cudaError_t launch_pack(const float* w, int64_t N, int64_t K, uint8_t* packed, float* w_scale,
                         float* w_mean, const PackWorkspace& pws, cudaStream_t stream);
+// The exact exponent-bin form of sum |w| over this w (bins[kAbsmeanBins] are
+// overwritten): integer bins that add across shards.
+cudaError_t launch_absmean_bins(const float* w, int64_t N, int64_t K, uint64_t* bins, cudaStream_t stream);
+// s_w and the exact mean from bins summed over all shards (n_total weights
+// in all), then the ternary codes of this w.
+cudaError_t launch_pack_from_bins(const float* w, int64_t N, int64_t K, const uint64_t* bins, int64_t n_total,
+                                  uint8_t* packed, float* w_scale, float* w_mean, const PackWorkspace& pws,
+                                  cudaStream_t stream);
+
+// ---- epilogue over summed partial accumulators (epilogue.cu) ---------------
+constexpr int kMaxParts = 8;
+struct EpilogueArgs {
+  const int32_t* part[kMaxParts];  // [M, N] int32 partial sums, added in order
+  int nparts;
+  const float* absmax;    // [M] tokens' absmax over the whole K
+  const float* w_scale;   // [1]
+  const uint16_t* bias;   // [N] or null
+  uint16_t* y;            // [M, N]
+  int32_t* acc_out;       // [M, N] or null: the summed accumulators
+  int64_t M, N;
+  int faithful;
+};
+cudaError_t launch_epilogue(const EpilogueArgs& a, int num_sms, cudaStream_t stream);
 
 // ---- shared forward arguments ----------------------------------------------
 // Rows [group_end[g-1], group_end[g]) of the packed matrix form group g,

@@ -285,6 +285,80 @@ int bitlinear_noalloc_check_status(void* stream);
  * up since the last reset.  `ws_bytes` is the size the calls were given. */
 int bitlinear_check_status(const void* ws, size_t ws_bytes, void* stream);
 
+/* ---- Tensor-parallel K-split (row-parallel) pieces -------------------------
+ *
+ * BitLinear.forward and _weight_quant (Falcon-Edge blog, section
+ * "Falcon-Edge, a series of universal models") reduce over whole tensors:
+ * s_x takes each token's absmax over all of K, and s_w takes mean |w| over the
+ * whole weight matrix.  When x and W are split along K over several GPUs
+ * (rank r holds x[:, K_r] and W[:, K_r]), these calls plus three exchanges
+ * reproduce the unsplit forward bit for bit:
+ *   packing:  bitlinear_absmean_bins on each shard -> all-reduce SUM of the
+ *             uint64 bins (exact integers) -> bitlinear_pack_weights_from_bins
+ *             on each shard with the summed bins and the total element count;
+ *   forward:  bitlinear_act_absmax -> all-reduce MAX of the [M] floats ->
+ *             bitlinear_forward_partial (int32 partial sums over K_r) ->
+ *             all-reduce SUM of the int32 [M, N] partials (exact) ->
+ *             bitlinear_epilogue_sum; or, with peer access, pass every rank's
+ *             partial sums to bitlinear_epilogue_sum, which adds them as it
+ *             reads them.
+ * Each exchange is exact and independent of order, so every rank gets the
+ * same bits as the unsplit call. */
+
+/* Number of exponent bins of the exact sum of |w|. */
+#define BITLINEAR_ABSMEAN_BINS 320
+
+/* The exact sum of |w| over this shard as integer exponent bins:
+ * sum |w| = sum_e bins[e] * 2^(max(e,1) - 150).  The bins of several shards
+ * add (as uint64) to the bins of their union.
+ *   w     [N, K] float32, finite (N * K below 2^39)
+ *   bins  [BITLINEAR_ABSMEAN_BINS] uint64 out (device), overwritten */
+int bitlinear_absmean_bins(const float* w, int64_t N, int64_t K, uint64_t* bins, void* stream);
+
+/* bitlinear_pack_weights for one shard of a larger weight matrix: s_w and
+ * the exact mean come from `bins` -- the bins of all shards added -- and
+ * n_total, the element count of the whole matrix (>= N * K, below 2^39);
+ * the codes of this shard are then packed with that s_w.  Other arguments
+ * as for bitlinear_pack_weights. */
+int bitlinear_pack_weights_from_bins(const float* w, int64_t N, int64_t K, const uint64_t* bins, int64_t n_total,
+                                     uint8_t* packed, float* w_scale, float* w_mean, void* ws, size_t ws_bytes,
+                                     void* stream);
+
+/* Each token's max_k |x[m, k]| over this x (one K-shard of the row), as
+ * float32 (exact: bf16 widens exactly).
+ *   x       [M, K] bf16
+ *   absmax  [M] float32 out (device) */
+int bitlinear_act_absmax(const uint16_t* x, int64_t M, int64_t K, float* absmax, void* stream);
+
+/* The contraction of one K-shard: x is quantised with s_x = 127 / max(a,
+ * 1e-5) from the whole row's absmax a (the all-reduced output of
+ * bitlinear_act_absmax), and contracted with this shard's packed weights.
+ *   x        [M, K] bf16, this shard's columns
+ *   absmax   [M] float32 (device), absmax over the whole K
+ *   packed_w [N, K/4] uint8, this shard's packed columns
+ *   acc      [M, N] int32 out: sum over this shard's k of q * u (exact)
+ *   flags    0, or BITLINEAR_BF16_FAITHFUL for the bf16 module's s_x and q
+ *            (give the same flag to bitlinear_epilogue_sum)
+ *   ws       workspace of bitlinear_workspace_bytes(M, N, K) bytes
+ * Same shape rules and engines as bitlinear_forward. */
+int bitlinear_forward_partial(const uint16_t* x, int64_t M, int64_t K, const float* absmax, const uint8_t* packed_w,
+                              int64_t N, int32_t* acc, unsigned flags, void* ws, size_t ws_bytes, void* stream);
+
+/* The epilogue on partial sums: acc = partials[0] + ... + partials[n-1]
+ * (int32, exact), then y = bf16(acc / (s_x * s_w) (+ bias)) with s_x from
+ * absmax, as the forward does (flags: 0 or BITLINEAR_BF16_FAITHFUL).
+ *   partials  host array of nparts (1 .. BITLINEAR_MAX_PARTS) device
+ *             pointers, each [M, N] int32; they may point into other GPUs'
+ *             memory through peer access (plain loads only).  Every partial
+ *             sum must be complete before this call's kernel starts.
+ *   absmax    [M] float32 (device), the tokens' absmax over the whole K
+ *   w_scale   [1] float32 (device); bias [N] bf16 or NULL; y [M, N] bf16 out
+ *   acc_out   [M, N] int32 out, the summed accumulators, or NULL */
+#define BITLINEAR_MAX_PARTS 8
+int bitlinear_epilogue_sum(const int32_t* const* partials, int nparts, int64_t M, int64_t N, const float* absmax,
+                           const float* w_scale, const uint16_t* bias, uint16_t* y, int32_t* acc_out,
+                           unsigned flags, void* stream);
+
 /* Test hook for the failure path of the device-side waits.  While it is on
  * (on != 0), every forward launched by this process -- bitlinear_forward and
  * its variants, both engines -- makes one wait on a barrier that nothing

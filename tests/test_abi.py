@@ -177,9 +177,50 @@ def test_valid_arguments_pass_every_host_check(lib):
         "host_async": lib.bitlinear_forward_host_async(18, 8, 256, 16, 512, 16, None, 18, 3, 16, host_ws, None),
         "noalloc": lib.bitlinear_forward_noalloc(16, 8, 256, 16, 512, 16, None, 16, None),
         "noalloc status": lib.bitlinear_noalloc_check_status(None),
+        "absmean bins": lib.bitlinear_absmean_bins(16, 512, 256, 16, None),
+        "pack from bins": lib.bitlinear_pack_weights_from_bins(16, 512, 256, 16, 1024 * 256, 16, 16, 16, 16, 4096,
+                                                               None),
+        "act absmax": lib.bitlinear_act_absmax(16, 4, 256, 16, None),
+        "forward partial": lib.bitlinear_forward_partial(16, 8, 256, 16, 16, 512, 16, 0, 16, 1 << 20, None),
+        "forward partial M=40": lib.bitlinear_forward_partial(16, 40, 256, 16, 16, 512, 16, 2, 16, 1 << 20, None),
+        "epilogue sum": lib.bitlinear_epilogue_sum((ctypes.c_void_p * 2)(16, 32), 2, 8, 512, 16, 16, 16, 16, None,
+                                                   0, None),
         "pack": lib.bitlinear_pack_weights(16, 512, 256, 16, 16, 16, 16, 4096, None),
         "quant_act": lib.bitlinear_quant_act(16, 4, 256, 16, 16, 16, None),
         "dequant": lib.bitlinear_dequant_weights(16, 512, 256, 16, 16, None),
     }
     wrong = {k: v for k, v in calls.items() if v not in no_device}
     assert not wrong, wrong
+
+
+def test_ksplit_entry_points_reject_bad_arguments(lib):
+    """The tensor-parallel K-split calls check shapes, pointers, alignment and
+    workspace before anything is enqueued."""
+    bins = lib.bitlinear_absmean_bins
+    assert bins(16, 512, 100, 16, None) == -2
+    assert bins(None, 512, 256, 16, None) == -1
+    assert bins(16, 512, 256, 18, None) == -3
+    pfb = lib.bitlinear_pack_weights_from_bins
+    assert pfb(16, 512, 256, 16, 512 * 256 - 1, 16, 16, None, 16, 4096, None) == -2   # n_total below N*K
+    assert pfb(16, 512, 256, 16, 1 << 39, 16, 16, None, 16, 4096, None) == -2
+    assert pfb(16, 512, 256, None, 512 * 256, 16, 16, None, 16, 4096, None) == -1
+    assert pfb(16, 512, 256, 16, 512 * 256, 16, 16, None, 16, 100, None) == -4
+    am = lib.bitlinear_act_absmax
+    assert am(16, 4, 100, 16, None) == -2
+    assert am(16, 0, 256, None, None) == 0
+    assert am(16, 4, 256, 20, None) == -3
+    part = lib.bitlinear_forward_partial
+    assert part(16, 8, 256, None, 16, 512, 16, 0, 16, 1 << 20, None) == -1
+    assert part(16, 8, 256, 16, 16, 512, 16, 4, 16, 1 << 20, None) == -2        # unknown flag
+    assert part(16, 8, 256, 16, 16, 512, 16, 0, 16, 64, None) == -4
+    assert part(16, 8, 256, 16, 16, 512, 24, 0, 16, 1 << 20, None) == -3
+    assert part(16, 0, 256, 16, 16, 512, 16, 0, 16, 1 << 20, None) == 0
+    ep = lib.bitlinear_epilogue_sum
+    two = (ctypes.c_void_p * 2)(16, 32)
+    assert ep(two, 0, 8, 512, 16, 16, None, 16, None, 0, None) == -2
+    assert ep(two, 9, 8, 512, 16, 16, None, 16, None, 0, None) == -2
+    assert ep(None, 2, 8, 512, 16, 16, None, 16, None, 0, None) == -1
+    assert ep((ctypes.c_void_p * 2)(16, None), 2, 8, 512, 16, 16, None, 16, None, 0, None) == -1
+    assert ep((ctypes.c_void_p * 2)(16, 20), 2, 8, 512, 16, 16, None, 16, None, 0, None) == -3
+    assert ep(two, 2, 8, 512, 16, 16, None, 16, None, 8, None) == -2
+    assert ep(two, 2, 0, 512, 16, 16, None, 16, None, 0, None) == 0
