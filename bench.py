@@ -98,18 +98,18 @@ def kernel_src_hash(name):
     return hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
 
 
-def traffic_from_profile(profile_md, src_name):
-    """DRAM bytes per launch recorded in a committed ncu summary, or None when
-    the summary is missing or the kernel source changed since the capture."""
-    p = os.path.join(ROOT, "profiles", profile_md)
+def traffic_from_profile(kernel, src_name):
+    """DRAM bytes per launch of ``kernel`` from an ncu capture, as recorded in
+    profiles/traffic.json (written beside the capture's summary), or None
+    when there is no record or the kernel's source changed since the
+    capture."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
-    text = open(p).read()
-    m = re.search(r"dram_bytes_per_launch_full_workload:\s*([0-9.eE+]+)", text)
-    h = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
-    if not m or not h or h.group(1) != kernel_src_hash(src_name):
+    rec = json.load(open(p)).get(kernel)
+    if not rec or rec.get("source_sha256_16") != kernel_src_hash(src_name):
         return None
-    return float(m.group(1))
+    return float(rec["dram_bytes_per_launch"])
 
 
 class ClockSampler:
@@ -329,7 +329,7 @@ def run_decode(args, hbm_gbs, l2_bytes, peak_kind):
     per_case = [{"M": p.M, "N": p.N, "K": p.K, "isolated_us": round(t * 1e3, 3),
                  "isolated_gbs": round(decode_bytes(p.M, p.N, p.K) / (t * 1e-3) / 1e9, 1)}
                 for p, t in zip(probs, kt)]
-    traffic = traffic_from_profile("decode_kernel_w2.md", "gemv_decode.cu")
+    traffic = traffic_from_profile("decode_kernel", "gemv_decode.cu")
     roof = {"kernel": "decode_kernel", "bound": "hbm", "achieved": round(achieved, 1),
             "peak": hbm_gbs, "unit": "GB/s", "frac": round(achieved / hbm_gbs, 4),
             "peak_source": f"{peak_kind} HBM copy bandwidth (burst figure)",
@@ -341,38 +341,76 @@ def run_decode(args, hbm_gbs, l2_bytes, peak_kind):
 
 
 def run_e2e(args, probs, steps):
+    """The headline metric end to end through bitlinear_forward_host_async:
+    every call copies its bf16 x from pinned host memory to the device and
+    its bf16 y back, and each step waits for its results.  The step's six
+    calls (12 copies, 6 kernels) are captured once as a CUDA graph -- the
+    library's calls are stream-ordered, so a graph holds them as they are --
+    and each step is one graph launch plus one synchronisation.  The same
+    steps issued call by call (no graph) are reported beside it."""
     import bitlinear_fwd_b200 as bl
     xs = [p.x.cpu().pin_memory() for p in probs]
     ys = [torch.empty((p.M, p.N), dtype=torch.bfloat16).pin_memory() for p in probs]
     wss = [bl.workspace(p.M, p.N, p.K, "cuda", host=True) for p in probs]
+    bytes_step = sum(decode_bytes(p.M, p.N, p.K, p.bias is not None) for p in probs)
+    copies = len(probs[0].packed)
 
-    def step(r):
-        # the step's six calls are enqueued (host x in, host y out), then the
-        # step waits for its results
+    def enqueue(r):
         for p, x, y, ws in zip(probs, xs, ys, wss):
-            bl.bitlinear_forward_host_async(x, p.packed[r % len(p.packed)], p.s_w, p.bias, y_host=y, ws=ws,
+            bl.bitlinear_forward_host_async(x, p.packed[r % copies], p.s_w, p.bias, y_host=y, ws=ws,
                                             flags=bl.WEIGHTS_RESIDENT)
+
+    def timed(step_fn):
+        for i in range(3):
+            step_fn(i)
+        sync_all()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(steps):
+            step_fn(i)
+        e1.record()
+        e1.synchronize()
+        sync_all()
+        return elapsed_max_over_ranks(e0.elapsed_time(e1))
+
+    def plain_step(r):
+        enqueue(r)
         torch.cuda.current_stream().synchronize()
 
-    for i in range(3):
-        step(i)
-    sync_all()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for i in range(steps):
-        step(i)
-    e1.record()
-    e1.synchronize()
-    sync_all()
-    ms = elapsed_max_over_ranks(e0.elapsed_time(e1))
-    bytes_step = sum(decode_bytes(p.M, p.N, p.K, p.bias is not None) for p in probs)
-    return {"value": round(whole_job_gbs(bytes_step, steps, ms, world_size()), 2), "unit": "GB/s",
+    ms_plain = timed(plain_step)
+    # one graph per weight copy, captured on a side stream
+    graphs = []
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        enqueue(0)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    for r in range(copies):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            enqueue(r)
+        graphs.append(g)
+
+    def graph_step(r):
+        graphs[r % copies].replay()
+        torch.cuda.current_stream().synchronize()
+
+    ms = timed(graph_step)
+    del graphs
+    world = world_size()
+    return {"value": round(whole_job_gbs(bytes_step, steps, ms, world), 2), "unit": "GB/s",
             "h2d_bytes_per_step": sum(2 * p.M * p.K for p in probs),
             "d2h_bytes_per_step": sum(2 * p.M * p.N for p in probs),
-            "api": "bitlinear_forward_host_async (pinned host x in, host y out), one stream sync per step"}
+            "us_per_step": round(ms * 1e3 / steps, 2),
+            "api": "bitlinear_forward_host_async (pinned host x in, host y out) x 6 per step, the step "
+                   "captured once as a CUDA graph; one graph launch and one stream sync per step",
+            "without_graph": {"value": round(whole_job_gbs(bytes_step, steps, ms_plain, world), 2),
+                              "unit": "GB/s", "us_per_step": round(ms_plain * 1e3 / steps, 2),
+                              "api": "the same six calls issued one by one, one stream sync per step"}}
 
 
-def run_prefill(args, bf16_tflops, peak_kind, l2_bytes):
+def run_prefill(args, bf16_tflops, peak_kind, l2_bytes, i8_peak=None):
     cases = wl.workload3()
     probs, copies = make_problems(cases, l2_bytes, rotate_factor=1.0, max_copies=3, force_copies=args.copies)
     graphs = capture_steps(probs, copies, "forward")
@@ -383,10 +421,11 @@ def run_prefill(args, bf16_tflops, peak_kind, l2_bytes):
     kt = kernel_times(probs, copies, reps=8)
     ops = [2 * p.M * p.N * p.K for p in probs]
     achieved = sum(ops) / (sum(kt) * 1e-3) / 1e12
-    peak = bf16_tflops * INT8_OVER_BF16
+    peak_bf16x2 = bf16_tflops * INT8_OVER_BF16
+    peak = i8_peak["tops"] if i8_peak else peak_bf16x2
     per_case = [{"M": p.M, "N": p.N, "K": p.K, "us": round(t * 1e3, 2),
                  "tops": round(o / (t * 1e-3) / 1e12, 1)} for p, t, o in zip(probs, kt, ops)]
-    traffic = traffic_from_profile("gemm_prefill_w3.md", "gemm_prefill.cu")
+    traffic = traffic_from_profile("gemm_prefill_kernel", "gemm_prefill.cu")
     del graphs
     return {"metric": "BitLinear prefill int8 TOPS (bitlinear_forward incl. activation quantisation)",
             "value": round(tops, 1), "unit": "TOPS", "ms_per_step": round(ms / steps, 4), "steps": steps,
@@ -394,7 +433,10 @@ def run_prefill(args, bf16_tflops, peak_kind, l2_bytes):
                         "bf16, W N(0,0.02) ternarised; 6 forwards per step",
             "roofline": {"kernel": "gemm_prefill_kernel", "bound": "tensor", "achieved": round(achieved, 1),
                          "peak": round(peak, 1), "unit": "TOPS", "frac": round(achieved / peak, 4),
-                         "peak_source": f"{peak_kind} bf16 dense x {INT8_OVER_BF16:g} (nominal int8/bf16)",
+                         "peak_source": ("measured int8 tensor-core rate (bitlinear_measure_i8_peak, this run)"
+                                         if i8_peak else
+                                         f"{peak_kind} bf16 dense x {INT8_OVER_BF16:g} (nominal int8/bf16)"),
+                         "peak_bf16x2": round(peak_bf16x2, 1), "frac_of_bf16x2": round(achieved / peak_bf16x2, 4),
                          "traffic": traffic, "per_case": per_case}}
 
 
@@ -655,7 +697,8 @@ class OracleDecode:
     row): the numpy oracle, or with ``impl="cpp"`` the plain C++ one.
     Inputs are generated and packed by that oracle once, untimed."""
 
-    def __init__(self, impl="numpy"):
+    def __init__(self, impl="numpy", threads=1):
+        self.threads = max(1, int(threads))
         if impl == "cpp":
             from oracle import cpp as oracle
         else:
@@ -677,10 +720,12 @@ class OracleDecode:
             self.items.append((synth.bf16_bits(c.x()), packed, s_w, synth.bf16_bits(c.bias()),
                                decode_bytes(c.M, c.N, c.K)))
         if impl == "cpp":
-            self.cores = 1
+            self.cores = self.threads
             self.desc = ("the C++ oracle's forward (plain loops: act quant, unpack, int64 contraction, "
-                         "epilogue) on the 6 decode problems with every weight row, packing untimed; "
-                         "one thread")
+                         "epilogue) on the 6 decode problems with every weight row, packing untimed; " +
+                         ("one thread" if self.threads == 1 else
+                          f"{self.threads} host threads, each calling it on its own block of weight rows "
+                          "(the oracle itself unchanged)"))
         else:
             self.cores = self.blas
             self.desc = ("oracle.forward (act quant, unpack, exact contraction, epilogue) on the 6 decode "
@@ -690,18 +735,36 @@ class OracleDecode:
     def step(self):
         """One pass over the workload; returns (bytes, seconds)."""
         b, s = 0, 0.0
-        for xb, packed, s_w, bb, nbytes in self.items:
-            t0 = time.perf_counter()
-            self.oracle.forward(xb, packed, s_w, bb)
-            s += time.perf_counter() - t0
-            b += nbytes
+        pool = None
+        if self.threads > 1:
+            import concurrent.futures as fut
+            pool = fut.ThreadPoolExecutor(self.threads)
+        try:
+            for xb, packed, s_w, bb, nbytes in self.items:
+                t0 = time.perf_counter()
+                if pool is None:
+                    self.oracle.forward(xb, packed, s_w, bb)
+                else:
+                    # rows are independent: each thread runs the oracle on one block of them
+                    N = packed.shape[0]
+                    cuts = np.linspace(0, N, self.threads + 1).astype(int)
+                    jobs = [pool.submit(self.oracle.forward, xb, np.ascontiguousarray(packed[a:c]), s_w,
+                                        None if bb is None else np.ascontiguousarray(bb[a:c]))
+                            for a, c in zip(cuts[:-1], cuts[1:]) if c > a]
+                    for j in jobs:
+                        j.result()
+                s += time.perf_counter() - t0
+                b += nbytes
+        finally:
+            if pool is not None:
+                pool.shutdown()
         return b, s
 
 
-def timed_oracle(impl, budget_s, max_passes=8):
+def timed_oracle(impl, budget_s, max_passes=8, threads=1):
     """Passes of one CPU oracle over the decode workload until ``budget_s``
     seconds of oracle time; a cpu_baseline-style dict."""
-    od = OracleDecode(impl)
+    od = OracleDecode(impl, threads)
     b, s, n = 0, 0.0, 0
     while s < budget_s and n < max_passes:
         bb, ss = od.step()
@@ -765,9 +828,15 @@ def oracle_workloads_baseline():
 
 
 def cpp_oracle_baseline(budget_s=5.0):
-    """The C++ oracle timed beside the numpy one; never fails the line."""
+    """The C++ oracle timed beside the numpy one, on one thread and on every
+    host core (nproc); never fails the line."""
     try:
-        return timed_oracle("cpp", budget_s)
+        one = timed_oracle("cpp", budget_s)
+        nproc = os.cpu_count() or 1
+        one["nproc"] = nproc
+        if nproc > 1:
+            one["all_cores"] = timed_oracle("cpp", budget_s, threads=nproc)
+        return one
     except Exception as e:                      # e.g. no C++ compiler on the host
         return {"unavailable": f"{type(e).__name__}: {e}"}
 
@@ -837,7 +906,10 @@ def main():
     l2_bytes = torch.cuda.get_device_properties(local).L2_cache_size
 
     if args.only == "prefill":
-        print(json.dumps(run_prefill(args, bf16_tflops, peak_kind, l2_bytes)), flush=True)
+        i8 = measured_i8_peak()
+        out = run_prefill(args, bf16_tflops, peak_kind, l2_bytes, i8)
+        out["i8_peak"] = i8
+        print(json.dumps(out), flush=True)
         return 0
     if args.only == "stack3b":
         print(json.dumps(run_stack3b(hbm_gbs)), flush=True)
@@ -853,7 +925,14 @@ def main():
     dec = run_decode(args, hbm_gbs, l2_bytes, peak_kind)
     clocks = sampler.stop()
     e2e = None if args.no_e2e else run_e2e(args, dec["probs"], max(3, min(200, args.steps // 10)))
-    pre = None if args.no_prefill else run_prefill(args, bf16_tflops, peak_kind, l2_bytes)
+    try:
+        i8 = measured_i8_peak()
+    except Exception as e:
+        i8 = None
+        i8_err = f"{type(e).__name__}: {e}"
+    pre = None if args.no_prefill else run_prefill(args, bf16_tflops, peak_kind, l2_bytes, i8)
+    if pre is not None:
+        pre["i8_peak"] = i8 if i8 is not None else {"unavailable": i8_err}
     deq = run_dequant(hbm_gbs)
     stack = run_stack3b(hbm_gbs)
     try:
@@ -868,11 +947,12 @@ def main():
         cpu["per_workload"] = oracle_workloads_baseline()
         pack["cpu_oracle"] = oracle_pack_baseline()
     try:
-        ffn = run_ffn100b(hbm_gbs, bf16_tflops * INT8_OVER_BF16)
+        ffn = run_ffn100b(hbm_gbs, i8["tops"] if i8 else bf16_tflops * INT8_OVER_BF16)
     except Exception as e:
         ffn = {"unavailable": f"{type(e).__name__}: {e}"}
     try:
-        stack_pre = run_stack3b(hbm_gbs, M=2048, reps=5, int8_tops=bf16_tflops * INT8_OVER_BF16)
+        stack_pre = run_stack3b(hbm_gbs, M=2048, reps=5,
+                                int8_tops=i8["tops"] if i8 else bf16_tflops * INT8_OVER_BF16)
     except Exception as e:
         stack_pre = {"unavailable": f"{type(e).__name__}: {e}"}
 

@@ -61,6 +61,7 @@ _SIGS = {
                                                  _c_p, _c_sz, _c_p]),
     "bitlinear_epilogue_sum": (ctypes.c_int, [_c_p, ctypes.c_int, _c_i64, _c_i64, _c_p, _c_p, _c_p, _c_p, _c_p,
                                               ctypes.c_uint, _c_p]),
+    "bitlinear_measure_i8_peak": (ctypes.c_int, [ctypes.c_int, _c_p, _c_p, _c_sz, _c_p]),
 }
 
 _lib = None
@@ -512,3 +513,30 @@ def bitlinear_epilogue_sum(partials, absmax: torch.Tensor, w_scale: torch.Tensor
     _check(lib().bitlinear_epilogue_sum(arr, len(parts), M, N, _ptr(absmax), _ptr(w_scale), _ptr(bias), _ptr(y),
                                         _ptr(acc_out), flags, _stream(dev)), "bitlinear_epilogue_sum")
     return y
+
+
+def measure_i8_peak(iters: int = 20000, reps: int = 3, device=None) -> dict:
+    """The dense int8 tensor-core rate, timed with CUDA events on the current
+    stream (best of ``reps`` launches after one warm-up): int8 TOPS and
+    MAC/clock/SM at the given SM clock is left to the caller."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    grid = ctypes.c_int(0)
+    call = lambda: _check(lib().bitlinear_measure_i8_peak(iters, ctypes.byref(grid), _ptr(ws), ws.numel(),
+                                                          _stream(dev)), "bitlinear_measure_i8_peak")
+    call()
+    torch.cuda.synchronize(dev)
+    best = None
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        call()
+        e1.record()
+        e1.synchronize()
+        ms = e0.elapsed_time(e1)
+        best = ms if best is None else min(best, ms)
+    if bitlinear_check_status(ws) != 0:
+        raise BitLinearError(-6, "bitlinear_measure_i8_peak")
+    ops = 2.0 * 128 * 256 * 32 * 4 * iters * grid.value
+    return {"tops": ops / (best * 1e-3) / 1e12, "ms": best, "iters": iters, "grid": grid.value,
+            "macs_per_sm": ops / 2 / grid.value}

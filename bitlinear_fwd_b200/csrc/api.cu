@@ -606,6 +606,19 @@ int bitlinear_epilogue_sum(const int32_t* const* partials, int nparts, int64_t M
   return status_of(launch_epilogue(a, sms, static_cast<cudaStream_t>(stream)));
 }
 
+int bitlinear_measure_i8_peak(int iters, int* grid, void* ws, size_t ws_bytes, void* stream) {
+  if (iters < 1 || iters > (1 << 24)) return BITLINEAR_ERR_SHAPE;
+  if (!grid) return BITLINEAR_ERR_NULL;
+  if (!ws || ws_bytes < 256) return BITLINEAR_ERR_WORKSPACE;
+  if (misaligned(ws)) return BITLINEAR_ERR_ALIGN;
+  int sms = 148;
+  int st = check_device(&sms);
+  if (st != BITLINEAR_OK) return st;
+  *grid = sms;
+  if (cudaMemsetAsync(ws, 0, 4, static_cast<cudaStream_t>(stream)) != cudaSuccess) return BITLINEAR_ERR_CUDA;
+  return status_of(launch_tc_i8_peak(iters, sms, static_cast<uint32_t*>(ws), static_cast<cudaStream_t>(stream)));
+}
+
 int bitlinear_test_force_timeout(int on) {
   return g_force_timeout.exchange(on ? 1 : 0);
 }

@@ -6,63 +6,80 @@
 // The weights are the MMA's A operand and come from tensor memory; the
 // tokens are the B operand and come from shared memory:
 //   D[weight row n][token m] += A[n][k] * B[m][k],  M_mma = 128 weight rows,
-//   N_mma = 128 tokens, K = 32 per instruction.
-// Persistent kernel: one CTA per SM walks the 128 x 128 tiles
-// (weight tile fastest, so the CTAs running at the same time share the
-// token tile in L2), k-blocks of 128, with a 6-stage operand ring and a
-// double-buffered accumulator in tensor memory:
-//   warp 0       TMA producer: x tile (128 tokens x 128 int8, 128-byte
+//   N_mma = BT = 192 tokens, K = 32 per instruction.
+// Tile shape.  Per 128-k block the shared memory of an SM carries the x tile
+// twice (written by TMA, read by the MMA) plus the 2-bit codes; with 192
+// tokens that is 56 KB against 384 cycles of MMA, where 128 tokens would be
+// 40 KB against 256 cycles: the wider tile moves fewer bytes per MMA cycle.
+// Tensor memory holds two 192-column accumulators (the epilogue of one tile
+// runs while the MMAs of the next one fill the other) and four 32-column
+// stages of unpacked weights: 512 columns.
+// Persistent kernel: one CTA per SM walks the 128 x 192 tiles (weight tile
+// fastest, so the CTAs running at the same time share the token tile in L2),
+// k-blocks of 128, with a 6-stage operand ring in shared memory:
+//   warp 0       TMA producer: x tile (192 tokens x 128 int8, 128-byte
 //                swizzle) + packed weight tile (128 rows x 32 bytes) per stage
 //   warp 1       MMA issuer: 4 x tcgen05.mma.kind::i8 per k-block, A from
-//                tensor memory, into accumulator buffer (tile & 1)
+//                tensor-memory stage (k-block & 3), into accumulator buffer
+//                (tile & 1); commits free the shared stage and the A stage
 //   warp 2       tensor-memory allocation
 //   warps 4..7   weight unpack: thread = weight row; its 32 packed bytes become
 //                32 registers of codes c = u + 1 (one word -> four registers
-//                of four consecutive k) and one tcgen05.st of 32 columns
+//                of four consecutive k) and one tcgen05.st of 32 columns; a
+//                quarter-warp reads its 16-byte pieces in an order that keeps
+//                them in distinct banks
 //   warps 8..15  epilogue of the previous tile while the MMAs of the next one
 //                run; warps w and w + 4 share a lane quarter of tensor memory
 //                and take one half of the tile's tokens each: tcgen05.ld of a
-//                row's 64 accumulators, acc - sum_k q (code offset),
-//                y = acc / (s_x s_w) (+ bias), bf16 stores (coalesced along
-//                weight rows); s_w is the scale of the row's group (stacked
-//                layers)
-// Barriers: per stage full (TMA bytes landed), ready (A stage written),
-// empty (MMAs done); per accumulator buffer acc_full (tile's MMAs done) and
-// acc_empty (epilogue has read it).  Shared memory carries only x and the
-// 2-bit codes.  Out-of-range rows/columns are zero-filled by TMA, so a code
-// 0 or an activation 0 adds nothing; the epilogue masks rows >= N and
-// tokens >= M.  Every wait is bounded in time; a wait that gives up sets the
-// status word, and the CTA drains its copies and MMAs before freeing tensor
-// memory.
+//                row's 96 accumulators (the next 32 columns load while 32 are
+//                processed), acc - sum_k q (code offset), y = acc / (s_x s_w)
+//                (+ bias), bf16 stores (coalesced along weight rows); s_w is
+//                the scale of the row's group (stacked layers)
+// Barriers: per shared stage full (TMA bytes landed) and empty (MMAs done);
+// per A stage ready (written) and afree (MMAs done); per accumulator buffer
+// acc_full (tile's MMAs done) and acc_empty (epilogue has read it).
+// Out-of-range rows/columns are zero-filled by TMA, so a code 0 or an
+// activation 0 adds nothing; the epilogue masks rows >= N and tokens >= M.
+// Every wait is bounded in time; a wait that gives up sets the status word,
+// and the CTA drains its copies and MMAs (with the fixed 1 s limit) before
+// freeing tensor memory.
 #include "kernels.h"
 
 namespace bitlinear {
 
 namespace {
 
+#ifndef BITLINEAR_GEMM_BT
+#define BITLINEAR_GEMM_BT 192
+#endif
 constexpr int BW = 128;                      // weight rows per tile (MMA M)
-constexpr int BT = 128;                      // tokens per tile (MMA N)
+constexpr int BT = BITLINEAR_GEMM_BT;        // tokens per tile (MMA N)
 constexpr int BK = 128;                      // k per block
-constexpr int STAGES = 6;
+constexpr int STAGES = 6;                    // shared-memory operand stages
+constexpr int ASTAGES = 4;                   // tensor-memory stages of unpacked weights
 constexpr int kThreads = 512;
-constexpr int kEpiWarps = 8;                // two per tensor-memory lane quarter
-constexpr int kEpiCols = BT / 2;            // tokens of a tile per epilogue warp
-constexpr uint32_t kXBytes = BT * BK;        // 16 KB x tile per stage
+constexpr int kEpiWarps = 8;                 // two per tensor-memory lane quarter
+constexpr int kEpiCols = BT / 2;             // tokens of a tile per epilogue warp
+constexpr int kEpiChunks = kEpiCols / 32;
+constexpr uint32_t kXBytes = BT * BK;        // x tile per stage
 constexpr uint32_t kWpBytes = BW * BK / 4;   // 4 KB packed weights per stage
 constexpr uint32_t kACols = BK / 4;          // tensor-memory columns of one A stage
-constexpr uint32_t kTmemCols = 512;          // 2 x 128 accumulator + 6 x 32 A
+constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kCodeMask = 0x03030303u;
+static_assert(BT % 64 == 0 && BT <= 256, "two halves of whole 32-column chunks; MMA N <= 256");
+static_assert(2 * BT + ASTAGES * kACols <= kTmemCols, "two accumulators and the A stages fit in tensor memory");
 
 constexpr uint32_t kOffX = 0;
 constexpr uint32_t kOffWp = kOffX + STAGES * kXBytes;
 constexpr uint32_t kOffD = kOffWp + STAGES * kWpBytes;       // s_x per token [BT]
 constexpr uint32_t kOffRs = kOffD + 4 * BT;                  // row sums per token [BT]
 constexpr uint32_t kOffBar = kOffRs + 4 * BT;
-constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;        // + barriers, alignment slack
+constexpr uint32_t kSmemBytes = kOffBar + 512 + 1024;        // + barriers, alignment slack
 // tcgen05.alloc of all 512 columns waits until the columns are free, with no
 // time limit.  It never waits here because two CTAs of this kernel cannot
 // share an SM (their shared memory exceeds the SM's 228 KB), and no other
-// kernel of the library uses tensor memory.
+// kernel of the library allocates tensor memory beside it (the int8 rate
+// measurement runs on its own).
 static_assert(2 * kSmemBytes > 228 * 1024, "one GEMM CTA per SM keeps the 512-column allocation uncontended");
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -71,18 +88,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kOffBar);
-  uint64_t* ready = full + STAGES;
-  uint64_t* empty = ready + STAGES;
-  uint64_t* acc_full = empty + STAGES;        // [2]
+  uint64_t* empty = full + STAGES;
+  uint64_t* ready = empty + STAGES;           // [ASTAGES]
+  uint64_t* afree = ready + ASTAGES;          // [ASTAGES]
+  uint64_t* acc_full = afree + ASTAGES;       // [2]
   uint64_t* acc_empty = acc_full + 2;         // [2]
   uint64_t* drain = acc_empty + 2;            // every issued MMA has completed
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* stall_bar = drain + 1;            // never signalled (test hook)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(stall_bar + 1);
   volatile int* failed = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* drain_bad = failed + 1;       // a drain gave up: MMAs may still run
-  uint64_t* stall_bar = reinterpret_cast<uint64_t*>(smem + kOffBar + 224);   // never signalled (test hook)
-  const uint64_t wait_ns = a.wait_ns;
   float* d_s = reinterpret_cast<float*>(smem + kOffD);
   int* rs_s = reinterpret_cast<int*>(smem + kOffRs);
+  const uint64_t wait_ns = a.wait_ns;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int num_kb = (a.K + BK - 1) / BK;
@@ -92,8 +110,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&ready[s], 4);
       mbar_init(&empty[s], 1);
+    }
+    for (int s = 0; s < ASTAGES; ++s) {
+      mbar_init(&ready[s], 4);
+      mbar_init(&afree[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
@@ -169,8 +190,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t tmem_d = tmem_base + b * BT;
         for (int kb = 0; kb < num_kb; ++kb, ++g) {
-          const int s = g % STAGES;
-          if (!mbar_wait(&ready[s], (g / STAGES) & 1, wait_ns)) {
+          const int s = g % STAGES, as = g % ASTAGES;
+          // the A stage is written, which also means the x stage has landed
+          if (!mbar_wait(&ready[as], (g / ASTAGES) & 1, wait_ns)) {
             *failed = 1;
             break;
           }
@@ -178,9 +200,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t x_addr = smem_u32(smem + kOffX + s * kXBytes);
 #pragma unroll
           for (int jj = 0; jj < BK / 32; ++jj)
-            umma_i8_ts(tmem_d, tmem_a + s * kACols + 8 * jj, umma_desc_sw128(x_addr + 32 * jj), idesc,
+            umma_i8_ts(tmem_d, tmem_a + as * kACols + 8 * jj, umma_desc_sw128(x_addr + 32 * jj), idesc,
                        (kb | jj) != 0);
-          umma_commit(&empty[s]);
+          umma_commit(&empty[s]);                 // the shared stage can be refilled
+          umma_commit(&afree[as]);                // the A stage can be rewritten
         }
         if (*failed) break;
         umma_commit(&acc_full[b]);                // the tile's accumulator is complete
@@ -198,16 +221,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;
     const int row = 32 * q + lane;
     const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
+    // lanes 4..7 of every quarter-warp read their second 16-byte piece first:
+    // rows are 32 bytes apart, so the eight pieces of one access then fall in
+    // eight different 4-bank groups
+    const int first = (lane >> 2) & 1;
     int g = 0;
     for (int tile = blockIdx.x; tile < ntiles && !*failed; tile += gridDim.x) {
       for (int kb = 0; kb < num_kb; ++kb, ++g) {
-        const int s = g % STAGES;
-        if (!mbar_wait(&full[s], (g / STAGES) & 1, wait_ns)) {
+        const int s = g % STAGES, as = g % ASTAGES;
+        bool ok = mbar_wait(&full[s], (g / STAGES) & 1, wait_ns);
+        if (ok && g >= ASTAGES) ok = mbar_wait(&afree[as], ((g / ASTAGES) - 1) & 1, wait_ns);
+        if (!ok) {
           *failed = 1;
           break;
         }
         const uint4* wp = reinterpret_cast<const uint4*>(smem + kOffWp + s * kWpBytes + row * 32);
-        const uint4 p0 = wp[0], p1 = wp[1];
+        const uint4 pa = wp[first], pb = wp[first ^ 1];
+        const uint4 p0 = first ? pb : pa, p1 = first ? pa : pb;
         const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
         uint32_t codes[32];
 #pragma unroll
@@ -217,11 +247,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           codes[4 * jj + 2] = (w[jj] >> 4) & kCodeMask;
           codes[4 * jj + 3] = (w[jj] >> 6) & kCodeMask;
         }
-        tmem_st_32x32b_x32(tmem_a + lane_base + s * kACols, codes);
+        tc_fence_after();
+        tmem_st_32x32b_x32(tmem_a + lane_base + as * kACols, codes);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&ready[s]);
+        if (lane == 0) mbar_arrive(&ready[as]);
       }
     }
   } else if (warp >= 8) {
@@ -268,24 +299,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int g = 1; g < kMaxGroups; ++g)
         if (g < a.ngroups && n >= a.group_end[g - 1]) s_w = swg[g];
       if (a.faithful) s_w = bf16_round(s_w);       // a bf16 module holds s_w in bf16
-#pragma unroll 1
-      for (int c = half * (kEpiCols / 32); c < (half + 1) * (kEpiCols / 32); ++c) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tmem_base + b * BT + lane_base + 32 * c, r);
-        tmem_wait_ld();
-        if (c == (half + 1) * (kEpiCols / 32) - 1) {
-          // the whole accumulator is in registers: hand the buffer back
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[b]);
-        }
-        if (!nv) continue;
-        auto emit = [&](int mi, int accv, float y32) {
-          const size_t o = static_cast<size_t>(m0 + mi) * a.N + n;
-          if (a.y) a.y[o] = f32_to_bf16_bits(y32);
-          if (a.acc_out) a.acc_out[o] = accv;
-          if (a.y32_out) a.y32_out[o] = y32;
-        };
+      auto emit = [&](int mi, int accv, float y32) {
+        const size_t o = static_cast<size_t>(m0 + mi) * a.N + n;
+        if (a.y) a.y[o] = f32_to_bf16_bits(y32);
+        if (a.acc_out) a.acc_out[o] = accv;
+        if (a.y32_out) a.y32_out[o] = y32;
+      };
+      auto process = [&](const uint32_t (&r)[32], int c) {
+        if (!nv) return;
         if (simple) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
@@ -319,6 +340,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             emit(mi, accv, y32);
           }
         }
+      };
+      // the next 32 columns load while the current ones are processed; once
+      // the last load has landed the whole accumulator half is in registers
+      // and the buffer goes back to the MMA warp
+      const uint32_t col0 = tmem_base + b * BT + lane_base + 32 * (half * kEpiChunks);
+      uint32_t r0[32], r1[32];
+      tmem_ld_32x32b_x32(col0, r0);
+      tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < kEpiChunks; ++c) {
+        const bool last = c + 1 == kEpiChunks;
+        if (!last) tmem_ld_32x32b_x32(col0 + 32 * (c + 1), (c & 1) ? r0 : r1);
+        if (last) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[b]);
+        }
+        process((c & 1) ? r1 : r0, half * kEpiChunks + c);
+        if (!last) tmem_wait_ld();
       }
     }
   }

@@ -6,34 +6,40 @@
 //
 // Work split.  The N weight rows form 16-row units; the grid is one wave of
 // CTAs (at most one per SM) and CTA c owns a contiguous, balanced range of
-// units over the whole of K.  CTAs never talk to each other.
+// units over the whole of K.  CTAs never talk to each other.  K is cut into
+// 512-k chunks (the last one maybe partial), and the chunks into rounds of
+// eight (4096 k: the x of one round sits in shared memory as int8).
 //
-// Inside a CTA (8 consumer warps + 1 producer warp):
-//   * The producer thread streams the CTA's weights through a shared-memory
-//     ring with TMA and full/empty mbarriers, one load per (4096-k round,
-//     unit): a 3-D box of up to 8 sub-boxes of 16 rows x 128 bytes (512 k
-//     each, 128-byte swizzle), so each TMA instruction moves 16 KB (per-SM
-//     TMA throughput on B200 is set by the number of loads more than by their
-//     size), plus a 2-D box for a last 512-k chunk that K only partly fills
-//     (the 3-D view cannot bound it).  When the weights are resident it starts
-//     before the wait on the previous kernel of the stream, so the stream
-//     overlaps that kernel's tail.
-//   * The consumer warps form each token's absmax over the row, s_x =
-//     127 / max(absmax, 1e-5) in float32, and q = round_half_even(x s_x) as
-//     int8 into shared memory, one 4096-k round at a time, with the sum of q
+// Inside a CTA every one of the 8 warps streams and computes:
+//   * The CTA's work of a round is a list of items (chunk group, unit), chunk
+//     group outer: a group is kc consecutive full chunks of one unit, loaded
+//     by one TMA instruction as a 3-D box of kc sub-boxes of 16 rows x 128
+//     bytes (128-byte swizzle); a partial last chunk is an item of its own,
+//     loaded through a 2-D view that K bounds (zero fill beyond K).  Warp w
+//     takes items w, w + 8, ... of every round, so the warps' shares differ
+//     by at most one item.
+//   * Each warp streams its own items through its own ring of shared-memory
+//     slots: its lane 0 issues the TMA loads up to `ring` items ahead and
+//     refills a slot as soon as the warp has read it; the warp waits on the
+//     slot's mbarrier.  No warp ever waits for another warp's loads, so TMA
+//     issue is spread over all 8 warps.  When the weights are resident the
+//     first loads are issued before the wait on the previous kernel of the
+//     stream, so the stream overlaps that kernel's tail.
+//   * Before the items, all warps form each token's absmax over the row,
+//     s_x = 127 / max(absmax, 1e-5) in float32, and q = round_half_even(x
+//     s_x) as int8 into shared memory, one round at a time, with the sum of q
 //     per token.  For M <= 4 and K <= 4096 each lane's share of x is read
 //     once and held in registers between the two steps; otherwise x is read
 //     again for the quantising step.  Pre-quantised int8 input is copied in
 //     instead.
-//   * In round r warp w takes sub-box w (k = 4096r + 512w ..) of every unit
-//     of the CTA, so it loads its x fragment once per round and reuses it for
-//     all units.  Per sub-box a thread
-//     takes one 16-byte vector of two weight rows and issues mma.sync
-//     m16n8k32 (weights as A, u8; tokens as B, s8; a second 8-token tile for
-//     M > 8).  The codes c = u + 1 enter unshifted: A_i = word &
-//     (0x03030303 << 2i) holds 4^i c per byte lane, so field i accumulates
-//     4^i sum(c q); the fields are combined with exact shifts and added to the
-//     unit's int32 sums in shared memory.
+//   * Per chunk of an item, a thread takes one 16-byte vector of two weight
+//     rows and issues mma.sync m16n8k32 (weights as A, u8; tokens as B, s8;
+//     a second 8-token tile for M > 8).  The codes c = u + 1 enter
+//     unshifted: A_i = word & (0x03030303 << 2i) holds 4^i c per byte lane,
+//     so field i accumulates 4^i sum(c q); the fields are combined with
+//     exact shifts and added to the unit's int32 sums in shared memory.  The
+//     x fragment of a chunk stays in registers while consecutive items share
+//     the chunk.
 //   * Epilogue: acc = sum(c q) - sum(q) = sum(u q); y = acc / (s_x s_w)
 //     (+ bias) -> bf16, with s_w the scale of the row's layer when several
 //     layers are stacked.  The bf16-faithful mode rounds the scale, the
@@ -54,15 +60,15 @@ namespace bitlinear {
 
 namespace {
 
-constexpr int kConsumerWarps = 8;
-constexpr int kThreads = 32 * (kConsumerWarps + 1);   // + one producer warp
-constexpr int kConsumerThreads = 32 * kConsumerWarps;
+constexpr int kWarps = 8;
+constexpr int kThreads = 32 * kWarps;
 constexpr int kUnitRows = 16;
-constexpr int kBoxK = 512;                            // k per sub-box
+constexpr int kBoxK = 512;                            // k per chunk (sub-box)
 constexpr int kSubBytes = kUnitRows * kBoxK / 4;      // 2 KB
-constexpr int kChunkK = kConsumerWarps * kBoxK;       // k per round (one sub-box per warp)
-constexpr int kMaxRing = 16;
-constexpr int kMaxUnits = 16;                         // units per CTA
+constexpr int kRoundChunks = 8;                       // chunks per x round
+constexpr int kChunkK = kRoundChunks * kBoxK;         // k per round
+constexpr int kMaxRing = 8;                           // slots per warp
+constexpr int kMaxUnits = 32;                         // units per CTA
 constexpr int kXB = 8;                                // bf16 x loads in flight per lane (absmax)
 constexpr int kQB = 2;                                // the same in the quantising pass
 constexpr int kHold = 4;                              // 32-byte x chunks per lane and token held in
@@ -77,11 +83,6 @@ __device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, 
       "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
       : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-// Barrier among the consumer warps only (the producer warp is busy).
-__device__ __forceinline__ void consumer_sync() {
-  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads) : "memory");
 }
 
 __device__ __forceinline__ void red_shared_add(int* p, int v) {
@@ -156,14 +157,12 @@ __device__ __forceinline__ int bytesum16(uint4 v, int sum) {
 }
 
 struct SmemTail {
-  uint64_t full[kMaxRing];
-  uint64_t empty[kMaxRing];
+  uint64_t full[kWarps][kMaxRing];   // per warp: its ring slots' TMA barriers
   uint64_t stall;                    // never signalled (forced-timeout test hook)
   uint32_t amax[16];                 // absmax per token (bf16 bits)
   int rsum[16];                      // sum of q per token
   float sx[16];                      // s_x per token
   float swg[kMaxGroups];             // s_w of each row group
-  int issued;                        // loads issued (producer)
   int failed;                        // a wait of this CTA timed out
 };
 
@@ -171,19 +170,51 @@ struct SmemLayout {
   size_t ring, xs, acc, bias, tail, total;
 };
 
-// ring slots of slot_bytes (1024-aligned base), x rows of one round for the
-// M tokens, per-unit int32 sums [unit][row][8 * token tiles], bias, tail
+// 8 warps' rings of `ring` slots of slot_bytes (1024-aligned base), x rows of
+// one round for the M tokens, per-unit int32 sums [unit][row][8 * token
+// tiles], bias, tail
 __host__ __device__ SmemLayout smem_layout(int M, int ring, size_t slot_bytes, int units) {
   const int ntok = M <= 8 ? 8 : 16;
   SmemLayout L;
   L.ring = 0;
-  L.xs = L.ring + static_cast<size_t>(ring) * slot_bytes;
+  L.xs = L.ring + static_cast<size_t>(kWarps) * ring * slot_bytes;
   L.acc = L.xs + static_cast<size_t>(M) * (kChunkK + 16);
   L.bias = L.acc + static_cast<size_t>(units) * kUnitRows * ntok * 4;
   L.tail = (L.bias + static_cast<size_t>(units) * kUnitRows * 2 + 15) & ~size_t(15);
   L.total = 1024 + L.tail + sizeof(SmemTail);
   return L;
 }
+
+// The items of one warp, in order: round r, item j of the round (j = warp,
+// warp + 8, ...); item j is chunk group j / U of unit j % U.  A round's
+// groups are its full chunks in groups of kc (the last one maybe short: the
+// 3-D view zero-fills chunks >= F) and, in the round that holds it, the
+// partial last chunk as a group of its own.
+struct ItemCursor {
+  int r, j;
+  __device__ __forceinline__ static int full_groups(int r, int F, int kc) {
+    const int fc = min(max(F - kRoundChunks * r, 0), kRoundChunks);
+    return (fc + kc - 1) / kc;
+  }
+  __device__ __forceinline__ static int groups(int r, int F, int kc, int tail) {
+    return full_groups(r, F, kc) + ((tail && F / kRoundChunks == r) ? 1 : 0);
+  }
+  __device__ __forceinline__ void settle(int warp, int nround, int F, int kc, int tail, int U) {
+    while (r < nround && j >= groups(r, F, kc, tail) * U) {
+      ++r;
+      j = warp;
+    }
+  }
+  __device__ __forceinline__ void start(int warp, int nround, int F, int kc, int tail, int U) {
+    r = 0;
+    j = warp;
+    settle(warp, nround, F, kc, tail, U);
+  }
+  __device__ __forceinline__ void next(int warp, int nround, int F, int kc, int tail, int U) {
+    j += kWarps;
+    settle(warp, nround, F, kc, tail, U);
+  }
+};
 
 template <int NT>
 __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
@@ -193,10 +224,9 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   const int ring = a.ring;
-  const int kc = a.kc;                               // sub-boxes per 3-D load (0 when K < 512)
-  const size_t slot_bytes = static_cast<size_t>(kc + a.tail) * kSubBytes;
+  const int kc = a.kc;                               // chunks per 3-D item
+  const size_t slot_bytes = static_cast<size_t>(kc) * kSubBytes;
   const SmemLayout L = smem_layout(a.M, ring, slot_bytes, a.units_max);
-  uint8_t* rbuf = base + L.ring;
   int8_t* xs = reinterpret_cast<int8_t*>(base + L.xs);
   int* acc_s = reinterpret_cast<int*>(base + L.acc);            // [unit][row][token]
   uint16_t* bias_s = reinterpret_cast<uint16_t*>(base + L.bias);
@@ -210,332 +240,336 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
   const int units_total = (N + kUnitRows - 1) / kUnitRows;
   const int u_begin = static_cast<int>(static_cast<long long>(blockIdx.x) * units_total / gridDim.x);
   const int U = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * units_total / gridDim.x) - u_begin;
-  const int nbox = (K + kBoxK - 1) / kBoxK;          // 512-k chunks, the last maybe partial
   const int F = K / kBoxK;                           // full 512-k chunks (the 3-D view's extent)
+  const int tail = (K % kBoxK) != 0;                 // a partial last chunk
   const int nround = (K + kChunkK - 1) / kChunkK;
+  uint8_t* wring = base + L.ring + static_cast<size_t>(warp) * ring * slot_bytes;   // this warp's ring
+  uint64_t* full = sm.full[warp];
 
+  if (lane == 0)
+    for (int s = 0; s < ring; ++s) mbar_init(&full[s], 1);
   if (threadIdx.x == 0) {
-    for (int s = 0; s < ring; ++s) {
-      mbar_init(&sm.full[s], 1);
-      mbar_init(&sm.empty[s], kConsumerWarps);
-    }
     mbar_init(&sm.stall, 1);
-    fence_mbar_init();
-    if (kc > 0) tma_prefetch_desc(&tm3);
-    if (a.tail) tma_prefetch_desc(&tm2);
+    if (F > 0) tma_prefetch_desc(&tm3);
+    if (tail) tma_prefetch_desc(&tm2);
+    sm.failed = 0;
   }
+  fence_mbar_init();
   if (threadIdx.x < 16) {
     sm.amax[threadIdx.x] = 0u;
     sm.rsum[threadIdx.x] = 0;
   }
-  if (threadIdx.x == 0) {
-    sm.issued = 0;
-    sm.failed = 0;
-  }
   for (int i = threadIdx.x; i < U * kUnitRows * NTOK; i += kThreads) acc_s[i] = 0;
   __syncthreads();
 
-  bool ok = true;
-  if (warp == kConsumerWarps) {
-    // ======================= producer warp =======================
-    if (!a.weights_early) pdl_wait_primary();
-    for (int i = lane; i < U * kUnitRows; i += 32) {
-      const int n = u_begin * kUnitRows + i;
-      bias_s[i] = (a.bias && n < N) ? a.bias[n] : static_cast<uint16_t>(0);
-    }
-    if (lane < a.ngroups) sm.swg[lane] = a.w_scale[lane];
+  // ---- this warp's weight stream (lane 0 issues; every lane keeps the count)
+  ItemCursor ic;                                     // next item to issue
+  ic.start(warp, nround, F, kc, tail, U);
+  int issued = 0;
+  auto issue_next = [&]() {
+    if (ic.r >= nround) return;
     if (lane == 0) {
-      int q = 0;
-      for (int r = 0; r < nround && ok; ++r) {
-        const bool has3 = kc > 0 && 8 * r < F;       // full chunks of this round, one 3-D load
-        const bool hast = a.tail && (F >> 3) == r;   // the partial chunk, one 2-D load
-        const uint32_t bytes = (has3 ? kc * kSubBytes : 0) + (hast ? kSubBytes : 0);
-        for (int u = 0; u < U; ++u, ++q) {
-          const int s = q % ring;
-          if (q >= ring && !mbar_wait(&sm.empty[s], ((q / ring) - 1) & 1, a.wait_ns)) {
-            ok = false;
-            break;
-          }
-          uint8_t* dst = rbuf + s * slot_bytes;
-          const int row = (u_begin + u) * kUnitRows;
-          mbar_arrive_expect_tx(&sm.full[s], bytes);
-          if (has3) tma_load_3d(dst, &tm3, &sm.full[s], 0, row, 8 * r);
-          if (hast) tma_load_2d(dst + kc * kSubBytes, &tm2, &sm.full[s], F * (kBoxK / 4), row);
-        }
+      const int s = issued % ring;
+      const int g = ic.j / U, u = ic.j - g * U;
+      const int row = (u_begin + u) * kUnitRows;
+      uint8_t* dst = wring + s * slot_bytes;
+      if (g < ItemCursor::full_groups(ic.r, F, kc)) {
+        mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(kc * kSubBytes));
+        tma_load_3d(dst, &tm3, &full[s], 0, row, kRoundChunks * ic.r + g * kc);
+      } else {
+        mbar_arrive_expect_tx(&full[s], kSubBytes);
+        tma_load_2d(dst, &tm2, &full[s], F * (kBoxK / 4), row);
       }
-      sm.issued = q;
     }
-    __syncwarp();
+    ++issued;
+    ic.next(warp, nround, F, kc, tail, U);
+  };
+  if (a.weights_early)
+    for (int i = 0; i < ring; ++i) issue_next();
+
+  pdl_wait_primary();
+  if (!a.weights_early)
+    for (int i = 0; i < ring; ++i) issue_next();
+  if (a.status && blockIdx.x == 0 && threadIdx.x == 0) *a.status = 0u;
+  for (int i = threadIdx.x; i < U * kUnitRows; i += kThreads) {
+    const int n = u_begin * kUnitRows + i;
+    bias_s[i] = (a.bias && n < N) ? a.bias[n] : static_cast<uint16_t>(0);
+  }
+  if (threadIdx.x < a.ngroups) sm.swg[threadIdx.x] = a.w_scale[threadIdx.x];
+
+  bool ok = true;
+  const int g = lane >> 2, t = lane & 3;
+
+  // ---- per-token absmax over the whole row: warp w takes token(s)
+  // m = w / P (+ 8 / P, ...) and a 1/P share of the row, P = max(1, 8 / M)
+  const int cpr = K >> 4;                            // 16-element chunks per row
+  const int P = M >= kWarps ? 1 : kWarps / M;
+  const int part = warp % P, mstep = kWarps / P;
+  const int C = (cpr + 32 * P - 1) / (32 * P);       // chunks per lane per token
+  // One pass over x when the row is one round and this lane's share fits in
+  // registers: the values loaded for the absmax are quantised in place.
+  const bool single = NT == 1 && a.x && nround == 1 && C <= kHold;
+  if (single) {
+    const uint4* xrow0 = reinterpret_cast<const uint4*>(a.x);
+    uint4 v[kHold * NT][2];
+#pragma unroll
+    for (int i = 0; i < kHold * NT; ++i) {
+      const int j = (NT == 2 && i >= C) ? 1 : 0;     // token slot of this warp
+      const int m = warp / P + j * mstep;
+      const int ch = part * 32 + lane + (i - j * C) * 32 * P;
+      v[i][0] = v[i][1] = make_uint4(0, 0, 0, 0);
+      if (i < NT * C && m < M && ch < cpr) {
+        v[i][0] = __ldg(xrow0 + (static_cast<size_t>(m) * K >> 3) + 2 * ch);
+        v[i][1] = __ldg(xrow0 + (static_cast<size_t>(m) * K >> 3) + 2 * ch + 1);
+      }
+    }
+    uint32_t mx[NT];
+#pragma unroll
+    for (int j = 0; j < NT; ++j) mx[j] = 0;
+#pragma unroll
+    for (int i = 0; i < kHold * NT; ++i) {
+      const uint32_t am = absmax16_bits(v[i][0], v[i][1]);   // zeros where nothing was loaded
+      if (NT == 2 && i >= C) mx[NT - 1] = max(mx[NT - 1], am);
+      else mx[0] = max(mx[0], am);
+    }
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      const int m = warp / P + j * mstep;
+      const uint32_t r = __reduce_max_sync(0xffffffffu, mx[j]);
+      if (lane == 0 && m < M) atomicMax(&sm.amax[m], r);
+    }
+    __syncthreads();
+    float sxr[NT];
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      const int m = min(warp / P + j * mstep, M - 1);
+      sxr[j] = act_scale(bf16_bits_to_f32(sm.amax[m]), a.faithful);
+    }
+    if (threadIdx.x < M) {
+      const float sxv = act_scale(bf16_bits_to_f32(sm.amax[threadIdx.x]), a.faithful);
+      sm.sx[threadIdx.x] = sxv;
+      if (blockIdx.x == 0 && a.sx_out) a.sx_out[threadIdx.x] = sxv;
+    }
+    int sum[NT];
+#pragma unroll
+    for (int j = 0; j < NT; ++j) sum[j] = 0;
+#pragma unroll
+    for (int i = 0; i < kHold * NT; ++i) {
+      const int j = (NT == 2 && i >= C) ? 1 : 0;
+      const int m = warp / P + j * mstep;
+      const int ch = part * 32 + lane + (i - j * C) * 32 * P;
+      if (i < NT * C && m < M && ch < cpr) {
+        int ps = 0;
+        const uint4 qv = quant16(v[i][0], v[i][1], j ? sxr[NT - 1] : sxr[0], ps, a.faithful);
+        if (j) sum[NT - 1] += ps;
+        else sum[0] += ps;
+        *reinterpret_cast<uint4*>(xs + m * S + 16 * xs_chunk(ch)) = qv;
+        if (blockIdx.x == 0 && a.xq_out) *reinterpret_cast<uint4*>(a.xq_out + static_cast<size_t>(m) * K + 16 * ch) = qv;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      const int m = warp / P + j * mstep;
+      const int r = __reduce_add_sync(0xffffffffu, sum[j]);
+      if (lane == 0 && m < M) atomicAdd(&sm.rsum[m], r);
+    }
+  } else if (a.x) {
+    for (int m = warp / P; m < M; m += mstep) {
+      const uint4* row = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(m) * K);
+      uint32_t mx = 0;
+      // kXB 32-byte loads in flight per lane before any is used
+      for (int ch0 = part * 32 + lane; ch0 < cpr; ch0 += 32 * P * kXB) {
+        uint4 v[kXB][2];
+#pragma unroll
+        for (int j = 0; j < kXB; ++j) {
+          const int ch = ch0 + j * 32 * P;
+          v[j][0] = v[j][1] = make_uint4(0, 0, 0, 0);
+          if (ch < cpr) {
+            v[j][0] = __ldg(row + 2 * ch);
+            v[j][1] = __ldg(row + 2 * ch + 1);
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < kXB; ++j) mx = max(mx, absmax16_bits(v[j][0], v[j][1]));
+      }
+      mx = __reduce_max_sync(0xffffffffu, mx);
+      if (lane == 0) atomicMax(&sm.amax[m], mx);
+    }
+    __syncthreads();
+    if (threadIdx.x < M) {
+      const float sxv = act_scale(bf16_bits_to_f32(sm.amax[threadIdx.x]), a.faithful);
+      sm.sx[threadIdx.x] = sxv;
+      if (blockIdx.x == 0 && a.sx_out) a.sx_out[threadIdx.x] = sxv;
+    }
   } else {
-    // ======================= consumer warps =======================
-    pdl_wait_primary();
-    if (a.status && blockIdx.x == 0 && threadIdx.x == 0) *a.status = 0u;
-    const int g = lane >> 2, t = lane & 3;
+    if (threadIdx.x < M) sm.sx[threadIdx.x] = a.s_x[threadIdx.x];
+  }
+  __syncthreads();
 
-    // ---- per-token absmax over the whole row: warp w takes token(s)
-    // m = w / P (+ 8 / P, ...) and a 1/P share of the row, P = max(1, 8 / M)
-    const int cpr = K >> 4;                          // 16-element chunks per row
-    const int P = M >= kConsumerWarps ? 1 : kConsumerWarps / M;
-    const int part = warp % P, mstep = kConsumerWarps / P;
-    const int C = (cpr + 32 * P - 1) / (32 * P);     // chunks per lane per token
-    // One pass over x when the row is one round and this lane's share fits in
-    // registers: the values loaded for the absmax are quantised in place.
-    const bool single = NT == 1 && a.x && nround == 1 && C <= kHold;
-    if (single) {
-      const uint4* xrow0 = reinterpret_cast<const uint4*>(a.x);
-      uint4 v[kHold * NT][2];
+  // forced-timeout test: a wait that nothing completes runs out, and the
+  // CTA takes the same path as after any wait that gives up
+  if (a.stall && !mbar_wait(&sm.stall, 0, a.wait_ns)) ok = false;
+  ok = __all_sync(0xffffffffu, ok);
+
+  const int r0 = mma_row_to_box(g);                  // sub-box rows r0 and r0 + 8
+  ItemCursor cc;                                     // next item to consume
+  cc.start(warp, nround, F, kc, tail, U);
+  int consumed = 0;
+  int xchunk = -1;                                   // round-local chunk of the x fragment held
+  uint32_t xw[2][2][NT][8];                          // [v][pair][token tile][word]
+  for (int r = 0; r < nround; ++r) {
+    const int c0 = r * kChunkK;
+    const int ccpr = min(kChunkK, K - c0) >> 4;      // 16-element chunks of x in this round
+    if (r > 0) __syncthreads();                      // every warp is done with the previous round's x
+    // ---- x round -> int8 in shared memory (tokens < M only)
+    for (int m = warp / P; m < (single ? 0 : M); m += mstep) {
+      int8_t* xrow = xs + m * S;
+      const float sxm = sm.sx[m];
+      int sum = 0;
+      const size_t roff = static_cast<size_t>(m) * K + c0;
+      for (int ch0 = part * 32 + lane; ch0 < ccpr; ch0 += 32 * P * kQB) {
+        if (a.x) {
+          const uint4* src = reinterpret_cast<const uint4*>(a.x + roff);
+          uint4 v[kQB][2];
 #pragma unroll
-      for (int i = 0; i < kHold * NT; ++i) {
-        const int j = (NT == 2 && i >= C) ? 1 : 0;   // token slot of this warp
-        const int m = warp / P + j * mstep;
-        const int ch = part * 32 + lane + (i - j * C) * 32 * P;
-        v[i][0] = v[i][1] = make_uint4(0, 0, 0, 0);
-        if (i < NT * C && m < M && ch < cpr) {
-          v[i][0] = __ldg(xrow0 + (static_cast<size_t>(m) * K >> 3) + 2 * ch);
-          v[i][1] = __ldg(xrow0 + (static_cast<size_t>(m) * K >> 3) + 2 * ch + 1);
-        }
-      }
-      uint32_t mx[NT];
-#pragma unroll
-      for (int j = 0; j < NT; ++j) mx[j] = 0;
-#pragma unroll
-      for (int i = 0; i < kHold * NT; ++i) {
-        const uint32_t am = absmax16_bits(v[i][0], v[i][1]);   // zeros where nothing was loaded
-        if (NT == 2 && i >= C) mx[NT - 1] = max(mx[NT - 1], am);
-        else mx[0] = max(mx[0], am);
-      }
-#pragma unroll
-      for (int j = 0; j < NT; ++j) {
-        const int m = warp / P + j * mstep;
-        const uint32_t r = __reduce_max_sync(0xffffffffu, mx[j]);
-        if (lane == 0 && m < M) atomicMax(&sm.amax[m], r);
-      }
-      consumer_sync();
-      float sxr[NT];
-#pragma unroll
-      for (int j = 0; j < NT; ++j) {
-        const int m = min(warp / P + j * mstep, M - 1);
-        sxr[j] = act_scale(bf16_bits_to_f32(sm.amax[m]), a.faithful);
-      }
-      if (threadIdx.x < M) {
-        const float sxv = act_scale(bf16_bits_to_f32(sm.amax[threadIdx.x]), a.faithful);
-        sm.sx[threadIdx.x] = sxv;
-        if (blockIdx.x == 0 && a.sx_out) a.sx_out[threadIdx.x] = sxv;
-      }
-      int sum[NT];
-#pragma unroll
-      for (int j = 0; j < NT; ++j) sum[j] = 0;
-#pragma unroll
-      for (int i = 0; i < kHold * NT; ++i) {
-        const int j = (NT == 2 && i >= C) ? 1 : 0;
-        const int m = warp / P + j * mstep;
-        const int ch = part * 32 + lane + (i - j * C) * 32 * P;
-        if (i < NT * C && m < M && ch < cpr) {
-          int ps = 0;
-          const uint4 qv = quant16(v[i][0], v[i][1], j ? sxr[NT - 1] : sxr[0], ps, a.faithful);
-          if (j) sum[NT - 1] += ps;
-          else sum[0] += ps;
-          *reinterpret_cast<uint4*>(xs + m * S + 16 * xs_chunk(ch)) = qv;
-          if (blockIdx.x == 0 && a.xq_out) *reinterpret_cast<uint4*>(a.xq_out + static_cast<size_t>(m) * K + 16 * ch) = qv;
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < NT; ++j) {
-        const int m = warp / P + j * mstep;
-        const int r = __reduce_add_sync(0xffffffffu, sum[j]);
-        if (lane == 0 && m < M) atomicAdd(&sm.rsum[m], r);
-      }
-    } else if (a.x) {
-      for (int m = warp / P; m < M; m += mstep) {
-        const uint4* row = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(m) * K);
-        uint32_t mx = 0;
-        // kXB 32-byte loads in flight per lane before any is used
-        for (int ch0 = part * 32 + lane; ch0 < cpr; ch0 += 32 * P * kXB) {
-          uint4 v[kXB][2];
-#pragma unroll
-          for (int j = 0; j < kXB; ++j) {
+          for (int j = 0; j < kQB; ++j) {
             const int ch = ch0 + j * 32 * P;
-            v[j][0] = v[j][1] = make_uint4(0, 0, 0, 0);
-            if (ch < cpr) {
-              v[j][0] = __ldg(row + 2 * ch);
-              v[j][1] = __ldg(row + 2 * ch + 1);
+            if (ch < ccpr) {
+              v[j][0] = __ldg(src + 2 * ch);
+              v[j][1] = __ldg(src + 2 * ch + 1);
             }
           }
 #pragma unroll
-          for (int j = 0; j < kXB; ++j) mx = max(mx, absmax16_bits(v[j][0], v[j][1]));
+          for (int j = 0; j < kQB; ++j) {
+            const int ch = ch0 + j * 32 * P;
+            if (ch < ccpr) {
+              const uint4 qv = quant16(v[j][0], v[j][1], sxm, sum, a.faithful);
+              if (blockIdx.x == 0 && a.xq_out) *reinterpret_cast<uint4*>(a.xq_out + roff + 16 * ch) = qv;
+              *reinterpret_cast<uint4*>(xrow + 16 * xs_chunk(ch)) = qv;
+            }
+          }
+        } else {
+          const uint4* src = reinterpret_cast<const uint4*>(a.xq + roff);
+          uint4 v[kQB];
+#pragma unroll
+          for (int j = 0; j < kQB; ++j) {
+            const int ch = ch0 + j * 32 * P;
+            if (ch < ccpr) v[j] = __ldg(src + ch);
+          }
+#pragma unroll
+          for (int j = 0; j < kQB; ++j) {
+            const int ch = ch0 + j * 32 * P;
+            if (ch < ccpr) {
+              sum = bytesum16(v[j], sum);
+              *reinterpret_cast<uint4*>(xrow + 16 * xs_chunk(ch)) = v[j];
+            }
+          }
         }
-        mx = __reduce_max_sync(0xffffffffu, mx);
-        if (lane == 0) atomicMax(&sm.amax[m], mx);
       }
-      consumer_sync();
-      if (threadIdx.x < M) {
-        const float sxv = act_scale(bf16_bits_to_f32(sm.amax[threadIdx.x]), a.faithful);
-        sm.sx[threadIdx.x] = sxv;
-        if (blockIdx.x == 0 && a.sx_out) a.sx_out[threadIdx.x] = sxv;
-      }
-    } else {
-      if (threadIdx.x < M) sm.sx[threadIdx.x] = a.s_x[threadIdx.x];
+      sum = __reduce_add_sync(0xffffffffu, sum);
+      if (lane == 0) atomicAdd(&sm.rsum[m], sum);
     }
-    consumer_sync();
+    if (!single) __syncthreads();
+    xchunk = -1;
 
-    // forced-timeout test: a wait that nothing completes runs out, and the
-    // CTA takes the same path as after any wait that gives up
-    if (a.stall && !mbar_wait(&sm.stall, 0, a.wait_ns)) ok = false;
-    const int r0 = mma_row_to_box(g);                // sub-box rows r0 and r0 + 8
-    for (int r = 0; r < nround; ++r) {
-      const int c0 = r * kChunkK;
-      const int ccpr = min(kChunkK, K - c0) >> 4;    // 16-element chunks of x in this round
-      if (r > 0) consumer_sync();                    // previous round's fragments are loaded
-      // ---- x round -> int8 in shared memory (tokens < M only)
-      for (int m = warp / P; m < (single ? 0 : M); m += mstep) {
-        int8_t* xrow = xs + m * S;
-        const float sxm = sm.sx[m];
-        int sum = 0;
-        const size_t roff = static_cast<size_t>(m) * K + c0;
-        for (int ch0 = part * 32 + lane; ch0 < ccpr; ch0 += 32 * P * kQB) {
-          if (a.x) {
-            const uint4* src = reinterpret_cast<const uint4*>(a.x + roff);
-            uint4 v[kQB][2];
-#pragma unroll
-            for (int j = 0; j < kQB; ++j) {
-              const int ch = ch0 + j * 32 * P;
-              if (ch < ccpr) {
-                v[j][0] = __ldg(src + 2 * ch);
-                v[j][1] = __ldg(src + 2 * ch + 1);
-              }
-            }
-#pragma unroll
-            for (int j = 0; j < kQB; ++j) {
-              const int ch = ch0 + j * 32 * P;
-              if (ch < ccpr) {
-                const uint4 qv = quant16(v[j][0], v[j][1], sxm, sum, a.faithful);
-                if (blockIdx.x == 0 && a.xq_out) *reinterpret_cast<uint4*>(a.xq_out + roff + 16 * ch) = qv;
-                *reinterpret_cast<uint4*>(xrow + 16 * xs_chunk(ch)) = qv;
-              }
-            }
-          } else {
-            const uint4* src = reinterpret_cast<const uint4*>(a.xq + roff);
-            uint4 v[kQB];
-#pragma unroll
-            for (int j = 0; j < kQB; ++j) {
-              const int ch = ch0 + j * 32 * P;
-              if (ch < ccpr) v[j] = __ldg(src + ch);
-            }
-#pragma unroll
-            for (int j = 0; j < kQB; ++j) {
-              const int ch = ch0 + j * 32 * P;
-              if (ch < ccpr) {
-                sum = bytesum16(v[j], sum);
-                *reinterpret_cast<uint4*>(xrow + 16 * xs_chunk(ch)) = v[j];
-              }
-            }
-          }
-        }
-        sum = __reduce_add_sync(0xffffffffu, sum);
-        if (lane == 0) atomicAdd(&sm.rsum[m], sum);
+    // ---- this warp's items of round r
+    while (ok && cc.r == r) {
+      const int s = consumed % ring;
+      const bool got = mbar_wait(&full[s], (consumed / ring) & 1, a.wait_ns);
+      if (!__all_sync(0xffffffffu, got)) {
+        ok = false;
+        break;
       }
-      if (!single) consumer_sync();
-
-      // ---- contraction: this warp's sub-box of every unit
-      const int nw = min(kConsumerWarps, nbox - 8 * r);
-      const bool mine = warp < nw;
-      const int sub = (a.tail && 8 * r + warp == F) ? kc : warp;   // partial chunk: the 2-D box
-      uint32_t xw[2][2][NT][8];                      // [v][pair][token tile][word]
+      const int grp = cc.j / U, u = cc.j - grp * U;
+      const bool is3 = grp < ItemCursor::full_groups(r, F, kc);
+      const int first = is3 ? grp * kc : F - kRoundChunks * r;   // round-local chunk of the item's first sub-box
+      const int nsub = is3 ? min(kc, F - kRoundChunks * r - grp * kc) : 1;
+      int acc[4][NT][4];
 #pragma unroll
-      for (int v = 0; v < 2; ++v)
+      for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int pr = 0; pr < 2; ++pr)
+        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            const int m = nt * 8 + g;
+          for (int rr = 0; rr < 4; ++rr) acc[i][nt][rr] = 0;
+      for (int sb = 0; sb < nsub; ++sb) {
+        const int lc = first + sb;                   // round-local chunk
+        if (lc != xchunk) {
 #pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-              uint4 xv = make_uint4(0, 0, 0, 0);
-              if (mine && m < M)
-                xv = *reinterpret_cast<const uint4*>(xs + m * S +
-                                                     16 * xs_chunk(32 * warp + 16 * v + 4 * t + 2 * pr + cc));
-              xw[v][pr][nt][4 * cc + 0] = xv.x; xw[v][pr][nt][4 * cc + 1] = xv.y;
-              xw[v][pr][nt][4 * cc + 2] = xv.z; xw[v][pr][nt][4 * cc + 3] = xv.w;
-            }
-          }
-      for (int u = 0; u < U; ++u) {
-        const int q = r * U + u;
-        const int s = q % ring;
-        // every consumer warp waits for every load (also when it has no
-        // sub-box in it): its arrival on the empty barrier must not run ahead
-        // of the slot's phases
-        if (ok && !mbar_wait(&sm.full[s], (q / ring) & 1, a.wait_ns)) ok = false;
-        if (!ok) break;
-        int acc[4][NT][4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int rr = 0; rr < 4; ++rr) acc[i][nt][rr] = 0;
-        if (mine) {
-          const uint8_t* box = rbuf + s * slot_bytes + sub * kSubBytes;
-#pragma unroll
-          for (int v = 0; v < 2; ++v) {
-            const int cw = 4 * v + t;                // 16-byte chunk of the 128-byte row
-            const uint4 wa = *reinterpret_cast<const uint4*>(box + r0 * 128 + ((cw ^ r0) << 4));
-            const uint4 wb = *reinterpret_cast<const uint4*>(box + (r0 + 8) * 128 + ((cw ^ r0) << 4));
-            const uint32_t w0[4] = {wa.x, wa.y, wa.z, wa.w};
-            const uint32_t w1[4] = {wb.x, wb.y, wb.z, wb.w};
+          for (int v = 0; v < 2; ++v)
 #pragma unroll
             for (int pr = 0; pr < 2; ++pr)
 #pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const uint32_t mask = kCodeMask << (2 * i);
-                const uint32_t a0 = w0[2 * pr] & mask, a1 = w1[2 * pr] & mask;
-                const uint32_t a2 = w0[2 * pr + 1] & mask, a3 = w1[2 * pr + 1] & mask;
+              for (int nt = 0; nt < NT; ++nt) {
+                const int m = nt * 8 + g;
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-                  mma_u8s8(acc[i][nt], a0, a1, a2, a3, xw[v][pr][nt][i], xw[v][pr][nt][4 + i]);
+                for (int c2 = 0; c2 < 2; ++c2) {
+                  uint4 xv = make_uint4(0, 0, 0, 0);
+                  if (m < M)
+                    xv = *reinterpret_cast<const uint4*>(xs + m * S +
+                                                         16 * xs_chunk(32 * lc + 16 * v + 4 * t + 2 * pr + c2));
+                  xw[v][pr][nt][4 * c2 + 0] = xv.x; xw[v][pr][nt][4 * c2 + 1] = xv.y;
+                  xw[v][pr][nt][4 * c2 + 2] = xv.z; xw[v][pr][nt][4 * c2 + 3] = xv.w;
+                }
               }
-          }
+          xchunk = lc;
         }
-        // the slot's shared memory is read: hand it back to the producer
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.empty[s]);
-        if (mine) {
-          int* au = acc_s + u * kUnitRows * NTOK;
+        const uint8_t* box = wring + s * slot_bytes + sb * kSubBytes;
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            int cv[4];
+        for (int v = 0; v < 2; ++v) {
+          const int cw = 4 * v + t;                  // 16-byte chunk of the 128-byte row
+          const uint4 wa = *reinterpret_cast<const uint4*>(box + r0 * 128 + ((cw ^ r0) << 4));
+          const uint4 wb = *reinterpret_cast<const uint4*>(box + (r0 + 8) * 128 + ((cw ^ r0) << 4));
+          const uint32_t w0[4] = {wa.x, wa.y, wa.z, wa.w};
+          const uint32_t w1[4] = {wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
-            for (int rr = 0; rr < 4; ++rr)
-              cv[rr] = acc[0][nt][rr] + (acc[1][nt][rr] >> 2) + (acc[2][nt][rr] >> 4) + (acc[3][nt][rr] >> 6);
-            const int m0 = nt * 8 + 2 * t;
-            if (m0 < M) {
-              red_shared_add(au + r0 * NTOK + m0, cv[0]);
-              red_shared_add(au + (r0 + 8) * NTOK + m0, cv[2]);
+          for (int pr = 0; pr < 2; ++pr)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const uint32_t mask = kCodeMask << (2 * i);
+              const uint32_t a0 = w0[2 * pr] & mask, a1 = w1[2 * pr] & mask;
+              const uint32_t a2 = w0[2 * pr + 1] & mask, a3 = w1[2 * pr + 1] & mask;
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt)
+                mma_u8s8(acc[i][nt], a0, a1, a2, a3, xw[v][pr][nt][i], xw[v][pr][nt][4 + i]);
             }
-            if (m0 + 1 < M) {
-              red_shared_add(au + r0 * NTOK + m0 + 1, cv[1]);
-              red_shared_add(au + (r0 + 8) * NTOK + m0 + 1, cv[3]);
-            }
-          }
+        }
+      }
+      // the slot is read: refill it with this warp's next item
+      __syncwarp();
+      ++consumed;
+      cc.next(warp, nround, F, kc, tail, U);
+      issue_next();
+      // fields -> the unit's sums (4^i sum(c q) >> 2i is exact: at most 8 chunks
+      // of 512 k per item keep 64 * 2 * 127 * 4096 below 2^31)
+      int* au = acc_s + u * kUnitRows * NTOK;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        int cv[4];
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr)
+          cv[rr] = acc[0][nt][rr] + (acc[1][nt][rr] >> 2) + (acc[2][nt][rr] >> 4) + (acc[3][nt][rr] >> 6);
+        const int m0 = nt * 8 + 2 * t;
+        if (m0 < M) {
+          red_shared_add(au + r0 * NTOK + m0, cv[0]);
+          red_shared_add(au + (r0 + 8) * NTOK + m0, cv[2]);
+        }
+        if (m0 + 1 < M) {
+          red_shared_add(au + r0 * NTOK + m0 + 1, cv[1]);
+          red_shared_add(au + (r0 + 8) * NTOK + m0 + 1, cv[3]);
         }
       }
     }
   }
   if (!ok) {
     report_status(a.status, kStatusTimeout);
-    sm.failed = 1;
+    if (lane == 0) {
+      sm.failed = 1;
+      // every load this warp issued lands before the CTA exits (fixed limit)
+      for (int q = consumed; q < issued; ++q) mbar_wait(&full[q % ring], (q / ring) & 1, kWaitLimitNs);
+    }
+    __syncwarp();
   }
   __syncthreads();
-  if (sm.failed && threadIdx.x == kConsumerWarps * 32) {
-    // After a timeout some loads may still be in flight, and every load
-    // issued must land before the CTA exits.  The last load into a slot
-    // completes that slot's latest phase: the loads before it were consumed,
-    // which needed them complete.
-    const int q = sm.issued;
-    for (int s = 0; s < ring && s < q; ++s) {
-      const int last = s + ((q - 1 - s) / ring) * ring;
-      mbar_wait(&sm.full[s], (last / ring) & 1, kWaitLimitNs);
-    }
-  }
 
   // ---------------- epilogue: U units x 16 rows x M tokens ----------------
   const int rows = U * kUnitRows;
@@ -546,7 +580,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
     const int accv = acc_s[rl * NTOK + m] - sm.rsum[m];
     int gi = 0;                                      // the row's group (scale)
 #pragma unroll
-    for (int g = 0; g + 1 < kMaxGroups; ++g) gi += (g + 1 < a.ngroups && n >= a.group_end[g]) ? 1 : 0;
+    for (int gg = 0; gg + 1 < kMaxGroups; ++gg) gi += (gg + 1 < a.ngroups && n >= a.group_end[gg]) ? 1 : 0;
     float y32;
     if (!a.faithful) {
       const float d = __fmul_rn(sm.sx[m], sm.swg[gi]);
@@ -588,6 +622,13 @@ cudaError_t launch_nt(const CUtensorMap& tm3, const CUtensorMap& tm2, const Deco
 
 }  // namespace
 
+#ifndef BITLINEAR_DECODE_KC
+#define BITLINEAR_DECODE_KC 2       // chunks (2 KB sub-boxes) per TMA load
+#endif
+#ifndef BITLINEAR_DECODE_RING
+#define BITLINEAR_DECODE_RING 8     // largest ring per warp
+#endif
+
 DecodePlan plan_decode(int M, int N, int K, int num_sms) {
   DecodePlan p;
   const int units_total = (N + kUnitRows - 1) / kUnitRows;
@@ -595,16 +636,23 @@ DecodePlan plan_decode(int M, int N, int K, int num_sms) {
   if ((units_total + p.grid - 1) / p.grid > kMaxUnits) p.grid = (units_total + kMaxUnits - 1) / kMaxUnits;
   p.units_max = (units_total + p.grid - 1) / p.grid;
   const int F = K / kBoxK;
-  p.kc = F < kConsumerWarps ? F : kConsumerWarps;
+  // loads of kc chunks when there are full chunks to group, else one chunk
+  p.kc = F >= 2 * BITLINEAR_DECODE_KC ? BITLINEAR_DECODE_KC : 1;
   p.tail = (K % kBoxK) != 0;
-  p.slot_bytes = static_cast<size_t>(p.kc + p.tail) * kSubBytes;
+  p.slot_bytes = static_cast<size_t>(p.kc) * kSubBytes;
   // shared-memory budget: two CTAs per SM for the 8-token kernel (the next
   // kernel on the stream can start beside this one), one for 16 tokens
   const long long budget = M <= 8 ? 110 * 1024 : 220 * 1024;
   const long long room = budget - static_cast<long long>(smem_layout(M, 0, p.slot_bytes, p.units_max).total);
-  long long ring = room > 0 ? room / static_cast<long long>(p.slot_bytes) : 0;
-  ring = ring > kMaxRing ? kMaxRing : ring;
-  p.ring = ring < 2 ? 2 : static_cast<int>(ring);
+  long long ring = room > 0 ? room / (static_cast<long long>(kWarps) * static_cast<long long>(p.slot_bytes)) : 0;
+  ring = ring > BITLINEAR_DECODE_RING ? BITLINEAR_DECODE_RING : ring;
+  if (ring < 2 && p.kc > 1) {                     // fall back to single-chunk loads
+    p.kc = 1;
+    p.slot_bytes = kSubBytes;
+    ring = room > 0 ? room / (static_cast<long long>(kWarps) * kSubBytes) : 0;
+    ring = ring > BITLINEAR_DECODE_RING ? BITLINEAR_DECODE_RING : ring;
+  }
+  p.ring = ring < 1 ? 1 : static_cast<int>(ring);
   p.smem = smem_layout(M, p.ring, p.slot_bytes, p.units_max).total;
   return p;
 }
@@ -623,7 +671,7 @@ cudaError_t launch_decode(DecodeArgs a, int num_sms, cudaStream_t stream) {
                     static_cast<uint64_t>(a.K) / 4, kBoxK / 4, kUnitRows, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   tm3 = tm2;
-  if (p.kc > 0) {
+  if (a.K >= kBoxK) {
     // 3-D view [full chunk][row][128 bytes]: a box is kc consecutive 512-k
     // chunks of 16 rows, each chunk landing as its own 16 x 128-byte sub-box
     const uint64_t dims[3] = {static_cast<uint64_t>(kBoxK / 4), static_cast<uint64_t>(a.N),

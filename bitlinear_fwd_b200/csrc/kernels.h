@@ -115,6 +115,9 @@ cudaError_t set_smem_attr_once(Kern kern, int bytes, unsigned long long* done_ma
   return e;
 }
 
+// ---- the int8 tensor-core rate (tc_peak.cu), a measurement utility ---------
+cudaError_t launch_tc_i8_peak(int iters, int num_sms, uint32_t* status, cudaStream_t stream);
+
 // ---- decode engine, M <= 16 (gemv_decode.cu) --------------------------------
 struct DecodeArgs {
   const uint16_t* x;      // bf16 [M, K], quantised inside the kernel; or null

@@ -359,6 +359,18 @@ int bitlinear_epilogue_sum(const int32_t* const* partials, int nparts, int64_t M
                            const float* w_scale, const uint16_t* bias, uint16_t* y, int32_t* acc_out,
                            unsigned flags, void* stream);
 
+/* Measurement utility, not part of the method (the pages have no
+ * counterpart): enqueues a kernel that runs the int8 tensor cores alone at
+ * full rate -- one CTA per SM, `iters` x 4 back-to-back tcgen05.mma kind::i8
+ * of 128 x 256 x 32 on zero operands -- so that the caller can time it with
+ * CUDA events and derive the GPU's dense int8 rate:
+ *   int8 ops = 2 * 128 * 256 * 32 * 4 * iters * (*grid).
+ *   iters   1 .. 2^24
+ *   grid    host out: the number of CTAs launched (the SM count)
+ *   ws      at least 256 bytes of device memory: its first word is a status
+ *           word (bitlinear_check_status reads it) */
+int bitlinear_measure_i8_peak(int iters, int* grid, void* ws, size_t ws_bytes, void* stream);
+
 /* Test hook for the failure path of the device-side waits.  While it is on
  * (on != 0), every forward launched by this process -- bitlinear_forward and
  * its variants, both engines -- makes one wait on a barrier that nothing

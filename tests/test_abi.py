@@ -185,6 +185,7 @@ def test_valid_arguments_pass_every_host_check(lib):
         "forward partial M=40": lib.bitlinear_forward_partial(16, 40, 256, 16, 16, 512, 16, 2, 16, 1 << 20, None),
         "epilogue sum": lib.bitlinear_epilogue_sum((ctypes.c_void_p * 2)(16, 32), 2, 8, 512, 16, 16, 16, 16, None,
                                                    0, None),
+        "i8 peak": lib.bitlinear_measure_i8_peak(10, ctypes.byref(ctypes.c_int(0)), 16, 256, None),
         "pack": lib.bitlinear_pack_weights(16, 512, 256, 16, 16, 16, 16, 4096, None),
         "quant_act": lib.bitlinear_quant_act(16, 4, 256, 16, 16, 16, None),
         "dequant": lib.bitlinear_dequant_weights(16, 512, 256, 16, 16, None),
@@ -224,3 +225,12 @@ def test_ksplit_entry_points_reject_bad_arguments(lib):
     assert ep((ctypes.c_void_p * 2)(16, 20), 2, 8, 512, 16, 16, None, 16, None, 0, None) == -3
     assert ep(two, 2, 8, 512, 16, 16, None, 16, None, 8, None) == -2
     assert ep(two, 2, 0, 512, 16, 16, None, 16, None, 0, None) == 0
+
+
+def test_i8_peak_rejects_bad_arguments(lib):
+    g = ctypes.c_int(0)
+    assert lib.bitlinear_measure_i8_peak(0, ctypes.byref(g), 16, 256, None) == -2
+    assert lib.bitlinear_measure_i8_peak((1 << 24) + 1, ctypes.byref(g), 16, 256, None) == -2
+    assert lib.bitlinear_measure_i8_peak(10, None, 16, 256, None) == -1
+    assert lib.bitlinear_measure_i8_peak(10, ctypes.byref(g), 16, 128, None) == -4
+    assert lib.bitlinear_measure_i8_peak(10, ctypes.byref(g), 20, 256, None) == -3

@@ -73,7 +73,8 @@ def test_extreme_activations(M, engine, faithful):
     out = bl.bitlinear_forward_debug(x.cuda(), packed, s_w, bias.cuda(), engine=engine, flags=flags)
     torch.cuda.synchronize()
     assert bl.bitlinear_check_status(out["ws"]) == 0
-    want = oracle_out(x, packed.cpu().numpy(), s_w.item(), bias, faithful)
+    opk, osw, _ = oracle.pack_weights(w.numpy())               # the oracle's own packing
+    want = oracle_out(x, opk, osw, bias, faithful)
     assert np.all(np.isfinite(want["y32"]))
     assert np.array_equal(out["xq"].cpu().numpy(), want["q"])
     assert np.array_equal(out["s_x"].cpu().numpy().view(np.uint32), want["s_x"].view(np.uint32))

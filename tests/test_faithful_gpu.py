@@ -26,8 +26,9 @@ def _compare(x, w, bias, engine, rows=None):
     M = x.shape[0]
     rows = np.arange(M) if rows is None else rows
     xb = synth.bf16_bits(x)
-    want = oracle.forward_bf16(xb[rows], packed.cpu().numpy(), np.float32(s_w.item()),
-                               None if bias is None else synth.bf16_bits(bias))
+    # the oracle packs the same weights itself; nothing the GPU computed feeds it
+    opk, osw, _ = oracle.pack_weights(w.numpy())
+    want = oracle.forward_bf16(xb[rows], opk, osw, None if bias is None else synth.bf16_bits(bias))
     assert np.array_equal(out["xq"].cpu().numpy()[rows], want["q"])
     assert np.array_equal(out["s_x"].cpu().numpy()[rows], want["s_x"])
     assert np.array_equal(out["acc"].cpu().numpy()[rows], want["acc"])

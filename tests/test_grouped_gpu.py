@@ -16,17 +16,22 @@ pytestmark = pytest.mark.gpu
 
 
 def _stack(rows, K, seed, std=0.02):
-    packs, scales, ws = [], [], []
+    """The layers' weights packed by the GPU, and the same weights packed by
+    the oracle (its own packing feeds its expected values)."""
+    packs, scales, opks, oscales = [], [], [], []
     for g, n in enumerate(rows):
         w = synth.normal_f32(seed, 100 * g + n, (n, K), std * (1 + 0.5 * g))
         p, s, _ = bl.bitlinear_pack_weights(w.cuda())
         packs.append(p)
         scales.append(s)
-    return torch.cat(packs), torch.cat(scales), packs, scales
+        op, osw, _ = oracle.pack_weights(w.numpy())
+        opks.append(op)
+        oscales.append(osw)
+    return torch.cat(packs), torch.cat(scales), packs, scales, np.concatenate(opks), oscales
 
 
 def _check(M, K, rows, seed, with_bias, flags=0, sample=None):
-    packed, s_ws, packs, scales = _stack(rows, K, seed)
+    packed, s_ws, packs, scales, opk, oscales = _stack(rows, K, seed)
     N = sum(rows)
     x = synth.normal_bf16(seed, M + K, (M, K))
     b = synth.normal_bf16(seed, N, (N,), 0.05) if with_bias else None
@@ -42,8 +47,7 @@ def _check(M, K, rows, seed, with_bias, flags=0, sample=None):
     torch.cuda.synchronize()
     mrows = np.arange(M) if sample is None else sample_rows(M, sample)
     xb = synth.bf16_bits(x)[mrows]
-    want = oracle.forward_grouped(xb, packed.cpu().numpy(), rows, [np.float32(v) for v in s_ws.cpu().numpy()],
-                                  None if b is None else synth.bf16_bits(b))
+    want = oracle.forward_grouped(xb, opk, rows, oscales, None if b is None else synth.bf16_bits(b))
     got = y.cpu()[mrows].view(torch.int16).numpy().view(np.uint16)
     assert np.array_equal(got, want["y"])
 
