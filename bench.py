@@ -410,6 +410,23 @@ def run_e2e(args, probs, steps):
                               "api": "the same six calls issued one by one, one stream sync per step"}}
 
 
+def measured_i8_peak():
+    """The dense int8 tensor-core rate of this GPU from the library's own
+    tcgen05 kind::i8 loop (bitlinear_measure_i8_peak), with the SM clock
+    sampled while it ran."""
+    import bitlinear_fwd_b200 as bl
+    sampler = ClockSampler(torch.cuda.current_device())
+    r = bl.measure_i8_peak(iters=20000, reps=3)
+    clk = sampler.stop()
+    mhz = clk.get("sm_mhz") or None
+    out = {"tops": round(r["tops"], 1), "ms": round(r["ms"], 3), "clocks": clk,
+           "how": "tcgen05.mma.cta_group::1.kind::i8 128x256x32, smem operands, one CTA per SM, "
+                  f"{r['iters']} x 4 per CTA, best of 3 launches (CUDA events)"}
+    if mhz:
+        out["mac_per_clk_per_sm"] = round(r["macs_per_sm"] / (r["ms"] * 1e-3) / (mhz * 1e6), 1)
+    return out
+
+
 def run_prefill(args, bf16_tflops, peak_kind, l2_bytes, i8_peak=None):
     cases = wl.workload3()
     probs, copies = make_problems(cases, l2_bytes, rotate_factor=1.0, max_copies=3, force_copies=args.copies)

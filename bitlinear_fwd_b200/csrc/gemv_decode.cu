@@ -28,10 +28,10 @@
 //   * Before the items, all warps form each token's absmax over the row,
 //     s_x = 127 / max(absmax, 1e-5) in float32, and q = round_half_even(x
 //     s_x) as int8 into shared memory, one round at a time, with the sum of q
-//     per token.  For M <= 4 and K <= 4096 each lane's share of x is read
-//     once and held in registers between the two steps; otherwise x is read
-//     again for the quantising step.  Pre-quantised int8 input is copied in
-//     instead.
+//     per token.  For K <= 4096 each lane's share of x (at most 8 x 32
+//     bytes per token, two tokens per warp when M > 8) is read once and held
+//     in registers between the two steps; otherwise x is read again for the
+//     quantising step.  Pre-quantised int8 input is copied in instead.
 //   * Per chunk of an item, a thread takes one 16-byte vector of two weight
 //     rows and issues mma.sync m16n8k32 (weights as A, u8; tokens as B, s8;
 //     a second 8-token tile for M > 8).  The codes c = u + 1 enter
@@ -71,7 +71,7 @@ constexpr int kMaxRing = 8;                           // slots per warp
 constexpr int kMaxUnits = 32;                         // units per CTA
 constexpr int kXB = 8;                                // bf16 x loads in flight per lane (absmax)
 constexpr int kQB = 2;                                // the same in the quantising pass
-constexpr int kHold = 4;                              // 32-byte x chunks per lane and token held in
+constexpr int kHold = 8;                              // 32-byte x chunks per lane and token held in
                                                       // registers by the one-pass path
 constexpr uint32_t kCodeMask = 0x03030303u;
 constexpr float kRoundMagic = 12582912.0f;            // 1.5 * 2^23
@@ -308,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
   const int C = (cpr + 32 * P - 1) / (32 * P);       // chunks per lane per token
   // One pass over x when the row is one round and this lane's share fits in
   // registers: the values loaded for the absmax are quantised in place.
-  const bool single = NT == 1 && a.x && nround == 1 && C <= kHold;
+  const bool single = a.x && nround == 1 && C <= kHold;
   if (single) {
     const uint4* xrow0 = reinterpret_cast<const uint4*>(a.x);
     uint4 v[kHold * NT][2];

@@ -92,7 +92,10 @@ __global__ void __launch_bounds__(kThreads) absmean_bins_kernel(const float4* __
   e0 = __reduce_max_sync(kFull, e0);
   const int B = max(static_cast<int>(e0) - kAnchorBelow, 1);
 
-  uint64_t lo = 0, hi = 0;
+  // one 128-bit sum per unrolled load: four independent carry chains
+  uint64_t lo[kUnroll], hi[kUnroll];
+#pragma unroll
+  for (int u = 0; u < kUnroll; ++u) lo[u] = hi[u] = 0;
   for (int64_t base = warp_base; base < n4; base += stride * kUnroll) {
     float4 v[kUnroll];
 #pragma unroll
@@ -103,10 +106,10 @@ __global__ void __launch_bounds__(kThreads) absmean_bins_kernel(const float4* __
     bool out = false;
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      out |= window_add(__float_as_uint(v[u].x), B, lo, hi);
-      out |= window_add(__float_as_uint(v[u].y), B, lo, hi);
-      out |= window_add(__float_as_uint(v[u].z), B, lo, hi);
-      out |= window_add(__float_as_uint(v[u].w), B, lo, hi);
+      out |= window_add(__float_as_uint(v[u].x), B, lo[u], hi[u]);
+      out |= window_add(__float_as_uint(v[u].y), B, lo[u], hi[u]);
+      out |= window_add(__float_as_uint(v[u].z), B, lo[u], hi[u]);
+      out |= window_add(__float_as_uint(v[u].w), B, lo[u], hi[u]);
     }
     if (__any_sync(kFull, out)) {
       // rare: weights outside the window go to their own exponent's bin
@@ -125,9 +128,14 @@ __global__ void __launch_bounds__(kThreads) absmean_bins_kernel(const float4* __
   }
   // the thread's sum is below 2^96 (fewer than 2^33 terms below 2^63): four
   // 24-bit chunks, chunk j of weight 2^(B + 24j - 150)
-  const uint32_t ch[4] = {static_cast<uint32_t>(lo & 0xFFFFFFull), static_cast<uint32_t>((lo >> 24) & 0xFFFFFFull),
-                          static_cast<uint32_t>(((lo >> 48) | (hi << 16)) & 0xFFFFFFull),
-                          static_cast<uint32_t>((hi >> 8) & 0xFFFFFFull)};
+  uint64_t lo_t = lo[0], hi_t = hi[0];
+#pragma unroll
+  for (int u = 1; u < kUnroll; ++u)
+    asm("add.cc.u64 %0, %0, %2;\n\taddc.u64 %1, %1, %3;" : "+l"(lo_t), "+l"(hi_t) : "l"(lo[u]), "l"(hi[u]));
+  const uint64_t lo_s = lo_t, hi_s = hi_t;
+  const uint32_t ch[4] = {static_cast<uint32_t>(lo_s & 0xFFFFFFull), static_cast<uint32_t>((lo_s >> 24) & 0xFFFFFFull),
+                          static_cast<uint32_t>(((lo_s >> 48) | (hi_s << 16)) & 0xFFFFFFull),
+                          static_cast<uint32_t>((hi_s >> 8) & 0xFFFFFFull)};
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const uint32_t s = __reduce_add_sync(kFull, ch[j]);   // < 32 * 2^24

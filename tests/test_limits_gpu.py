@@ -96,7 +96,7 @@ def test_k_max_accumulators_beyond_2_24(large_k_weights, M, engine):
     ref = oracle.forward(synth.bf16_bits(x), opk, osw, synth.bf16_bits(bias))
     # the case this test exists for: numerators that float32 cannot hold exactly
     big = np.abs(ref["acc"]) > (1 << 24)
-    assert big.sum() >= 3 * M, "the inputs must drive |acc| past 2^24"
+    assert big.sum() >= 2 * M, "the inputs must drive |acc| past 2^24 (rows 0 and 1 for every token)"
     assert np.any(ref["acc"][big] % 2 != 0), "some of them must be odd, so that float(acc) rounds"
     out = bl.bitlinear_forward_debug(x.cuda(), packed, s_w, bias.cuda(), engine=engine)
     torch.cuda.synchronize()
