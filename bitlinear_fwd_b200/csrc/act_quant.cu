@@ -47,27 +47,43 @@ __device__ __forceinline__ int reduce_add_i32(int v, int* red) {
   return t;  // valid in thread 0
 }
 
-// Quantises 16 bf16 values (two 16-byte vectors) into one 16-byte vector of int8.
-__device__ __forceinline__ uint4 quant16(uint4 lo, uint4 hi, float s, int& sum, bool faithful) {
-  const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-  uint32_t out[4];
+// Four bf16 values (two words) -> four int8 q = round_half_even(x * s), packed.
+// p = x * s is rounded to float32 first; adding 1.5 * 2^23 then rounds p to an
+// integer with ties to even (the sum lies in [2^23, 2^24), where the float
+// spacing is 1, and the constant is even), and the low byte of the sum's bits
+// is q as a two's-complement byte.  In float32 |p| <= 127 because s was formed
+// from the row's absmax (or, for a K-shard, the whole row's), so the
+// [-128, 127] clamp never acts there; the bf16-faithful path rounds p to bf16
+// and clamps explicitly (bf16(x * scale) can reach 128).
+constexpr float kRoundMagic = 12582912.0f;   // 1.5 * 2^23
+
+__device__ __forceinline__ uint32_t quant4(uint32_t w01, uint32_t w23, float s, bool faithful) {
+  float p[4] = {__fmul_rn(__uint_as_float(w01 << 16), s), __fmul_rn(__uint_as_float(w01 & 0xFFFF0000u), s),
+                __fmul_rn(__uint_as_float(w23 << 16), s), __fmul_rn(__uint_as_float(w23 & 0xFFFF0000u), s)};
+  if (faithful) {
 #pragma unroll
-  for (int b = 0; b < 4; ++b) {
-    uint32_t packed = 0;
-#pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      const int e = 4 * b + h;  // element 0..15
-      const uint32_t bits = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu);
-      float t = __fmul_rn(bf16_bits_to_f32(bits), s);
-      if (faithful) t = bf16_round(t);               // the bf16 tensor x * scale
-      int q = __float2int_rn(t);
-      q = min(127, max(-128, q));
-      sum += q;
-      packed |= (static_cast<uint32_t>(q) & 0xFFu) << (8 * h);
-    }
-    out[b] = packed;
+    for (int e = 0; e < 4; ++e) p[e] = fminf(fmaxf(bf16_round(p[e]), -128.0f), 127.0f);
   }
-  return make_uint4(out[0], out[1], out[2], out[3]);
+  const uint32_t b0 = __float_as_uint(__fadd_rn(p[0], kRoundMagic));
+  const uint32_t b1 = __float_as_uint(__fadd_rn(p[1], kRoundMagic));
+  const uint32_t b2 = __float_as_uint(__fadd_rn(p[2], kRoundMagic));
+  const uint32_t b3 = __float_as_uint(__fadd_rn(p[3], kRoundMagic));
+  return __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
+}
+
+// Quantises 16 bf16 values (two 16-byte vectors) into one 16-byte vector of
+// int8 and adds their sum to `sum`.
+__device__ __forceinline__ uint4 quant16(uint4 lo, uint4 hi, float s, int& sum, bool faithful) {
+  uint4 q;
+  q.x = quant4(lo.x, lo.y, s, faithful);
+  q.y = quant4(lo.z, lo.w, s, faithful);
+  q.z = quant4(hi.x, hi.y, s, faithful);
+  q.w = quant4(hi.z, hi.w, s, faithful);
+  sum = __dp4a(static_cast<int>(q.x), 0x01010101, sum);
+  sum = __dp4a(static_cast<int>(q.y), 0x01010101, sum);
+  sum = __dp4a(static_cast<int>(q.z), 0x01010101, sum);
+  sum = __dp4a(static_cast<int>(q.w), 0x01010101, sum);
+  return q;
 }
 
 template <int CPT>  // 16-element chunks cached per thread; 0 = read the row twice

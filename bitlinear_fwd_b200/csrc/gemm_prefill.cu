@@ -71,8 +71,8 @@ static_assert(2 * BT + ASTAGES * kACols <= kTmemCols, "two accumulators and the 
 
 constexpr uint32_t kOffX = 0;
 constexpr uint32_t kOffWp = kOffX + STAGES * kXBytes;
-constexpr uint32_t kOffD = kOffWp + STAGES * kWpBytes;       // s_x per token [BT]
-constexpr uint32_t kOffRs = kOffD + 4 * BT;                  // row sums per token [BT]
+constexpr uint32_t kOffD = kOffWp + STAGES * kWpBytes;       // per token: 1 / d in double [BT], or s_x
+constexpr uint32_t kOffRs = kOffD + 8 * BT;                  // row sums per token [BT]
 constexpr uint32_t kOffBar = kOffRs + 4 * BT;
 constexpr uint32_t kSmemBytes = kOffBar + 512 + 1024;        // + barriers, alignment slack
 // tcgen05.alloc of all 512 columns waits until the columns are free, with no
@@ -98,7 +98,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(stall_bar + 1);
   volatile int* failed = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* drain_bad = failed + 1;       // a drain gave up: MMAs may still run
-  float* d_s = reinterpret_cast<float*>(smem + kOffD);
+  double* rcp_s = reinterpret_cast<double*>(smem + kOffD);   // per token, when the tile has one scale
+  float* sx_s = reinterpret_cast<float*>(smem + kOffD);      // per token s_x, when it has several
   int* rs_s = reinterpret_cast<int*>(smem + kOffRs);
   const uint64_t wait_ns = a.wait_ns;
 
@@ -265,7 +266,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     float swg[kMaxGroups];                         // s_w of each row group
 #pragma unroll
     for (int g = 0; g < kMaxGroups; ++g) swg[g] = g < a.ngroups ? a.w_scale[g] : 0.0f;
-    const bool simple = a.ngroups == 1 && !a.faithful;
     int j = 0;
     // The eight epilogue warps meet at a named barrier twice per tile; every
     // one of them runs every iteration (a failure only skips work), so the
@@ -273,13 +273,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++j) {
       const int b = j & 1;
       const int n0 = (tile % wtiles) * BW, m0 = (tile / wtiles) * BT;
+      // The tile's rows share one layer's scale unless a group boundary of
+      // stacked layers falls inside it (rare: only grouped calls).
+      const int nlast = min(n0 + BW, a.N) - 1;
+      int g0 = 0, g1 = 0;
+#pragma unroll
+      for (int g = 0; g + 1 < kMaxGroups; ++g) {
+        g0 += (g + 1 < a.ngroups && n0 >= a.group_end[g]) ? 1 : 0;
+        g1 += (g + 1 < a.ngroups && nlast >= a.group_end[g]) ? 1 : 0;
+      }
+      const bool uniform = g0 == g1;
+      float sw_tile = swg[0];
+#pragma unroll
+      for (int g = 1; g < kMaxGroups; ++g)
+        if (g == g0) sw_tile = swg[g];
       // per-token s_x and row sums of this tile
       asm volatile("bar.sync 1, 256;" ::: "memory");   // previous tile's readers are done
       if (et < BT) {
-        // one float32 layer: d = s_x * s_w per token; otherwise s_x (the
-        // row's scale enters per element)
         const int m = m0 + et;
-        d_s[et] = m < a.M ? (simple ? __fmul_rn(a.s_x[m], swg[0]) : a.s_x[m]) : 1.0f;
+        const float sx = m < a.M ? a.s_x[m] : 1.0f;
+        if (uniform) {
+          // d = s_x s_w (float32), or on a bf16 module bf16(bf16(s_w) s_x),
+          // kept as the double 1 / d: RN_f32(a * (1/d)) with a the float32
+          // (or bf16) numerator is RN_f32(a / d) -- a quotient of two floats
+          // lies at least 2^-49 (relative) from every float32 midpoint, and
+          // the double product is within 2^-52 of it.
+          const float d = a.faithful ? bf16_round(__fmul_rn(bf16_round(sw_tile), sx)) : __fmul_rn(sx, sw_tile);
+          rcp_s[et] = __drcp_rn(static_cast<double>(d));
+        } else {
+          sx_s[et] = sx;
+        }
         rs_s[et] = m < a.M ? a.rowsum[m] : 0;
       }
       asm volatile("bar.sync 1, 256;" ::: "memory");
@@ -294,7 +317,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int n = n0 + 32 * q + lane;
       const bool nv = n < a.N;
       const float bv = (a.bias && nv) ? bf16_bits_to_f32(a.bias[n]) : 0.0f;
-      float s_w = swg[0];                          // this row's group scale
+      float s_w = swg[0];                          // this row's group scale (tiles with several)
 #pragma unroll
       for (int g = 1; g < kMaxGroups; ++g)
         if (g < a.ngroups && n >= a.group_end[g - 1]) s_w = swg[g];
@@ -307,14 +330,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       auto process = [&](const uint32_t (&r)[32], int c) {
         if (!nv) return;
-        if (simple) {
+        if (uniform && !a.faithful) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const int mi = 32 * c + i;
             if (m0 + mi >= a.M) continue;
             const int accv = static_cast<int>(r[i]) - rs_s[mi];
-            float y32 = __fdiv_rn(static_cast<float>(accv), d_s[mi]);
+            float y32 = __double2float_rn(static_cast<double>(static_cast<float>(accv)) * rcp_s[mi]);
             if (a.bias) y32 = __fadd_rn(y32, bv);
+            emit(mi, accv, y32);
+          }
+        } else if (uniform) {
+          // bf16 module: the sum, the quotient and the bias add are each
+          // rounded to bf16 (the scale product is in rcp_s)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int mi = 32 * c + i;
+            if (m0 + mi >= a.M) continue;
+            const int accv = static_cast<int>(r[i]) - rs_s[mi];
+            float y32 = bf16_round(__double2float_rn(static_cast<double>(bf16_round(static_cast<float>(accv))) * rcp_s[mi]));
+            if (a.bias) y32 = bf16_round(__fadd_rn(y32, bv));
             emit(mi, accv, y32);
           }
         } else if (!a.faithful) {
@@ -323,19 +358,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int mi = 32 * c + i;
             if (m0 + mi >= a.M) continue;
             const int accv = static_cast<int>(r[i]) - rs_s[mi];
-            float y32 = __fdiv_rn(static_cast<float>(accv), __fmul_rn(d_s[mi], s_w));
+            float y32 = __fdiv_rn(static_cast<float>(accv), __fmul_rn(sx_s[mi], s_w));
             if (a.bias) y32 = __fadd_rn(y32, bv);
             emit(mi, accv, y32);
           }
         } else {
-          // bf16 module: the sum, the scale product, the quotient and the
-          // bias add are each rounded to bf16
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const int mi = 32 * c + i;
             if (m0 + mi >= a.M) continue;
             const int accv = static_cast<int>(r[i]) - rs_s[mi];
-            float y32 = bf16_round(__fdiv_rn(bf16_round(static_cast<float>(accv)), bf16_round(__fmul_rn(s_w, d_s[mi]))));
+            float y32 = bf16_round(__fdiv_rn(bf16_round(static_cast<float>(accv)), bf16_round(__fmul_rn(s_w, sx_s[mi]))));
             if (a.bias) y32 = bf16_round(__fadd_rn(y32, bv));
             emit(mi, accv, y32);
           }

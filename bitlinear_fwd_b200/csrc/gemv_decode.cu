@@ -12,26 +12,28 @@
 //
 // Inside a CTA every one of the 8 warps streams and computes:
 //   * The CTA's work of a round is a list of items (chunk group, unit), chunk
-//     group outer: a group is kc consecutive full chunks of one unit, loaded
-//     by one TMA instruction as a 3-D box of kc sub-boxes of 16 rows x 128
-//     bytes (128-byte swizzle); a partial last chunk is an item of its own,
-//     loaded through a 2-D view that K bounds (zero fill beyond K).  Warp w
-//     takes items w, w + 8, ... of every round, so the warps' shares differ
-//     by at most one item.
+//     group outer: a group is kc consecutive chunks of one unit (the last one
+//     of K maybe partial).  Warp w takes items w, w + 8, ... of every round,
+//     so the warps' shares differ by at most one item.
 //   * Each warp streams its own items through its own ring of shared-memory
-//     slots: its lane 0 issues the TMA loads up to `ring` items ahead and
-//     refills a slot as soon as the warp has read it; the warp waits on the
-//     slot's mbarrier.  No warp ever waits for another warp's loads, so TMA
-//     issue is spread over all 8 warps.  When the weights are resident the
-//     first loads are issued before the wait on the previous kernel of the
-//     stream, so the stream overlaps that kernel's tail.
+//     slots: every lane copies its own 16-byte pieces of an item with
+//     cp.async (128-byte rows, written in the 128-byte-swizzled order that
+//     keeps the fragment reads below conflict-free), one copy group per item,
+//     up to `ring` items ahead; pieces beyond N or K are zero-filled.  The
+//     warp waits for the oldest group and refills its slot once it has read
+//     it.  No warp ever waits for another warp's copies.  When the weights
+//     are resident the first copies (and the bias and scales, into
+//     registers) are issued before the wait on the previous kernel of the
+//     stream, so they overlap its tail.
 //   * Before the items, all warps form each token's absmax over the row,
 //     s_x = 127 / max(absmax, 1e-5) in float32, and q = round_half_even(x
 //     s_x) as int8 into shared memory, one round at a time, with the sum of q
 //     per token.  For K <= 4096 each lane's share of x (at most 8 x 32
 //     bytes per token, two tokens per warp when M > 8) is read once and held
 //     in registers between the two steps; otherwise x is read again for the
-//     quantising step.  Pre-quantised int8 input is copied in instead.
+//     quantising step.  CTA b starts its x reads at a different chunk, so the
+//     SMs do not ask for the same L2 lines at the same moment.  Pre-quantised
+//     int8 input is copied in instead.
 //   * Per chunk of an item, a thread takes one 16-byte vector of two weight
 //     rows and issues mma.sync m16n8k32 (weights as A, u8; tokens as B, s8;
 //     a second 8-token tile for M > 8).  The codes c = u + 1 enter
@@ -42,9 +44,11 @@
 //     the chunk.
 //   * Epilogue: acc = sum(c q) - sum(q) = sum(u q); y = acc / (s_x s_w)
 //     (+ bias) -> bf16, with s_w the scale of the row's layer when several
-//     layers are stacked.  The bf16-faithful mode rounds the scale, the
-//     products, the sum and the quotient to bf16 as a bf16 module does.
-// Rows beyond N and k beyond K are zero-filled by TMA (code 0), so they add
+//     layers are stacked, the division done as a product with the double
+//     1 / (s_x s_w) of the token and layer (exactly the float32 quotient).
+//     The bf16-faithful mode rounds the scale, the products, the sum and the
+//     quotient to bf16 as a bf16 module does.
+// Rows beyond N and k beyond K are zero-filled (code 0), so they add
 // nothing whatever the x bytes there are.
 //
 // Fragment layout.  MMA row g of a unit is box row pi(g) = (g >> 1) |
@@ -85,6 +89,27 @@ __device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, 
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// 16-byte asynchronous copy global -> shared (L2 only); src_bytes = 0 writes
+// zeros and reads nothing
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)), "l"(gsrc), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// waits until at most n of this thread's copy groups are still in flight
+__device__ __forceinline__ void cp_async_wait(int n) {
+  switch (n) {
+    case 0: asm volatile("cp.async.wait_group 0;" ::: "memory"); break;
+    case 1: asm volatile("cp.async.wait_group 1;" ::: "memory"); break;
+    case 2: asm volatile("cp.async.wait_group 2;" ::: "memory"); break;
+    case 3: asm volatile("cp.async.wait_group 3;" ::: "memory"); break;
+    case 4: asm volatile("cp.async.wait_group 4;" ::: "memory"); break;
+    case 5: asm volatile("cp.async.wait_group 5;" ::: "memory"); break;
+    case 6: asm volatile("cp.async.wait_group 6;" ::: "memory"); break;
+    default: asm volatile("cp.async.wait_group 7;" ::: "memory"); break;
+  }
+}
+
 __device__ __forceinline__ void red_shared_add(int* p, int v) {
   asm volatile("red.shared.add.s32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
 }
@@ -95,6 +120,14 @@ __device__ __forceinline__ void red_shared_add(int* p, int v) {
 __device__ __forceinline__ int xs_chunk(int ch) { return ch ^ (((ch >> 3) & 1) << 1); }
 
 __device__ __forceinline__ int mma_row_to_box(int g) { return (g >> 1) | ((g & 1) << 2); }
+
+// Every CTA reads the whole of x; CTA b starts its 16-element chunks at a
+// different place (chunk i of a row is read as chunk (i + rot) % n), so the
+// 148 SMs do not ask the same L2 lines for the same bytes at the same moment.
+__device__ __forceinline__ int rotated(int ch, int n, int rot) {
+  const int c = ch + rot;
+  return c >= n ? c - n : c;
+}
 
 // largest |x| of 16 bf16 values, as bf16 bits (finite values order like bits & 0x7FFF)
 __device__ __forceinline__ uint32_t absmax16_bits(uint4 lo, uint4 hi) {
@@ -157,12 +190,12 @@ __device__ __forceinline__ int bytesum16(uint4 v, int sum) {
 }
 
 struct SmemTail {
-  uint64_t full[kWarps][kMaxRing];   // per warp: its ring slots' TMA barriers
   uint64_t stall;                    // never signalled (forced-timeout test hook)
   uint32_t amax[16];                 // absmax per token (bf16 bits)
   int rsum[16];                      // sum of q per token
   float sx[16];                      // s_x per token
   float swg[kMaxGroups];             // s_w of each row group
+  double rcp[16][kMaxGroups];        // 1 / d per token and row group (double)
   int failed;                        // a wait of this CTA timed out
 };
 
@@ -187,39 +220,34 @@ __host__ __device__ SmemLayout smem_layout(int M, int ring, size_t slot_bytes, i
 
 // The items of one warp, in order: round r, item j of the round (j = warp,
 // warp + 8, ...); item j is chunk group j / U of unit j % U.  A round's
-// groups are its full chunks in groups of kc (the last one maybe short: the
-// 3-D view zero-fills chunks >= F) and, in the round that holds it, the
-// partial last chunk as a group of its own.
+// chunks (the last one of K maybe partial) form groups of kc, the last group
+// maybe shorter.
 struct ItemCursor {
   int r, j;
-  __device__ __forceinline__ static int full_groups(int r, int F, int kc) {
-    const int fc = min(max(F - kRoundChunks * r, 0), kRoundChunks);
-    return (fc + kc - 1) / kc;
+  __device__ __forceinline__ static int chunks(int r, int nchunks) {
+    return min(nchunks - kRoundChunks * r, kRoundChunks);
   }
-  __device__ __forceinline__ static int groups(int r, int F, int kc, int tail) {
-    return full_groups(r, F, kc) + ((tail && F / kRoundChunks == r) ? 1 : 0);
-  }
-  __device__ __forceinline__ void settle(int warp, int nround, int F, int kc, int tail, int U) {
-    while (r < nround && j >= groups(r, F, kc, tail) * U) {
+  __device__ __forceinline__ static int groups(int r, int nchunks, int kc) { return (chunks(r, nchunks) + kc - 1) / kc; }
+  __device__ __forceinline__ void settle(int warp, int nround, int nchunks, int kc, int U) {
+    while (r < nround && j >= groups(r, nchunks, kc) * U) {
       ++r;
       j = warp;
     }
   }
-  __device__ __forceinline__ void start(int warp, int nround, int F, int kc, int tail, int U) {
+  __device__ __forceinline__ void start(int warp, int nround, int nchunks, int kc, int U) {
     r = 0;
     j = warp;
-    settle(warp, nround, F, kc, tail, U);
+    settle(warp, nround, nchunks, kc, U);
   }
-  __device__ __forceinline__ void next(int warp, int nround, int F, int kc, int tail, int U) {
+  __device__ __forceinline__ void next(int warp, int nround, int nchunks, int kc, int U) {
     j += kWarps;
-    settle(warp, nround, F, kc, tail, U);
+    settle(warp, nround, nchunks, kc, U);
   }
 };
 
 template <int NT>
 __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
-    decode_kernel(const __grid_constant__ CUtensorMap tm3, const __grid_constant__ CUtensorMap tm2,
-                  const DecodeArgs a) {
+    decode_kernel(const DecodeArgs a) {
   constexpr int NTOK = NT * 8;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -240,18 +268,13 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
   const int units_total = (N + kUnitRows - 1) / kUnitRows;
   const int u_begin = static_cast<int>(static_cast<long long>(blockIdx.x) * units_total / gridDim.x);
   const int U = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * units_total / gridDim.x) - u_begin;
-  const int F = K / kBoxK;                           // full 512-k chunks (the 3-D view's extent)
-  const int tail = (K % kBoxK) != 0;                 // a partial last chunk
+  const int nchunks = (K + kBoxK - 1) / kBoxK;       // 512-k chunks, the last maybe partial
   const int nround = (K + kChunkK - 1) / kChunkK;
+  const uint32_t row_bytes = static_cast<uint32_t>(K) / 4;
   uint8_t* wring = base + L.ring + static_cast<size_t>(warp) * ring * slot_bytes;   // this warp's ring
-  uint64_t* full = sm.full[warp];
 
-  if (lane == 0)
-    for (int s = 0; s < ring; ++s) mbar_init(&full[s], 1);
   if (threadIdx.x == 0) {
     mbar_init(&sm.stall, 1);
-    if (F > 0) tma_prefetch_desc(&tm3);
-    if (tail) tma_prefetch_desc(&tm2);
     sm.failed = 0;
   }
   fence_mbar_init();
@@ -262,40 +285,58 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
   for (int i = threadIdx.x; i < U * kUnitRows * NTOK; i += kThreads) acc_s[i] = 0;
   __syncthreads();
 
-  // ---- this warp's weight stream (lane 0 issues; every lane keeps the count)
+  // ---- this warp's weight stream: every lane copies its own 16-byte
+  // pieces of an item (row p >> 3, piece p & 7 of each 128-byte chunk row,
+  // p = lane, lane + 32, ...) into the slot's 128-byte-swizzled layout; one
+  // copy group per item; pieces beyond N or K are zero-filled
   ItemCursor ic;                                     // next item to issue
-  ic.start(warp, nround, F, kc, tail, U);
+  ic.start(warp, nround, nchunks, kc, U);
   int issued = 0;
   auto issue_next = [&]() {
-    if (ic.r >= nround) return;
-    if (lane == 0) {
+    if (ic.r < nround) {
       const int s = issued % ring;
       const int g = ic.j / U, u = ic.j - g * U;
-      const int row = (u_begin + u) * kUnitRows;
+      const int c0 = kRoundChunks * ic.r + g * kc;                 // first chunk of the item
+      const int nc = min(kc, ItemCursor::chunks(ic.r, nchunks) - g * kc);
       uint8_t* dst = wring + s * slot_bytes;
-      if (g < ItemCursor::full_groups(ic.r, F, kc)) {
-        mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(kc * kSubBytes));
-        tma_load_3d(dst, &tm3, &full[s], 0, row, kRoundChunks * ic.r + g * kc);
-      } else {
-        mbar_arrive_expect_tx(&full[s], kSubBytes);
-        tma_load_2d(dst, &tm2, &full[s], F * (kBoxK / 4), row);
+      for (int p = lane; p < nc * 128; p += 32) {
+        const int cc = p >> 7, r = (p >> 3) & 15, q = p & 7;
+        const int n = (u_begin + u) * kUnitRows + r;
+        const uint32_t off = static_cast<uint32_t>(c0 + cc) * (kBoxK / 4) + 16u * q;
+        const bool valid = n < N && off < row_bytes;
+        const uint8_t* src = a.packed + (valid ? static_cast<size_t>(n) * row_bytes + off : 0);
+        cp_async16(dst + cc * kSubBytes + r * 128 + ((q ^ (r & 7)) << 4), src, valid ? 16u : 0u);
       }
+      ++issued;
+      ic.next(warp, nround, nchunks, kc, U);
     }
-    ++issued;
-    ic.next(warp, nround, F, kc, tail, U);
+    cp_async_commit();                               // one group per call, empty when nothing is left
   };
-  if (a.weights_early)
+  // the bias and the scales are read into registers as early as they may be
+  // (with the weights when those are resident) and stored to shared memory
+  // only before the epilogue, so no thread waits for them on the way to x
+  uint16_t bvals[2] = {0, 0};
+  float swv = 0.0f;
+  auto load_params = [&]() {
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int i = threadIdx.x + k * kThreads;
+      const int n = u_begin * kUnitRows + i;
+      if (i < U * kUnitRows && a.bias && n < N) bvals[k] = a.bias[n];
+    }
+    if (threadIdx.x < a.ngroups) swv = a.w_scale[threadIdx.x];
+  };
+  if (a.weights_early) {
     for (int i = 0; i < ring; ++i) issue_next();
+    load_params();
+  }
 
   pdl_wait_primary();
-  if (!a.weights_early)
+  if (!a.weights_early) {
     for (int i = 0; i < ring; ++i) issue_next();
-  if (a.status && blockIdx.x == 0 && threadIdx.x == 0) *a.status = 0u;
-  for (int i = threadIdx.x; i < U * kUnitRows; i += kThreads) {
-    const int n = u_begin * kUnitRows + i;
-    bias_s[i] = (a.bias && n < N) ? a.bias[n] : static_cast<uint16_t>(0);
+    load_params();
   }
-  if (threadIdx.x < a.ngroups) sm.swg[threadIdx.x] = a.w_scale[threadIdx.x];
+  if (a.status && blockIdx.x == 0 && threadIdx.x == 0) *a.status = 0u;
 
   bool ok = true;
   const int g = lane >> 2, t = lane & 3;
@@ -303,6 +344,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
   // ---- per-token absmax over the whole row: warp w takes token(s)
   // m = w / P (+ 8 / P, ...) and a 1/P share of the row, P = max(1, 8 / M)
   const int cpr = K >> 4;                            // 16-element chunks per row
+  const int xrot = static_cast<int>((static_cast<unsigned>(blockIdx.x) * 97u) % static_cast<unsigned>(cpr));
   const int P = M >= kWarps ? 1 : kWarps / M;
   const int part = warp % P, mstep = kWarps / P;
   const int C = (cpr + 32 * P - 1) / (32 * P);       // chunks per lane per token
@@ -316,9 +358,10 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
     for (int i = 0; i < kHold * NT; ++i) {
       const int j = (NT == 2 && i >= C) ? 1 : 0;     // token slot of this warp
       const int m = warp / P + j * mstep;
-      const int ch = part * 32 + lane + (i - j * C) * 32 * P;
+      const int ch0 = part * 32 + lane + (i - j * C) * 32 * P;
+      const int ch = ch0 < cpr ? rotated(ch0, cpr, xrot) : ch0;
       v[i][0] = v[i][1] = make_uint4(0, 0, 0, 0);
-      if (i < NT * C && m < M && ch < cpr) {
+      if (i < NT * C && m < M && ch0 < cpr) {
         v[i][0] = __ldg(xrow0 + (static_cast<size_t>(m) * K >> 3) + 2 * ch);
         v[i][1] = __ldg(xrow0 + (static_cast<size_t>(m) * K >> 3) + 2 * ch + 1);
       }
@@ -357,8 +400,9 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
     for (int i = 0; i < kHold * NT; ++i) {
       const int j = (NT == 2 && i >= C) ? 1 : 0;
       const int m = warp / P + j * mstep;
-      const int ch = part * 32 + lane + (i - j * C) * 32 * P;
-      if (i < NT * C && m < M && ch < cpr) {
+      const int ch0 = part * 32 + lane + (i - j * C) * 32 * P;
+      const int ch = ch0 < cpr ? rotated(ch0, cpr, xrot) : ch0;
+      if (i < NT * C && m < M && ch0 < cpr) {
         int ps = 0;
         const uint4 qv = quant16(v[i][0], v[i][1], j ? sxr[NT - 1] : sxr[0], ps, a.faithful);
         if (j) sum[NT - 1] += ps;
@@ -382,9 +426,10 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
         uint4 v[kXB][2];
 #pragma unroll
         for (int j = 0; j < kXB; ++j) {
-          const int ch = ch0 + j * 32 * P;
+          const int chu = ch0 + j * 32 * P;
           v[j][0] = v[j][1] = make_uint4(0, 0, 0, 0);
-          if (ch < cpr) {
+          if (chu < cpr) {
+            const int ch = rotated(chu, cpr, xrot);
             v[j][0] = __ldg(row + 2 * ch);
             v[j][1] = __ldg(row + 2 * ch + 1);
           }
@@ -413,7 +458,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
 
   const int r0 = mma_row_to_box(g);                  // sub-box rows r0 and r0 + 8
   ItemCursor cc;                                     // next item to consume
-  cc.start(warp, nround, F, kc, tail, U);
+  cc.start(warp, nround, nchunks, kc, U);
   int consumed = 0;
   int xchunk = -1;                                   // round-local chunk of the x fragment held
   uint32_t xw[2][2][NT][8];                          // [v][pair][token tile][word]
@@ -433,16 +478,18 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
           uint4 v[kQB][2];
 #pragma unroll
           for (int j = 0; j < kQB; ++j) {
-            const int ch = ch0 + j * 32 * P;
-            if (ch < ccpr) {
+            const int chu = ch0 + j * 32 * P;
+            if (chu < ccpr) {
+              const int ch = rotated(chu, ccpr, xrot % ccpr);
               v[j][0] = __ldg(src + 2 * ch);
               v[j][1] = __ldg(src + 2 * ch + 1);
             }
           }
 #pragma unroll
           for (int j = 0; j < kQB; ++j) {
-            const int ch = ch0 + j * 32 * P;
-            if (ch < ccpr) {
+            const int chu = ch0 + j * 32 * P;
+            if (chu < ccpr) {
+              const int ch = rotated(chu, ccpr, xrot % ccpr);
               const uint4 qv = quant16(v[j][0], v[j][1], sxm, sum, a.faithful);
               if (blockIdx.x == 0 && a.xq_out) *reinterpret_cast<uint4*>(a.xq_out + roff + 16 * ch) = qv;
               *reinterpret_cast<uint4*>(xrow + 16 * xs_chunk(ch)) = qv;
@@ -475,15 +522,13 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
     // ---- this warp's items of round r
     while (ok && cc.r == r) {
       const int s = consumed % ring;
-      const bool got = mbar_wait(&full[s], (consumed / ring) & 1, a.wait_ns);
-      if (!__all_sync(0xffffffffu, got)) {
-        ok = false;
-        break;
-      }
+      // this item's copies (the oldest group in flight) have landed, for
+      // every lane of the warp
+      cp_async_wait(ring - 1);
+      __syncwarp();
       const int grp = cc.j / U, u = cc.j - grp * U;
-      const bool is3 = grp < ItemCursor::full_groups(r, F, kc);
-      const int first = is3 ? grp * kc : F - kRoundChunks * r;   // round-local chunk of the item's first sub-box
-      const int nsub = is3 ? min(kc, F - kRoundChunks * r - grp * kc) : 1;
+      const int first = grp * kc;                    // round-local chunk of the item's first sub-box
+      const int nsub = min(kc, ItemCursor::chunks(r, nchunks) - first);
       int acc[4][NT][4];
 #pragma unroll
       for (int i = 0; i < 4; ++i)
@@ -537,7 +582,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
       // the slot is read: refill it with this warp's next item
       __syncwarp();
       ++consumed;
-      cc.next(warp, nround, F, kc, tail, U);
+      cc.next(warp, nround, nchunks, kc, U);
       issue_next();
       // fields -> the unit's sums (4^i sum(c q) >> 2i is exact: at most 8 chunks
       // of 512 k per item keep 64 * 2 * 127 * 4096 below 2^31)
@@ -560,14 +605,28 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
       }
     }
   }
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int i = threadIdx.x + k * kThreads;
+    if (i < U * kUnitRows) bias_s[i] = bvals[k];
+  }
+  if (threadIdx.x < a.ngroups) sm.swg[threadIdx.x] = swv;
+  // every copy this thread issued has landed before the CTA exits
+  cp_async_wait(0);
   if (!ok) {
     report_status(a.status, kStatusTimeout);
-    if (lane == 0) {
-      sm.failed = 1;
-      // every load this warp issued lands before the CTA exits (fixed limit)
-      for (int q = consumed; q < issued; ++q) mbar_wait(&full[q % ring], (q / ring) & 1, kWaitLimitNs);
-    }
-    __syncwarp();
+    if (lane == 0) sm.failed = 1;
+  }
+  // d = s_x s_w per token and row group (on a bf16 module bf16(bf16(s_w) s_x)),
+  // kept as the double 1 / d: RN_f32(a * (1/d)) is RN_f32(a / d) for every
+  // float32 (or bf16) numerator a -- a quotient of two floats lies at least
+  // 2^-49 (relative) from every float32 midpoint, and the double product is
+  // within 2^-52 of it
+  __syncthreads();                                   // s_w stored by its threads
+  if (threadIdx.x < M * a.ngroups) {
+    const int m = threadIdx.x / a.ngroups, gg = threadIdx.x - m * a.ngroups;
+    const float d = a.faithful ? bf16_round(__fmul_rn(bf16_round(sm.swg[gg]), sm.sx[m])) : __fmul_rn(sm.sx[m], sm.swg[gg]);
+    sm.rcp[m][gg] = __drcp_rn(static_cast<double>(d));
   }
   __syncthreads();
 
@@ -582,15 +641,14 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
 #pragma unroll
     for (int gg = 0; gg + 1 < kMaxGroups; ++gg) gi += (gg + 1 < a.ngroups && n >= a.group_end[gg]) ? 1 : 0;
     float y32;
+    const double r = sm.rcp[m][gi];
     if (!a.faithful) {
-      const float d = __fmul_rn(sm.sx[m], sm.swg[gi]);
-      y32 = __fdiv_rn(static_cast<float>(accv), d);
+      y32 = __double2float_rn(static_cast<double>(static_cast<float>(accv)) * r);
       if (a.bias) y32 = __fadd_rn(y32, bf16_bits_to_f32(bias_s[rl]));
     } else {
       // bf16 module: F.linear's sum, the scale product, the quotient and the
       // bias add are each a bf16 tensor
-      const float d = bf16_round(__fmul_rn(bf16_round(sm.swg[gi]), sm.sx[m]));
-      y32 = bf16_round(__fdiv_rn(bf16_round(static_cast<float>(accv)), d));
+      y32 = bf16_round(__double2float_rn(static_cast<double>(bf16_round(static_cast<float>(accv))) * r));
       if (a.bias) y32 = bf16_round(__fadd_rn(y32, bf16_bits_to_f32(bias_s[rl])));
     }
     const size_t o = static_cast<size_t>(m) * N + n;
@@ -601,8 +659,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
 }
 
 template <int NT>
-cudaError_t launch_nt(const CUtensorMap& tm3, const CUtensorMap& tm2, const DecodeArgs& a, const DecodePlan& p,
-                      cudaStream_t stream) {
+cudaError_t launch_nt(const DecodeArgs& a, const DecodePlan& p, cudaStream_t stream) {
   auto kern = decode_kernel<NT>;
   static unsigned long long attr_done = 0;        // one bit per device
   cudaError_t ea = set_smem_attr_once(kern, 227 * 1024, &attr_done);
@@ -617,16 +674,19 @@ cudaError_t launch_nt(const CUtensorMap& tm3, const CUtensorMap& tm2, const Deco
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, tm3, tm2, a);
+  return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
 }  // namespace
 
+// Items of 2 chunks (4 KB) and 2 items in flight per warp: 64 KB in flight per
+// CTA.  A streaming probe on B200 (chained launches, all SMs) found this as
+// fast as any deeper ring at every decode shape, and 128 KB per CTA slower.
 #ifndef BITLINEAR_DECODE_KC
-#define BITLINEAR_DECODE_KC 2       // chunks (2 KB sub-boxes) per TMA load
+#define BITLINEAR_DECODE_KC 2       // chunks (2 KB each) per item
 #endif
 #ifndef BITLINEAR_DECODE_RING
-#define BITLINEAR_DECODE_RING 8     // largest ring per warp
+#define BITLINEAR_DECODE_RING 2     // largest ring per warp
 #endif
 
 DecodePlan plan_decode(int M, int N, int K, int num_sms) {
@@ -635,9 +695,9 @@ DecodePlan plan_decode(int M, int N, int K, int num_sms) {
   p.grid = units_total < num_sms ? units_total : num_sms;
   if ((units_total + p.grid - 1) / p.grid > kMaxUnits) p.grid = (units_total + kMaxUnits - 1) / kMaxUnits;
   p.units_max = (units_total + p.grid - 1) / p.grid;
-  const int F = K / kBoxK;
-  // loads of kc chunks when there are full chunks to group, else one chunk
-  p.kc = F >= 2 * BITLINEAR_DECODE_KC ? BITLINEAR_DECODE_KC : 1;
+  const int nchunks = (K + kBoxK - 1) / kBoxK;
+  // items of kc chunks when K has that many, else one chunk
+  p.kc = nchunks >= 2 * BITLINEAR_DECODE_KC ? BITLINEAR_DECODE_KC : 1;
   p.tail = (K % kBoxK) != 0;
   p.slot_bytes = static_cast<size_t>(p.kc) * kSubBytes;
   // shared-memory budget: two CTAs per SM for the 8-token kernel (the next
@@ -665,24 +725,7 @@ cudaError_t launch_decode(DecodeArgs a, int num_sms, cudaStream_t stream) {
   a.kc = p.kc;
   a.tail = p.tail;
   if (p.smem > 227 * 1024) return cudaErrorInvalidValue;
-  // 2-D view [N][K/4] bytes: the partial last chunk (and the 3-D map's stand-in when K < 512)
-  CUtensorMap tm2, tm3;
-  if (!encode_2d_u8(&tm2, a.packed, static_cast<uint64_t>(a.K) / 4, static_cast<uint64_t>(a.N),
-                    static_cast<uint64_t>(a.K) / 4, kBoxK / 4, kUnitRows, CU_TENSOR_MAP_SWIZZLE_128B))
-    return cudaErrorInvalidValue;
-  tm3 = tm2;
-  if (a.K >= kBoxK) {
-    // 3-D view [full chunk][row][128 bytes]: a box is kc consecutive 512-k
-    // chunks of 16 rows, each chunk landing as its own 16 x 128-byte sub-box
-    const uint64_t dims[3] = {static_cast<uint64_t>(kBoxK / 4), static_cast<uint64_t>(a.N),
-                              static_cast<uint64_t>(a.K / kBoxK)};
-    const uint64_t strides[2] = {static_cast<uint64_t>(a.K) / 4, static_cast<uint64_t>(kBoxK / 4)};
-    const uint32_t box[3] = {static_cast<uint32_t>(kBoxK / 4), static_cast<uint32_t>(kUnitRows),
-                             static_cast<uint32_t>(p.kc)};
-    if (!encode_3d_u8(&tm3, a.packed, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
-      return cudaErrorInvalidValue;
-  }
-  return a.M <= 8 ? launch_nt<1>(tm3, tm2, a, p, stream) : launch_nt<2>(tm3, tm2, a, p, stream);
+  return a.M <= 8 ? launch_nt<1>(a, p, stream) : launch_nt<2>(a, p, stream);
 }
 
 }  // namespace bitlinear

@@ -15,10 +15,6 @@ int current_device_status();
 // ---- TMA tensor maps (tensor_map.cu) ---------------------------------------
 bool encode_2d_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
                   uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle);
-// 3-D map: dims[0] innermost (contiguous bytes), strides in bytes of dims 1
-// and 2 (multiples of 16), box dims <= 256 each.
-bool encode_3d_u8(CUtensorMap* map, const void* base, const uint64_t dims[3], const uint64_t strides[2],
-                  const uint32_t box[3], CUtensorMapSwizzle swizzle);
 
 // ---- activation quantisation (act_quant.cu) --------------------------------
 // pdl: launch as a programmatic dependent of the previous kernel on the stream

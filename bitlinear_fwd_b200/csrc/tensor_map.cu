@@ -1,4 +1,4 @@
-// Host-side encoding of 2-D and 3-D TMA tensor maps over byte arrays, through the
+// Host-side encoding of 2-D TMA tensor maps over byte arrays, through the
 // driver entry point obtained from the runtime (no link against libcuda).
 #include <cudaTypedefs.h>
 
@@ -32,19 +32,6 @@ bool encode_2d_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t o
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estr[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-bool encode_3d_u8(CUtensorMap* map, const void* base, const uint64_t dims[3], const uint64_t strides[2],
-                  const uint32_t box[3], CUtensorMapSwizzle swizzle) {
-  auto fn = get_encode_fn();
-  if (!fn) return false;
-  const cuuint64_t d[3] = {dims[0], dims[1], dims[2]};
-  const cuuint64_t st[2] = {strides[0], strides[1]};
-  const cuuint32_t bx[3] = {box[0], box[1], box[2]};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), d, st, bx, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
