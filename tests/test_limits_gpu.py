@@ -73,6 +73,12 @@ def _large_acc_inputs(M):
     w[2] = torch.where(torch.arange(K_MAX) % 3 == 0, -1.0, 1.0) * (1.0 + w[2] * 0.1)
     w[3] = 1.0 + w[3] * 0.1
     w[3, : K_MAX // 2] = 0.0
+    # rows 4..10: constant sign (alternating +, -) with the first r - 3 weights
+    # zeroed, so their sums differ from row 0's by a few small q values and
+    # some of them are odd (float(acc) then rounds)
+    for r in range(4, 11):
+        w[r] = (1.0 if r % 2 == 0 else -1.0) + w[r] * 0.1
+        w[r, : r - 3] = 0.0
     x = synth.normal_f32(SEED, 2, (M, K_MAX), 0.1).abs() + 0.6
     x[0, 7] = 2.0                              # one larger value: q = round(x * 63.5)
     return x.to(torch.bfloat16), w, synth.normal_bf16(SEED, 3, (N_K,), 0.01)
@@ -96,7 +102,7 @@ def test_k_max_accumulators_beyond_2_24(large_k_weights, M, engine):
     ref = oracle.forward(synth.bf16_bits(x), opk, osw, synth.bf16_bits(bias))
     # the case this test exists for: numerators that float32 cannot hold exactly
     big = np.abs(ref["acc"]) > (1 << 24)
-    assert big.sum() >= 2 * M, "the inputs must drive |acc| past 2^24 (rows 0 and 1 for every token)"
+    assert big.sum() >= 8 * M, "the inputs must drive |acc| past 2^24 (rows 0, 1 and 4..10 for every token)"
     assert np.any(ref["acc"][big] % 2 != 0), "some of them must be odd, so that float(acc) rounds"
     out = bl.bitlinear_forward_debug(x.cuda(), packed, s_w, bias.cuda(), engine=engine)
     torch.cuda.synchronize()
