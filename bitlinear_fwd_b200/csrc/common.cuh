@@ -103,6 +103,12 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 // ---------------------------------------------------------------------------
 // TMA (no multicast)
 // ---------------------------------------------------------------------------
+// Brings a global line into L2 (not L1): safe on data the previous kernel of
+// the stream may still write, since L2 is the point of coherence.
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -124,6 +130,19 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
       : "memory");
 }
+
+// Shared -> global tile store (TMA); the bulk group of this thread tracks it.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* smem_src, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(smem_src)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// the shared memory of every committed bulk store of this thread has been read
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// every committed bulk store of this thread has completed
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // ---------------------------------------------------------------------------
 // tcgen05: tensor memory and the 5th-generation tensor core
@@ -245,6 +264,13 @@ __device__ __forceinline__ float bf16_bits_to_f32(uint32_t bits16) {
 }
 __device__ __forceinline__ uint16_t f32_to_bf16_bits(float v) {
   return __bfloat16_as_ushort(__float2bfloat16_rn(v));
+}
+// The same rounding in integer instructions (no conversion unit): RNE on the
+// bits of a number, the canonical NaN for a NaN.
+__device__ __forceinline__ uint16_t f32_to_bf16_bits_alu(float v) {
+  const uint32_t b = __float_as_uint(v);
+  const uint32_t r = (b + 0x7FFFu + ((b >> 16) & 1u)) >> 16;
+  return static_cast<uint16_t>((b & 0x7FFFFFFFu) > 0x7F800000u ? 0x7FFFu : r);
 }
 // v rounded to bfloat16 (RNE) and widened back: one bf16 tensor op's result
 __device__ __forceinline__ float bf16_round(float v) { return bf16_bits_to_f32(f32_to_bf16_bits(v)); }

@@ -7,39 +7,47 @@
 // tokens are the B operand and come from shared memory:
 //   D[weight row n][token m] += A[n][k] * B[m][k],  M_mma = 128 weight rows,
 //   N_mma = BT = 192 tokens, K = 32 per instruction.
-// Tile shape.  Per 128-k block the shared memory of an SM carries the x tile
-// twice (written by TMA, read by the MMA) plus the 2-bit codes; with 192
-// tokens that is 56 KB against 384 cycles of MMA, where 128 tokens would be
-// 40 KB against 256 cycles: the wider tile moves fewer bytes per MMA cycle.
+// Tile shape.  Per 128 k the shared memory of an SM carries the x tile twice
+// (written by TMA, read by the MMA) plus the 2-bit codes; with 192 tokens
+// that is 56 KB against 384 cycles of MMA, where 128 tokens would be 40 KB
+// against 256 cycles: the wider tile moves fewer bytes per MMA cycle.
 // Tensor memory holds two 192-column accumulators (the epilogue of one tile
-// runs while the MMAs of the next one fill the other) and four 32-column
+// runs while the MMAs of the next one fill the other) and two 64-column
 // stages of unpacked weights: 512 columns.
+// Stages of 256 k.  The MMA warp waits once and commits twice per stage, so
+// a stage carries eight MMAs: a loop of four MMAs between one wait and two
+// commits ran at 78% of the tensor rate on B200, eight at 100%.
 // Persistent kernel: one CTA per SM walks the 128 x 192 tiles (weight tile
-// fastest, so the CTAs running at the same time share the token tile in L2),
-// k-blocks of 128, with a 6-stage operand ring in shared memory:
-//   warp 0       TMA producer: x tile (192 tokens x 128 int8, 128-byte
-//                swizzle) + packed weight tile (128 rows x 32 bytes) per stage
-//   warp 1       MMA issuer: 4 x tcgen05.mma.kind::i8 per k-block, A from
-//                tensor-memory stage (k-block & 3), into accumulator buffer
-//                (tile & 1); commits free the shared stage and the A stage
+// fastest, so the CTAs running at the same time share the token tile in L2)
+// through a 3-stage operand ring in shared memory:
+//   warp 0       TMA producer: x tile (192 tokens x 256 int8 as two
+//                128-byte-swizzled boxes of 128 k) + packed weight tile (128
+//                rows x 64 bytes, 64-byte swizzle) per stage
+//   warp 1       MMA issuer: 8 x tcgen05.mma.kind::i8 per stage (4 when its
+//                second half lies beyond K), A from tensor-memory stage
+//                (stage & 1), into accumulator buffer (tile & 1); commits free
+//                the shared stage and the A stage
 //   warp 2       tensor-memory allocation
-//   warps 4..7   weight unpack: thread = weight row; its 32 packed bytes become
-//                32 registers of codes c = u + 1 (one word -> four registers
-//                of four consecutive k) and one tcgen05.st of 32 columns; a
-//                quarter-warp reads its 16-byte pieces in an order that keeps
-//                them in distinct banks
+//   warps 4..7   weight unpack: thread = weight row; its 64 packed bytes become
+//                64 registers of codes c = u + 1 (one word -> four registers
+//                of four consecutive k) and two tcgen05.st of 32 columns; the
+//                swizzled rows keep a quarter-warp's reads in distinct banks
 //   warps 8..15  epilogue of the previous tile while the MMAs of the next one
 //                run; warps w and w + 4 share a lane quarter of tensor memory
 //                and take one half of the tile's tokens each: tcgen05.ld of a
 //                row's 96 accumulators (the next 32 columns load while 32 are
 //                processed), acc - sum_k q (code offset), y = acc / (s_x s_w)
-//                (+ bias), bf16 stores (coalesced along weight rows); s_w is
-//                the scale of the row's group (stacked layers)
+//                (+ bias) as a product with the double 1 / (s_x s_w) of the
+//                token, bf16 into a shared staging tile that one thread
+//                stores with TMA (plain stores when y's rows are not 16-byte
+//                multiples or a debug output is asked for); s_w is the scale
+//                of the row's group (stacked layers)
 // Barriers: per shared stage full (TMA bytes landed) and empty (MMAs done);
 // per A stage ready (written) and afree (MMAs done); per accumulator buffer
 // acc_full (tile's MMAs done) and acc_empty (epilogue has read it).
 // Out-of-range rows/columns are zero-filled by TMA, so a code 0 or an
-// activation 0 adds nothing; the epilogue masks rows >= N and tokens >= M.
+// activation 0 adds nothing; the epilogue masks rows >= N and tokens >= M
+// (the tile store clips them).
 // Every wait is bounded in time; a wait that gives up sets the status word,
 // and the CTA drains its copies and MMAs (with the fixed 1 s limit) before
 // freeing tensor memory.
@@ -54,24 +62,28 @@ namespace {
 #endif
 constexpr int BW = 128;                      // weight rows per tile (MMA M)
 constexpr int BT = BITLINEAR_GEMM_BT;        // tokens per tile (MMA N)
-constexpr int BK = 128;                      // k per block
-constexpr int STAGES = 6;                    // shared-memory operand stages
-constexpr int ASTAGES = 4;                   // tensor-memory stages of unpacked weights
+constexpr int BK = 256;                      // k per block (stage)
+constexpr int STAGES = 3;                    // shared-memory operand stages
+constexpr int ASTAGES = 2;                   // tensor-memory stages of unpacked weights
 constexpr int kThreads = 512;
 constexpr int kEpiWarps = 8;                 // two per tensor-memory lane quarter
 constexpr int kEpiCols = BT / 2;             // tokens of a tile per epilogue warp
 constexpr int kEpiChunks = kEpiCols / 32;
-constexpr uint32_t kXBytes = BT * BK;        // x tile per stage
-constexpr uint32_t kWpBytes = BW * BK / 4;   // 4 KB packed weights per stage
+constexpr uint32_t kXHalf = BT * 128;        // one 128-k half of the x tile (a 128-byte-swizzled TMA box)
+constexpr uint32_t kXBytes = 2 * kXHalf;     // x tile per stage
+constexpr uint32_t kWpBytes = BW * BK / 4;   // 8 KB packed weights per stage (64-byte-swizzled rows)
 constexpr uint32_t kACols = BK / 4;          // tensor-memory columns of one A stage
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kCodeMask = 0x03030303u;
 static_assert(BT % 64 == 0 && BT <= 256, "two halves of whole 32-column chunks; MMA N <= 256");
 static_assert(2 * BT + ASTAGES * kACols <= kTmemCols, "two accumulators and the A stages fit in tensor memory");
+static_assert(kXHalf % 1024 == 0 && kWpBytes % 512 == 0, "swizzle atoms stay aligned");
 
+constexpr uint32_t kStageBytes = BT * BW * 2;          // bf16 y tile [BT tokens][BW rows] for the TMA store
 constexpr uint32_t kOffX = 0;
 constexpr uint32_t kOffWp = kOffX + STAGES * kXBytes;
-constexpr uint32_t kOffD = kOffWp + STAGES * kWpBytes;       // per token: 1 / d in double [BT], or s_x
+constexpr uint32_t kOffStage = (kOffWp + STAGES * kWpBytes + 1023) & ~1023u;
+constexpr uint32_t kOffD = kOffStage + kStageBytes;          // per token: 1 / d in double [BT], or s_x
 constexpr uint32_t kOffRs = kOffD + 8 * BT;                  // row sums per token [BT]
 constexpr uint32_t kOffBar = kOffRs + 4 * BT;
 constexpr uint32_t kSmemBytes = kOffBar + 512 + 1024;        // + barriers, alignment slack
@@ -81,10 +93,12 @@ constexpr uint32_t kSmemBytes = kOffBar + 512 + 1024;        // + barriers, alig
 // kernel of the library allocates tensor memory beside it (the int8 rate
 // measurement runs on its own).
 static_assert(2 * kSmemBytes > 228 * 1024, "one GEMM CTA per SM keeps the 512-column allocation uncontended");
+static_assert(kSmemBytes <= 227 * 1024, "fits the shared memory of one CTA");
+static_assert(kOffD % 16 == 0 && kOffRs % 16 == 0, "per-token values are read as 16-byte vectors");
 
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_prefill_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
-                        const ForwardArgs a) {
+                        const __grid_constant__ CUtensorMap tm_y, const ForwardArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kOffBar);
@@ -101,6 +115,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   double* rcp_s = reinterpret_cast<double*>(smem + kOffD);   // per token, when the tile has one scale
   float* sx_s = reinterpret_cast<float*>(smem + kOffD);      // per token s_x, when it has several
   int* rs_s = reinterpret_cast<int*>(smem + kOffRs);
+  uint16_t* stage = reinterpret_cast<uint16_t*>(smem + kOffStage);   // y tile, token-major
   const uint64_t wait_ns = a.wait_ns;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -128,6 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tm_x);
     tma_prefetch_desc(&tm_w);
+    if (a.y_tma) tma_prefetch_desc(&tm_y);
   }
   if (warp == 2) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -159,7 +175,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             pdl_wait_primary();
             waited = true;
           }
+          // two 128-k halves (a half beyond K arrives zero-filled)
           tma_load_2d(smem + kOffX + s * kXBytes, &tm_x, &full[s], kb * BK, m0);
+          tma_load_2d(smem + kOffX + s * kXBytes + kXHalf, &tm_x, &full[s], kb * BK + 128, m0);
         }
       }
       // drain: the last copy issued into each stage has landed.  The drain
@@ -199,10 +217,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           const uint32_t x_addr = smem_u32(smem + kOffX + s * kXBytes);
+          // eight MMAs per stage, four when its second half lies beyond K
+          const int nmma = kb * BK + 128 < a.K ? 8 : 4;
 #pragma unroll
-          for (int jj = 0; jj < BK / 32; ++jj)
-            umma_i8_ts(tmem_d, tmem_a + as * kACols + 8 * jj, umma_desc_sw128(x_addr + 32 * jj), idesc,
-                       (kb | jj) != 0);
+          for (int jj = 0; jj < 8; ++jj)
+            if (jj < nmma)
+              umma_i8_ts(tmem_d, tmem_a + as * kACols + 8 * jj,
+                         umma_desc_sw128(x_addr + (jj >> 2) * kXHalf + 32 * (jj & 3)), idesc, (kb | jj) != 0);
           umma_commit(&empty[s]);                 // the shared stage can be refilled
           umma_commit(&afree[as]);                // the A stage can be rewritten
         }
@@ -222,10 +243,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;
     const int row = 32 * q + lane;
     const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
-    // lanes 4..7 of every quarter-warp read their second 16-byte piece first:
-    // rows are 32 bytes apart, so the eight pieces of one access then fall in
-    // eight different 4-bank groups
-    const int first = (lane >> 2) & 1;
+    // The weight rows are 64 bytes with TMA's 64-byte swizzle: 16-byte piece
+    // p of row r sits at piece p ^ ((r >> 1) & 3), so the eight rows of a
+    // quarter-warp read piece p from eight different 4-bank groups.
+    const int sw = (row >> 1) & 3;
     int g = 0;
     for (int tile = blockIdx.x; tile < ntiles && !*failed; tile += gridDim.x) {
       for (int kb = 0; kb < num_kb; ++kb, ++g) {
@@ -236,20 +257,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           *failed = 1;
           break;
         }
-        const uint4* wp = reinterpret_cast<const uint4*>(smem + kOffWp + s * kWpBytes + row * 32);
-        const uint4 pa = wp[first], pb = wp[first ^ 1];
-        const uint4 p0 = first ? pb : pa, p1 = first ? pa : pb;
-        const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-        uint32_t codes[32];
+        const uint4* wp = reinterpret_cast<const uint4*>(smem + kOffWp + s * kWpBytes + row * 64);
+        uint4 pc[4];
 #pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {          // word jj = k 16jj .. 16jj + 15 of the block
-          codes[4 * jj + 0] = w[jj] & kCodeMask;
-          codes[4 * jj + 1] = (w[jj] >> 2) & kCodeMask;
-          codes[4 * jj + 2] = (w[jj] >> 4) & kCodeMask;
-          codes[4 * jj + 3] = (w[jj] >> 6) & kCodeMask;
-        }
+        for (int p = 0; p < 4; ++p) pc[p] = wp[p ^ sw];
         tc_fence_after();
-        tmem_st_32x32b_x32(tmem_a + lane_base + as * kACols, codes);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {             // k 128h .. 128h + 127: 32 columns
+          const uint32_t w[8] = {pc[2 * h].x, pc[2 * h].y, pc[2 * h].z, pc[2 * h].w,
+                                 pc[2 * h + 1].x, pc[2 * h + 1].y, pc[2 * h + 1].z, pc[2 * h + 1].w};
+          uint32_t codes[32];
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) {        // word jj = k 16jj .. 16jj + 15 of the half
+            codes[4 * jj + 0] = w[jj] & kCodeMask;
+            codes[4 * jj + 1] = (w[jj] >> 2) & kCodeMask;
+            codes[4 * jj + 2] = (w[jj] >> 4) & kCodeMask;
+            codes[4 * jj + 3] = (w[jj] >> 6) & kCodeMask;
+          }
+          tmem_st_32x32b_x32(tmem_a + lane_base + as * kACols + 32 * h, codes);
+        }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -267,9 +293,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int g = 0; g < kMaxGroups; ++g) swg[g] = g < a.ngroups ? a.w_scale[g] : 0.0f;
     int j = 0;
-    // The eight epilogue warps meet at a named barrier twice per tile; every
-    // one of them runs every iteration (a failure only skips work), so the
-    // barrier always gets its 256 threads.
+    // acc = sum(c q) - sum(q) is exact in float32 and double below 2^24,
+    // |acc| <= 127 K: such a K takes the conversion-free path
+    const bool small_k = a.K <= (1 << 17);
+    // The eight epilogue warps meet at named barriers (1 twice, 2 once per
+    // tile); every one of them runs every iteration (a failure only skips
+    // work), so the barriers always get their 256 threads.
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++j) {
       const int b = j & 1;
       const int n0 = (tile % wtiles) * BW, m0 = (tile / wtiles) * BT;
@@ -287,6 +316,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int g = 1; g < kMaxGroups; ++g)
         if (g == g0) sw_tile = swg[g];
+      // the previous tile's TMA store has read the staging buffer
+      if (a.y_tma && et == 0) bulk_wait_read_all();
       // per-token s_x and row sums of this tile
       asm volatile("bar.sync 1, 256;" ::: "memory");   // previous tile's readers are done
       if (et < BT) {
@@ -309,91 +340,127 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = !__any_sync(0xffffffffu, *failed != 0);
       if (ok) ok = mbar_wait(&acc_full[b], (j >> 1) & 1, wait_ns);
       ok = __all_sync(0xffffffffu, ok);             // warp-uniform decision
-      if (!ok) {
-        *failed = 1;
-        continue;
-      }
-      tc_fence_after();
-      const int n = n0 + 32 * q + lane;
+      if (!ok) *failed = 1;
+      const int row = 32 * q + lane;                // row of the tile
+      const int n = n0 + row;
       const bool nv = n < a.N;
-      const float bv = (a.bias && nv) ? bf16_bits_to_f32(a.bias[n]) : 0.0f;
-      float s_w = swg[0];                          // this row's group scale (tiles with several)
+      if (ok) {
+        tc_fence_after();
+        const float bv = (a.bias && nv) ? bf16_bits_to_f32(a.bias[n]) : 0.0f;
+        float s_w = swg[0];                        // this row's group scale (tiles with several)
 #pragma unroll
-      for (int g = 1; g < kMaxGroups; ++g)
-        if (g < a.ngroups && n >= a.group_end[g - 1]) s_w = swg[g];
-      if (a.faithful) s_w = bf16_round(s_w);       // a bf16 module holds s_w in bf16
-      auto emit = [&](int mi, int accv, float y32) {
-        const size_t o = static_cast<size_t>(m0 + mi) * a.N + n;
-        if (a.y) a.y[o] = f32_to_bf16_bits(y32);
-        if (a.acc_out) a.acc_out[o] = accv;
-        if (a.y32_out) a.y32_out[o] = y32;
-      };
-      auto process = [&](const uint32_t (&r)[32], int c) {
-        if (!nv) return;
-        if (uniform && !a.faithful) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int mi = 32 * c + i;
-            if (m0 + mi >= a.M) continue;
-            const int accv = static_cast<int>(r[i]) - rs_s[mi];
-            float y32 = __double2float_rn(static_cast<double>(static_cast<float>(accv)) * rcp_s[mi]);
-            if (a.bias) y32 = __fadd_rn(y32, bv);
-            emit(mi, accv, y32);
+        for (int g = 1; g < kMaxGroups; ++g)
+          if (g < a.ngroups && n >= a.group_end[g - 1]) s_w = swg[g];
+        if (a.faithful) s_w = bf16_round(s_w);     // a bf16 module holds s_w in bf16
+        auto emit = [&](int mi, int accv, float y32) {
+          if (a.y_tma) {
+            stage[mi * BW + row] = f32_to_bf16_bits_alu(y32);   // tokens >= M are clipped by the store
+            return;
           }
-        } else if (uniform) {
-          // bf16 module: the sum, the quotient and the bias add are each
-          // rounded to bf16 (the scale product is in rcp_s)
+          if (m0 + mi >= a.M) return;
+          const size_t o = static_cast<size_t>(m0 + mi) * a.N + n;
+          if (a.y) a.y[o] = f32_to_bf16_bits(y32);
+          if (a.acc_out) a.acc_out[o] = accv;
+          if (a.y32_out) a.y32_out[o] = y32;
+        };
+        auto process = [&](const uint32_t (&r)[32], int c) {
+          if (!nv) return;
+          if (uniform && !a.faithful && small_k) {
+            // per-token values as 16-byte vectors, 4 tokens at a time; the
+            // int32 -> double conversion by the 1.5 * 2^52 + 2^31 bias
+            // (exact for every int32), one rounding double -> float
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int mi = 32 * c + i;
-            if (m0 + mi >= a.M) continue;
-            const int accv = static_cast<int>(r[i]) - rs_s[mi];
-            float y32 = bf16_round(__double2float_rn(static_cast<double>(bf16_round(static_cast<float>(accv))) * rcp_s[mi]));
-            if (a.bias) y32 = bf16_round(__fadd_rn(y32, bv));
-            emit(mi, accv, y32);
-          }
-        } else if (!a.faithful) {
+            for (int i4 = 0; i4 < 32; i4 += 4) {
+              const int mb = 32 * c + i4;
+              const int4 rs = *reinterpret_cast<const int4*>(rs_s + mb);
+              const double2 rc01 = *reinterpret_cast<const double2*>(rcp_s + mb);
+              const double2 rc23 = *reinterpret_cast<const double2*>(rcp_s + mb + 2);
+              const int rsv[4] = {rs.x, rs.y, rs.z, rs.w};
+              const double rcv[4] = {rc01.x, rc01.y, rc23.x, rc23.y};
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int mi = 32 * c + i;
-            if (m0 + mi >= a.M) continue;
-            const int accv = static_cast<int>(r[i]) - rs_s[mi];
-            float y32 = __fdiv_rn(static_cast<float>(accv), __fmul_rn(sx_s[mi], s_w));
-            if (a.bias) y32 = __fadd_rn(y32, bv);
-            emit(mi, accv, y32);
-          }
-        } else {
+              for (int i = 0; i < 4; ++i) {
+                const int accv = static_cast<int>(r[i4 + i]) - rsv[i];
+                const double num = __hiloint2double(0x43380000, accv ^ static_cast<int>(0x80000000u)) -
+                                   6755401588539392.0;
+                float y32 = __double2float_rn(num * rcv[i]);
+                if (a.bias) y32 = __fadd_rn(y32, bv);
+                emit(mb + i, accv, y32);
+              }
+            }
+          } else if (uniform && !a.faithful) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int mi = 32 * c + i;
-            if (m0 + mi >= a.M) continue;
-            const int accv = static_cast<int>(r[i]) - rs_s[mi];
-            float y32 = bf16_round(__fdiv_rn(bf16_round(static_cast<float>(accv)), bf16_round(__fmul_rn(s_w, sx_s[mi]))));
-            if (a.bias) y32 = bf16_round(__fadd_rn(y32, bv));
-            emit(mi, accv, y32);
+            for (int i = 0; i < 32; ++i) {
+              const int mi = 32 * c + i;
+              const int accv = static_cast<int>(r[i]) - rs_s[mi];
+              float y32 = __double2float_rn(static_cast<double>(static_cast<float>(accv)) * rcp_s[mi]);
+              if (a.bias) y32 = __fadd_rn(y32, bv);
+              emit(mi, accv, y32);
+            }
+          } else if (uniform) {
+            // bf16 module: the sum, the quotient and the bias add are each
+            // rounded to bf16 (the scale product is in rcp_s)
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int mi = 32 * c + i;
+              const int accv = static_cast<int>(r[i]) - rs_s[mi];
+              float y32 = bf16_round(__double2float_rn(static_cast<double>(bf16_round(static_cast<float>(accv))) * rcp_s[mi]));
+              if (a.bias) y32 = bf16_round(__fadd_rn(y32, bv));
+              emit(mi, accv, y32);
+            }
+          } else if (!a.faithful) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int mi = 32 * c + i;
+              const int accv = static_cast<int>(r[i]) - rs_s[mi];
+              float y32 = __fdiv_rn(static_cast<float>(accv), __fmul_rn(sx_s[mi], s_w));
+              if (a.bias) y32 = __fadd_rn(y32, bv);
+              emit(mi, accv, y32);
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int mi = 32 * c + i;
+              const int accv = static_cast<int>(r[i]) - rs_s[mi];
+              float y32 = bf16_round(__fdiv_rn(bf16_round(static_cast<float>(accv)), bf16_round(__fmul_rn(s_w, sx_s[mi]))));
+              if (a.bias) y32 = bf16_round(__fadd_rn(y32, bv));
+              emit(mi, accv, y32);
+            }
           }
+        };
+        // the next 32 columns load while the current ones are processed; once
+        // the last load has landed the whole accumulator half is in registers
+        // and the buffer goes back to the MMA warp
+        const uint32_t col0 = tmem_base + b * BT + lane_base + 32 * (half * kEpiChunks);
+        uint32_t r0[32], r1[32];
+        tmem_ld_32x32b_x32(col0, r0);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < kEpiChunks; ++c) {
+          const bool last = c + 1 == kEpiChunks;
+          if (!last) tmem_ld_32x32b_x32(col0 + 32 * (c + 1), (c & 1) ? r0 : r1);
+          if (last) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[b]);
+          }
+          process((c & 1) ? r1 : r0, half * kEpiChunks + c);
+          if (!last) tmem_wait_ld();
         }
-      };
-      // the next 32 columns load while the current ones are processed; once
-      // the last load has landed the whole accumulator half is in registers
-      // and the buffer goes back to the MMA warp
-      const uint32_t col0 = tmem_base + b * BT + lane_base + 32 * (half * kEpiChunks);
-      uint32_t r0[32], r1[32];
-      tmem_ld_32x32b_x32(col0, r0);
-      tmem_wait_ld();
-#pragma unroll
-      for (int c = 0; c < kEpiChunks; ++c) {
-        const bool last = c + 1 == kEpiChunks;
-        if (!last) tmem_ld_32x32b_x32(col0 + 32 * (c + 1), (c & 1) ? r0 : r1);
-        if (last) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[b]);
+      }
+      if (a.y_tma) {
+        // every epilogue thread's staging writes are visible to the async
+        // proxy; then one thread stores the tile (rows >= N and tokens >= M
+        // are clipped by the tensor map's bounds)
+        fence_proxy_async_smem();
+        asm volatile("bar.sync 2, 256;" ::: "memory");
+        if (et == 0 && !*failed) {
+          tma_store_2d(&tm_y, stage, n0, m0);
+          bulk_commit();
         }
-        process((c & 1) ? r1 : r0, half * kEpiChunks + c);
-        if (!last) tmem_wait_ld();
       }
     }
+    // the last stores have completed (their shared memory stays in use until then)
+    if (a.y_tma && et == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -411,15 +478,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-cudaError_t launch_gemm_prefill(const ForwardArgs& a, int num_sms, cudaStream_t stream) {
-  if (a.M <= 0) return cudaSuccess;
+cudaError_t launch_gemm_prefill(const ForwardArgs& args, int num_sms, cudaStream_t stream) {
+  if (args.M <= 0) return cudaSuccess;
+  ForwardArgs a = args;
   static unsigned long long attr_done = 0;        // one bit per device
   cudaError_t ea = set_smem_attr_once(gemm_prefill_kernel, static_cast<int>(kSmemBytes), &attr_done);
   if (ea != cudaSuccess) return ea;
   CUtensorMap tm_x, tm_w;
-  if (!encode_2d_u8(&tm_x, a.xq, a.K, a.M, a.K, BK, BT, CU_TENSOR_MAP_SWIZZLE_128B)) return cudaErrorInvalidValue;
-  if (!encode_2d_u8(&tm_w, a.packed, a.K / 4, a.N, a.K / 4, BK / 4, BW, CU_TENSOR_MAP_SWIZZLE_NONE))
+  if (!encode_2d_u8(&tm_x, a.xq, a.K, a.M, a.K, 128, BT, CU_TENSOR_MAP_SWIZZLE_128B)) return cudaErrorInvalidValue;
+  if (!encode_2d_u8(&tm_w, a.packed, a.K / 4, a.N, a.K / 4, BK / 4, BW, CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
+  // y by TMA tile stores when its rows are 16-byte multiples at a 16-byte
+  // aligned base and no debug output is asked for; else plain stores
+  CUtensorMap tm_y;
+  memset(&tm_y, 0, sizeof(tm_y));
+  a.y_tma = a.y != nullptr && a.acc_out == nullptr && a.y32_out == nullptr && (a.N % 8) == 0 &&
+            (reinterpret_cast<uintptr_t>(a.y) & 15) == 0 &&
+            encode_2d_u16(&tm_y, a.y, a.N, a.M, static_cast<uint64_t>(a.N) * 2, BW, BT);
   const long tiles = static_cast<long>((a.N + BW - 1) / BW) * ((a.M + BT - 1) / BT);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(tiles < num_sms ? tiles : num_sms), 1, 1);
@@ -431,7 +506,7 @@ cudaError_t launch_gemm_prefill(const ForwardArgs& a, int num_sms, cudaStream_t 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = a.pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, gemm_prefill_kernel, tm_x, tm_w, a);
+  return cudaLaunchKernelEx(&cfg, gemm_prefill_kernel, tm_x, tm_w, tm_y, a);
 }
 
 }  // namespace bitlinear

@@ -218,29 +218,36 @@ __host__ __device__ SmemLayout smem_layout(int M, int ring, size_t slot_bytes, i
   return L;
 }
 
-// The items of one warp, in order: round r, item j of the round (j = warp,
-// warp + 8, ...); item j is chunk group j / U of unit j % U.  A round's
-// chunks (the last one of K maybe partial) form groups of kc, the last group
-// maybe shorter.
+// The items of one warp, in order.  A round's chunks (the last one of K maybe
+// partial) form groups of kc, the last group maybe shorter; its T = groups x U
+// items are numbered chunk group major (item j: group j / U, unit j % U), and
+// warp w takes the contiguous range [w T / 8, (w + 1) T / 8) of them.  The
+// shares differ by at most one item, and the consecutive items of a warp
+// mostly share a chunk group, so its x fragment is loaded once per group.
 struct ItemCursor {
-  int r, j;
+  int r, j, jend;
   __device__ __forceinline__ static int chunks(int r, int nchunks) {
     return min(nchunks - kRoundChunks * r, kRoundChunks);
   }
   __device__ __forceinline__ static int groups(int r, int nchunks, int kc) { return (chunks(r, nchunks) + kc - 1) / kc; }
+  __device__ __forceinline__ void bounds(int warp, int nchunks, int kc, int U) {
+    const int T = groups(r, nchunks, kc) * U;
+    j = warp * T / kWarps;
+    jend = (warp + 1) * T / kWarps;
+  }
   __device__ __forceinline__ void settle(int warp, int nround, int nchunks, int kc, int U) {
-    while (r < nround && j >= groups(r, nchunks, kc) * U) {
+    while (r < nround && j >= jend) {
       ++r;
-      j = warp;
+      if (r < nround) bounds(warp, nchunks, kc, U);
     }
   }
   __device__ __forceinline__ void start(int warp, int nround, int nchunks, int kc, int U) {
     r = 0;
-    j = warp;
+    bounds(warp, nchunks, kc, U);
     settle(warp, nround, nchunks, kc, U);
   }
   __device__ __forceinline__ void next(int warp, int nround, int nchunks, int kc, int U) {
-    j += kWarps;
+    ++j;
     settle(warp, nround, nchunks, kc, U);
   }
 };
@@ -331,6 +338,15 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
     load_params();
   }
 
+  // x into L2 while the previous kernel finishes: each CTA takes every
+  // gridDim-th 128-byte line, so the lines are asked for once
+  {
+    const uint8_t* xb = a.x ? reinterpret_cast<const uint8_t*>(a.x) : reinterpret_cast<const uint8_t*>(a.xq);
+    const size_t xbytes = static_cast<size_t>(M) * K * (a.x ? 2 : 1);
+    for (size_t l = blockIdx.x + static_cast<size_t>(gridDim.x) * threadIdx.x; xb != nullptr && l * 128 < xbytes;
+         l += static_cast<size_t>(gridDim.x) * kThreads)
+      prefetch_l2(xb + l * 128);
+  }
   pdl_wait_primary();
   if (!a.weights_early) {
     for (int i = 0; i < ring; ++i) issue_next();
@@ -679,14 +695,15 @@ cudaError_t launch_nt(const DecodeArgs& a, const DecodePlan& p, cudaStream_t str
 
 }  // namespace
 
-// Items of 2 chunks (4 KB) and 2 items in flight per warp: 64 KB in flight per
-// CTA.  A streaming probe on B200 (chained launches, all SMs) found this as
-// fast as any deeper ring at every decode shape, and 128 KB per CTA slower.
+// Items of one chunk (2 KB) and up to 4 items in flight per warp: 64 KB in
+// flight per CTA.  A streaming probe on B200 (chained launches, all SMs)
+// found 64 KB per CTA as fast as any deeper ring at every decode shape, and
+// 128 KB per CTA slower.
 #ifndef BITLINEAR_DECODE_KC
-#define BITLINEAR_DECODE_KC 2       // chunks (2 KB each) per item
+#define BITLINEAR_DECODE_KC 1       // chunks (2 KB each) per item
 #endif
 #ifndef BITLINEAR_DECODE_RING
-#define BITLINEAR_DECODE_RING 2     // largest ring per warp
+#define BITLINEAR_DECODE_RING 4     // largest ring per warp
 #endif
 
 DecodePlan plan_decode(int M, int N, int K, int num_sms) {
@@ -697,7 +714,7 @@ DecodePlan plan_decode(int M, int N, int K, int num_sms) {
   p.units_max = (units_total + p.grid - 1) / p.grid;
   const int nchunks = (K + kBoxK - 1) / kBoxK;
   // items of kc chunks when K has that many, else one chunk
-  p.kc = nchunks >= 2 * BITLINEAR_DECODE_KC ? BITLINEAR_DECODE_KC : 1;
+  p.kc = (BITLINEAR_DECODE_KC > 1 && nchunks >= 2 * BITLINEAR_DECODE_KC) ? BITLINEAR_DECODE_KC : 1;
   p.tail = (K % kBoxK) != 0;
   p.slot_bytes = static_cast<size_t>(p.kc) * kSubBytes;
   // shared-memory budget: two CTAs per SM for the 8-token kernel (the next

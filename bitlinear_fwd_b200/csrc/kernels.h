@@ -15,6 +15,9 @@ int current_device_status();
 // ---- TMA tensor maps (tensor_map.cu) ---------------------------------------
 bool encode_2d_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
                   uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle);
+// 2-D map over 16-bit elements (no swizzle), for tile stores
+bool encode_2d_u16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                   uint32_t box_inner, uint32_t box_outer);
 
 // ---- activation quantisation (act_quant.cu) --------------------------------
 // pdl: launch as a programmatic dependent of the previous kernel on the stream
@@ -91,6 +94,7 @@ struct ForwardArgs {
   bool faithful;          // bf16-module epilogue: every step rounded to bf16
   uint64_t wait_ns;       // limit of the main-loop waits (drains keep kWaitLimitNs)
   int stall;              // test hook: first wait on a barrier nothing signals
+  bool y_tma;             // set by the launcher: y tiles staged in shared memory and stored by TMA
 };
 
 // ---- bf16 export of packed weights (dequant.cu) ----------------------------
