@@ -122,11 +122,22 @@ int forward_impl_g(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packe
   const bool faithful = (flags & BITLINEAR_BF16_FAITHFUL) != 0;
   const bool decode = engine == 1 || (engine == 0 && M <= 16);
   cudaError_t e;
+  float* s_x = reinterpret_cast<float*>(base + L.off_sx);
+  int32_t* rowsum = reinterpret_cast<int32_t*>(base + L.off_rs);
+  int8_t* xq = reinterpret_cast<int8_t*>(base + L.off_xq);
   if (decode) {
+    // Above 8 tokens the activations are quantised once by the act-quant
+    // kernel, and the GEMV reads int8 x: every CTA of the GEMV needs all of
+    // x, and quantising it 148 times over costs more than the extra launch.
+    const bool pre = M > 8;
+    if (pre) {
+      e = launch_act_quant(x, int(M), int(K), xq, s_x, rowsum, status, resident, stream, faithful);
+      if (e != cudaSuccess) return BITLINEAR_ERR_CUDA;
+    }
     DecodeArgs d;
-    d.x = x;
-    d.xq = nullptr;
-    d.s_x = nullptr;
+    d.x = pre ? nullptr : x;
+    d.xq = pre ? xq : nullptr;
+    d.s_x = pre ? s_x : nullptr;
     d.packed = packed_w;
     d.w_scale = w_scale;
     d.bias = bias;
@@ -145,11 +156,16 @@ int forward_impl_g(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packe
     for (int g = 0; g < kMaxGroups; ++g) d.group_end[g] = grp.end[g];
     d.wait_ns = launch_wait_ns();
     d.stall = launch_stall();
-    return status_of(launch_decode(d, sms, stream));
+    if (pre) {
+      d.xq_out = nullptr;                          // copied from the workspace below
+      d.sx_out = nullptr;
+    }
+    e = launch_decode(d, sms, stream);
+    if (e == cudaSuccess && pre && xq_out)
+      e = cudaMemcpyAsync(xq_out, xq, size_t(M) * size_t(K), cudaMemcpyDeviceToDevice, stream);
+    if (e == cudaSuccess && pre && sx_out) e = cudaMemcpyAsync(sx_out, s_x, 4 * size_t(M), cudaMemcpyDeviceToDevice, stream);
+    return status_of(e);
   }
-  float* s_x = reinterpret_cast<float*>(base + L.off_sx);
-  int32_t* rowsum = reinterpret_cast<int32_t*>(base + L.off_rs);
-  int8_t* xq = reinterpret_cast<int8_t*>(base + L.off_xq);
   e = launch_act_quant(x, int(M), int(K), xq, s_x, rowsum, status, resident, stream, faithful);
   if (e != cudaSuccess) return BITLINEAR_ERR_CUDA;
   ForwardArgs a;

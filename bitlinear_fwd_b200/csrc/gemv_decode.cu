@@ -225,29 +225,35 @@ __host__ __device__ SmemLayout smem_layout(int M, int ring, size_t slot_bytes, i
 // shares differ by at most one item, and the consecutive items of a warp
 // mostly share a chunk group, so its x fragment is loaded once per group.
 struct ItemCursor {
-  int r, j, jend;
+  int r, g, u, left;                               // round, item (group g, unit u), items left in the round
   __device__ __forceinline__ static int chunks(int r, int nchunks) {
     return min(nchunks - kRoundChunks * r, kRoundChunks);
   }
   __device__ __forceinline__ static int groups(int r, int nchunks, int kc) { return (chunks(r, nchunks) + kc - 1) / kc; }
-  __device__ __forceinline__ void bounds(int warp, int nchunks, int kc, int U) {
+  __device__ __forceinline__ void begin_round(int warp, int nchunks, int kc, int U) {
     const int T = groups(r, nchunks, kc) * U;
-    j = warp * T / kWarps;
-    jend = (warp + 1) * T / kWarps;
+    const int jb = warp * T / kWarps;
+    left = (warp + 1) * T / kWarps - jb;
+    g = jb / U;
+    u = jb - g * U;
   }
   __device__ __forceinline__ void settle(int warp, int nround, int nchunks, int kc, int U) {
-    while (r < nround && j >= jend) {
+    while (r < nround && left == 0) {
       ++r;
-      if (r < nround) bounds(warp, nchunks, kc, U);
+      if (r < nround) begin_round(warp, nchunks, kc, U);
     }
   }
   __device__ __forceinline__ void start(int warp, int nround, int nchunks, int kc, int U) {
     r = 0;
-    bounds(warp, nchunks, kc, U);
+    begin_round(warp, nchunks, kc, U);
     settle(warp, nround, nchunks, kc, U);
   }
   __device__ __forceinline__ void next(int warp, int nround, int nchunks, int kc, int U) {
-    ++j;
+    --left;
+    if (++u == U) {
+      u = 0;
+      ++g;
+    }
     settle(warp, nround, nchunks, kc, U);
   }
 };
@@ -298,14 +304,13 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
   // copy group per item; pieces beyond N or K are zero-filled
   ItemCursor ic;                                     // next item to issue
   ic.start(warp, nround, nchunks, kc, U);
-  int issued = 0;
+  int islot = 0;                                     // ring slot of the next copy
   auto issue_next = [&]() {
     if (ic.r < nround) {
-      const int s = issued % ring;
-      const int g = ic.j / U, u = ic.j - g * U;
+      const int g = ic.g, u = ic.u;
       const int c0 = kRoundChunks * ic.r + g * kc;                 // first chunk of the item
       const int nc = min(kc, ItemCursor::chunks(ic.r, nchunks) - g * kc);
-      uint8_t* dst = wring + s * slot_bytes;
+      uint8_t* dst = wring + islot * slot_bytes;
       for (int p = lane; p < nc * 128; p += 32) {
         const int cc = p >> 7, r = (p >> 3) & 15, q = p & 7;
         const int n = (u_begin + u) * kUnitRows + r;
@@ -314,7 +319,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
         const uint8_t* src = a.packed + (valid ? static_cast<size_t>(n) * row_bytes + off : 0);
         cp_async16(dst + cc * kSubBytes + r * 128 + ((q ^ (r & 7)) << 4), src, valid ? 16u : 0u);
       }
-      ++issued;
+      islot = islot + 1 == ring ? 0 : islot + 1;
       ic.next(warp, nround, nchunks, kc, U);
     }
     cp_async_commit();                               // one group per call, empty when nothing is left
@@ -475,7 +480,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
   const int r0 = mma_row_to_box(g);                  // sub-box rows r0 and r0 + 8
   ItemCursor cc;                                     // next item to consume
   cc.start(warp, nround, nchunks, kc, U);
-  int consumed = 0;
+  int cslot = 0;                                     // ring slot of the next item to consume
   int xchunk = -1;                                   // round-local chunk of the x fragment held
   uint32_t xw[2][2][NT][8];                          // [v][pair][token tile][word]
   for (int r = 0; r < nround; ++r) {
@@ -537,12 +542,12 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
 
     // ---- this warp's items of round r
     while (ok && cc.r == r) {
-      const int s = consumed % ring;
+      const int s = cslot;
       // this item's copies (the oldest group in flight) have landed, for
       // every lane of the warp
       cp_async_wait(ring - 1);
       __syncwarp();
-      const int grp = cc.j / U, u = cc.j - grp * U;
+      const int grp = cc.g, u = cc.u;
       const int first = grp * kc;                    // round-local chunk of the item's first sub-box
       const int nsub = min(kc, ItemCursor::chunks(r, nchunks) - first);
       int acc[4][NT][4];
@@ -597,7 +602,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
       }
       // the slot is read: refill it with this warp's next item
       __syncwarp();
-      ++consumed;
+      cslot = cslot + 1 == ring ? 0 : cslot + 1;
       cc.next(warp, nround, nchunks, kc, U);
       issue_next();
       // fields -> the unit's sums (4^i sum(c q) >> 2i is exact: at most 8 chunks
