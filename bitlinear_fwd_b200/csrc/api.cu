@@ -138,6 +138,7 @@ int forward_impl_g(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packe
     d.x = pre ? nullptr : x;
     d.xq = pre ? xq : nullptr;
     d.s_x = pre ? s_x : nullptr;
+    d.rowsum = pre ? rowsum : nullptr;
     d.packed = packed_w;
     d.w_scale = w_scale;
     d.bias = bias;
@@ -375,6 +376,7 @@ int bitlinear_forward_q8(const int8_t* xq, const float* x_scale, const int32_t* 
   d.x = nullptr;
   d.xq = xq;
   d.s_x = x_scale;
+  d.rowsum = xq_rowsum;
   d.packed = packed_w;
   d.w_scale = w_scale;
   d.bias = bias;
@@ -569,6 +571,7 @@ int bitlinear_forward_partial(const uint16_t* x, int64_t M, int64_t K, const flo
   d.x = nullptr;
   d.xq = xq;
   d.s_x = s_x;
+  d.rowsum = rowsum;
   d.packed = packed_w;
   d.w_scale = s_x;
   d.bias = nullptr;

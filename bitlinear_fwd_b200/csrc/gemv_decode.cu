@@ -11,43 +11,46 @@
 // eight (4096 k: the x of one round sits in shared memory as int8).
 //
 // Inside a CTA every one of the 8 warps streams and computes:
-//   * The CTA's work of a round is a list of items (chunk group, unit), chunk
-//     group outer: a group is kc consecutive chunks of one unit (the last one
-//     of K maybe partial).  Warp w takes items w, w + 8, ... of every round,
-//     so the warps' shares differ by at most one item.
+//   * An item is one chunk of one unit (16 rows x 128 bytes).  A round's
+//     items are numbered chunk-major, and warp w takes the contiguous w-th
+//     eighth of them, so a warp's consecutive items share a chunk (its x
+//     fragment is loaded once per chunk) and the shares differ by at most
+//     one item.
 //   * Each warp streams its own items through its own ring of shared-memory
-//     slots: every lane copies its own 16-byte pieces of an item with
-//     cp.async (128-byte rows, written in the 128-byte-swizzled order that
-//     keeps the fragment reads below conflict-free), one copy group per item,
-//     up to `ring` items ahead; pieces beyond N or K are zero-filled.  The
-//     warp waits for the oldest group and refills its slot once it has read
-//     it.  No warp ever waits for another warp's copies.  When the weights
-//     are resident the first copies (and the bias and scales, into
-//     registers) are issued before the wait on the previous kernel of the
-//     stream, so they overlap its tail.
-//   * Before the items, all warps form each token's absmax over the row,
+//     slots: every lane copies 4 x 16 bytes of an item with cp.async, at
+//     per-lane offsets fixed for the whole kernel (128-byte rows, written in
+//     the 128-byte-swizzled order that keeps the fragment reads below
+//     conflict-free), one copy group per item, up to `ring` items ahead;
+//     pieces beyond N or K are zero-filled.  The warp waits for the oldest
+//     group (once for all of them when its whole share fitted in the ring)
+//     and refills its slot once it has read it.  No warp ever waits for
+//     another warp's copies.  When the weights are resident the first
+//     copies, the bias and the scales, the x-phase plan and an L2 prefetch
+//     of x are issued before the wait on the previous kernel of the stream,
+//     so they overlap its tail; after the wait only x-dependent work is left.
+//   * bf16 x (M <= 8): all warps form each token's absmax over the row,
 //     s_x = 127 / max(absmax, 1e-5) in float32, and q = round_half_even(x
 //     s_x) as int8 into shared memory, one round at a time, with the sum of q
 //     per token.  For K <= 4096 each lane's share of x (at most 8 x 32
-//     bytes per token, two tokens per warp when M > 8) is read once and held
-//     in registers between the two steps; otherwise x is read again for the
-//     quantising step.  CTA b starts its x reads at a different chunk, so the
-//     SMs do not ask for the same L2 lines at the same moment.  Pre-quantised
-//     int8 input is copied in instead.
-//   * Per chunk of an item, a thread takes one 16-byte vector of two weight
-//     rows and issues mma.sync m16n8k32 (weights as A, u8; tokens as B, s8;
-//     a second 8-token tile for M > 8).  The codes c = u + 1 enter
+//     bytes per token) is read once and held in registers between the two
+//     steps; otherwise x is read again for the quantising step.
+//   * int8 x (above 8 tokens the act-quant kernel quantises x once; also the
+//     pre-quantised and K-split calls): the scales and row sums are read, and
+//     each warp loads its x fragments straight from global memory.
+//   * Per item a thread takes one 16-byte vector of two weight rows per
+//     256-k half and issues mma.sync m16n8k32 (weights as A, u8; tokens as B,
+//     s8; a second 8-token tile for M > 8).  The codes c = u + 1 enter
 //     unshifted: A_i = word & (0x03030303 << 2i) holds 4^i c per byte lane,
 //     so field i accumulates 4^i sum(c q); the fields are combined with
-//     exact shifts and added to the unit's int32 sums in shared memory.  The
-//     x fragment of a chunk stays in registers while consecutive items share
-//     the chunk.
+//     exact shifts and added to the unit's int32 sums in shared memory.
 //   * Epilogue: acc = sum(c q) - sum(q) = sum(u q); y = acc / (s_x s_w)
 //     (+ bias) -> bf16, with s_w the scale of the row's layer when several
 //     layers are stacked, the division done as a product with the double
-//     1 / (s_x s_w) of the token and layer (exactly the float32 quotient).
-//     The bf16-faithful mode rounds the scale, the products, the sum and the
-//     quotient to bf16 as a bf16 module does.
+//     1 / (s_x s_w) of the token and layer (exactly the float32 quotient),
+//     each output computing its own reciprocal.  The bf16-faithful mode (a
+//     template parameter, so neither mode carries the other's branches)
+//     rounds the scale, the products, the sum and the quotient to bf16 as a
+//     bf16 module does.
 // Rows beyond N and k beyond K are zero-filled (code 0), so they add
 // nothing whatever the x bytes there are.
 //
@@ -71,7 +74,6 @@ constexpr int kBoxK = 512;                            // k per chunk (sub-box)
 constexpr int kSubBytes = kUnitRows * kBoxK / 4;      // 2 KB
 constexpr int kRoundChunks = 8;                       // chunks per x round
 constexpr int kChunkK = kRoundChunks * kBoxK;         // k per round
-constexpr int kMaxRing = 8;                           // slots per warp
 constexpr int kMaxUnits = 32;                         // units per CTA
 constexpr int kXB = 8;                                // bf16 x loads in flight per lane (absmax)
 constexpr int kQB = 2;                                // the same in the quantising pass
@@ -120,14 +122,6 @@ __device__ __forceinline__ void red_shared_add(int* p, int v) {
 __device__ __forceinline__ int xs_chunk(int ch) { return ch ^ (((ch >> 3) & 1) << 1); }
 
 __device__ __forceinline__ int mma_row_to_box(int g) { return (g >> 1) | ((g & 1) << 2); }
-
-// Every CTA reads the whole of x; CTA b starts its 16-element chunks at a
-// different place (chunk i of a row is read as chunk (i + rot) % n), so the
-// 148 SMs do not ask the same L2 lines for the same bytes at the same moment.
-__device__ __forceinline__ int rotated(int ch, int n, int rot) {
-  const int c = ch + rot;
-  return c >= n ? c - n : c;
-}
 
 // largest |x| of 16 bf16 values, as bf16 bits (finite values order like bits & 0x7FFF)
 __device__ __forceinline__ uint32_t absmax16_bits(uint4 lo, uint4 hi) {
@@ -195,7 +189,6 @@ struct SmemTail {
   int rsum[16];                      // sum of q per token
   float sx[16];                      // s_x per token
   float swg[kMaxGroups];             // s_w of each row group
-  double rcp[16][kMaxGroups];        // 1 / d per token and row group (double)
   int failed;                        // a wait of this CTA timed out
 };
 
@@ -206,12 +199,14 @@ struct SmemLayout {
 // 8 warps' rings of `ring` slots of slot_bytes (1024-aligned base), x rows of
 // one round for the M tokens, per-unit int32 sums [unit][row][8 * token
 // tiles], bias, tail
-__host__ __device__ SmemLayout smem_layout(int M, int ring, size_t slot_bytes, int units) {
+// M tokens, of which xrows have their x staged in shared memory (M for bf16
+// x, 0 for int8 x read straight from global memory)
+__host__ __device__ SmemLayout smem_layout(int M, int xrows, int ring, size_t slot_bytes, int units) {
   const int ntok = M <= 8 ? 8 : 16;
   SmemLayout L;
   L.ring = 0;
   L.xs = L.ring + static_cast<size_t>(kWarps) * ring * slot_bytes;
-  L.acc = L.xs + static_cast<size_t>(M) * (kChunkK + 16);
+  L.acc = L.xs + static_cast<size_t>(xrows) * (kChunkK + 16);
   L.bias = L.acc + static_cast<size_t>(units) * kUnitRows * ntok * 4;
   L.tail = (L.bias + static_cast<size_t>(units) * kUnitRows * 2 + 15) & ~size_t(15);
   L.total = 1024 + L.tail + sizeof(SmemTail);
@@ -258,7 +253,7 @@ struct ItemCursor {
   }
 };
 
-template <int NT>
+template <int NT, bool FAITHFUL>
 __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
     decode_kernel(const DecodeArgs a) {
   constexpr int NTOK = NT * 8;
@@ -267,7 +262,10 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
   const int ring = a.ring;
   const int kc = a.kc;                               // chunks per 3-D item
   const size_t slot_bytes = static_cast<size_t>(kc) * kSubBytes;
-  const SmemLayout L = smem_layout(a.M, ring, slot_bytes, a.units_max);
+  // int8 x with its row sums is read straight from global memory (no x in
+  // shared memory); bf16 x is quantised into shared memory
+  const bool direct = a.xq != nullptr && a.rowsum != nullptr;
+  const SmemLayout L = smem_layout(a.M, direct ? 0 : a.M, ring, slot_bytes, a.units_max);
   int8_t* xs = reinterpret_cast<int8_t*>(base + L.xs);
   int* acc_s = reinterpret_cast<int*>(base + L.acc);            // [unit][row][token]
   uint16_t* bias_s = reinterpret_cast<uint16_t*>(base + L.bias);
@@ -305,19 +303,25 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
   ItemCursor ic;                                     // next item to issue
   ic.start(warp, nround, nchunks, kc, U);
   int islot = 0;                                     // ring slot of the next copy
+  // this lane's pieces of a chunk item (kc = 1): rows (lane >> 3) + 4 j,
+  // piece lane & 7 of each row, j = 0..3; their source and destination
+  // offsets are fixed, only the item's first row and chunk change
+  const int prow = lane >> 3, pq = lane & 7;
+  const uint32_t psrc = static_cast<uint32_t>(prow) * row_bytes + 16u * pq;   // + 4 j row_bytes
+  const uint32_t pdst0 = prow * 128 + ((pq ^ prow) << 4);          // rows prow, prow + 8
+  const uint32_t pdst1 = (prow + 4) * 128 + ((pq ^ (prow + 4)) << 4);   // rows prow + 4, prow + 12
   auto issue_next = [&]() {
     if (ic.r < nround) {
-      const int g = ic.g, u = ic.u;
-      const int c0 = kRoundChunks * ic.r + g * kc;                 // first chunk of the item
-      const int nc = min(kc, ItemCursor::chunks(ic.r, nchunks) - g * kc);
+      const int c = kRoundChunks * ic.r + ic.g;     // chunk of the item
+      const int n0 = (u_begin + ic.u) * kUnitRows;  // first row of the unit
       uint8_t* dst = wring + islot * slot_bytes;
-      for (int p = lane; p < nc * 128; p += 32) {
-        const int cc = p >> 7, r = (p >> 3) & 15, q = p & 7;
-        const int n = (u_begin + u) * kUnitRows + r;
-        const uint32_t off = static_cast<uint32_t>(c0 + cc) * (kBoxK / 4) + 16u * q;
-        const bool valid = n < N && off < row_bytes;
-        const uint8_t* src = a.packed + (valid ? static_cast<size_t>(n) * row_bytes + off : 0);
-        cp_async16(dst + cc * kSubBytes + r * 128 + ((q ^ (r & 7)) << 4), src, valid ? 16u : 0u);
+      const bool kin = static_cast<uint32_t>(c) * (kBoxK / 4) + 16u * pq < row_bytes;
+      const uint8_t* src = a.packed + static_cast<size_t>(n0) * row_bytes + static_cast<uint32_t>(c) * (kBoxK / 4) + psrc;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const bool valid = kin && n0 + prow + 4 * j < N;
+        cp_async16(dst + ((j & 1) ? pdst1 : pdst0) + (j >> 1) * 1024, valid ? src + static_cast<size_t>(4 * j) * row_bytes : a.packed,
+                   valid ? 16u : 0u);
       }
       islot = islot + 1 == ring ? 0 : islot + 1;
       ic.next(warp, nround, nchunks, kc, U);
@@ -343,6 +347,26 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
     load_params();
   }
 
+  // ---- the x-phase plan, worked out while the previous kernel finishes:
+  // warp w takes token(s) m = w / P (+ 8 / P, ...) and a 1/P share of the
+  // row, P = max(1, 8 / M); in the one-pass path load i of a lane reads the
+  // 16-element chunk part * 32 + lane + i * 32 P of its token
+  const int cpr = K >> 4;                            // 16-element chunks per row
+  const int P = M >= kWarps ? 1 : kWarps / M;
+  const int part = warp % P, mstep = kWarps / P;
+  const int C = (cpr + 32 * P - 1) / (32 * P);       // chunks per lane per token
+  // One pass over x when the row is one round and this lane's share fits in
+  // registers: the values loaded for the absmax are quantised in place.
+  const bool single = a.x && nround == 1 && C <= kHold;
+  const int ch_first = part * 32 + lane;             // first chunk of this lane
+  const int xstep = 64 * P;                          // uint4 between a lane's loads
+  const uint4* xl[NT];                               // this lane's first load, per token slot
+#pragma unroll
+  for (int j = 0; j < NT; ++j) {
+    const int m = min(warp / P + j * mstep, M - 1);
+    xl[j] = reinterpret_cast<const uint4*>(a.x) + ((static_cast<size_t>(m) * K) >> 3) + 2 * ch_first;
+  }
+
   // x into L2 while the previous kernel finishes: each CTA takes every
   // gridDim-th 128-byte line, so the lines are asked for once
   {
@@ -362,29 +386,25 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
   bool ok = true;
   const int g = lane >> 2, t = lane & 3;
 
-  // ---- per-token absmax over the whole row: warp w takes token(s)
-  // m = w / P (+ 8 / P, ...) and a 1/P share of the row, P = max(1, 8 / M)
-  const int cpr = K >> 4;                            // 16-element chunks per row
-  const int xrot = static_cast<int>((static_cast<unsigned>(blockIdx.x) * 97u) % static_cast<unsigned>(cpr));
-  const int P = M >= kWarps ? 1 : kWarps / M;
-  const int part = warp % P, mstep = kWarps / P;
-  const int C = (cpr + 32 * P - 1) / (32 * P);       // chunks per lane per token
-  // One pass over x when the row is one round and this lane's share fits in
-  // registers: the values loaded for the absmax are quantised in place.
-  const bool single = a.x && nround == 1 && C <= kHold;
-  if (single) {
-    const uint4* xrow0 = reinterpret_cast<const uint4*>(a.x);
+  // ---- per-token absmax over the whole row
+  if (direct) {
+    // int8 x from the act-quant kernel: the scales and row sums are read
+    // here, the fragments straight from global memory in the item loop
+    if (threadIdx.x < M) {
+      sm.sx[threadIdx.x] = a.s_x[threadIdx.x];
+      sm.rsum[threadIdx.x] = a.rowsum[threadIdx.x];
+    }
+  } else if (NT == 1 && single) {
     uint4 v[kHold * NT][2];
 #pragma unroll
     for (int i = 0; i < kHold * NT; ++i) {
       const int j = (NT == 2 && i >= C) ? 1 : 0;     // token slot of this warp
       const int m = warp / P + j * mstep;
-      const int ch0 = part * 32 + lane + (i - j * C) * 32 * P;
-      const int ch = ch0 < cpr ? rotated(ch0, cpr, xrot) : ch0;
+      const int ii = i - j * C;
       v[i][0] = v[i][1] = make_uint4(0, 0, 0, 0);
-      if (i < NT * C && m < M && ch0 < cpr) {
-        v[i][0] = __ldg(xrow0 + (static_cast<size_t>(m) * K >> 3) + 2 * ch);
-        v[i][1] = __ldg(xrow0 + (static_cast<size_t>(m) * K >> 3) + 2 * ch + 1);
+      if (i < NT * C && m < M && ch_first + ii * 32 * P < cpr) {
+        v[i][0] = __ldg(xl[j] + ii * xstep);
+        v[i][1] = __ldg(xl[j] + ii * xstep + 1);
       }
     }
     uint32_t mx[NT];
@@ -392,9 +412,11 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
     for (int j = 0; j < NT; ++j) mx[j] = 0;
 #pragma unroll
     for (int i = 0; i < kHold * NT; ++i) {
-      const uint32_t am = absmax16_bits(v[i][0], v[i][1]);   // zeros where nothing was loaded
-      if (NT == 2 && i >= C) mx[NT - 1] = max(mx[NT - 1], am);
-      else mx[0] = max(mx[0], am);
+      if (i < NT * C) {
+        const uint32_t am = absmax16_bits(v[i][0], v[i][1]);   // zeros where nothing was loaded
+        if (NT == 2 && i >= C) mx[NT - 1] = max(mx[NT - 1], am);
+        else mx[0] = max(mx[0], am);
+      }
     }
 #pragma unroll
     for (int j = 0; j < NT; ++j) {
@@ -407,10 +429,10 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
 #pragma unroll
     for (int j = 0; j < NT; ++j) {
       const int m = min(warp / P + j * mstep, M - 1);
-      sxr[j] = act_scale(bf16_bits_to_f32(sm.amax[m]), a.faithful);
+      sxr[j] = act_scale(bf16_bits_to_f32(sm.amax[m]), FAITHFUL);
     }
     if (threadIdx.x < M) {
-      const float sxv = act_scale(bf16_bits_to_f32(sm.amax[threadIdx.x]), a.faithful);
+      const float sxv = act_scale(bf16_bits_to_f32(sm.amax[threadIdx.x]), FAITHFUL);
       sm.sx[threadIdx.x] = sxv;
       if (blockIdx.x == 0 && a.sx_out) a.sx_out[threadIdx.x] = sxv;
     }
@@ -421,11 +443,10 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
     for (int i = 0; i < kHold * NT; ++i) {
       const int j = (NT == 2 && i >= C) ? 1 : 0;
       const int m = warp / P + j * mstep;
-      const int ch0 = part * 32 + lane + (i - j * C) * 32 * P;
-      const int ch = ch0 < cpr ? rotated(ch0, cpr, xrot) : ch0;
-      if (i < NT * C && m < M && ch0 < cpr) {
+      const int ch = ch_first + (i - j * C) * 32 * P;
+      if (i < NT * C && m < M && ch < cpr) {
         int ps = 0;
-        const uint4 qv = quant16(v[i][0], v[i][1], j ? sxr[NT - 1] : sxr[0], ps, a.faithful);
+        const uint4 qv = quant16(v[i][0], v[i][1], j ? sxr[NT - 1] : sxr[0], ps, FAITHFUL);
         if (j) sum[NT - 1] += ps;
         else sum[0] += ps;
         *reinterpret_cast<uint4*>(xs + m * S + 16 * xs_chunk(ch)) = qv;
@@ -438,7 +459,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
       const int r = __reduce_add_sync(0xffffffffu, sum[j]);
       if (lane == 0 && m < M) atomicAdd(&sm.rsum[m], r);
     }
-  } else if (a.x) {
+  } else if (NT == 1 && a.x) {
     for (int m = warp / P; m < M; m += mstep) {
       const uint4* row = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(m) * K);
       uint32_t mx = 0;
@@ -450,9 +471,8 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
           const int chu = ch0 + j * 32 * P;
           v[j][0] = v[j][1] = make_uint4(0, 0, 0, 0);
           if (chu < cpr) {
-            const int ch = rotated(chu, cpr, xrot);
-            v[j][0] = __ldg(row + 2 * ch);
-            v[j][1] = __ldg(row + 2 * ch + 1);
+            v[j][0] = __ldg(row + 2 * chu);
+            v[j][1] = __ldg(row + 2 * chu + 1);
           }
         }
 #pragma unroll
@@ -463,7 +483,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
     }
     __syncthreads();
     if (threadIdx.x < M) {
-      const float sxv = act_scale(bf16_bits_to_f32(sm.amax[threadIdx.x]), a.faithful);
+      const float sxv = act_scale(bf16_bits_to_f32(sm.amax[threadIdx.x]), FAITHFUL);
       sm.sx[threadIdx.x] = sxv;
       if (blockIdx.x == 0 && a.sx_out) a.sx_out[threadIdx.x] = sxv;
     }
@@ -481,6 +501,10 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
   ItemCursor cc;                                     // next item to consume
   cc.start(warp, nround, nchunks, kc, U);
   int cslot = 0;                                     // ring slot of the next item to consume
+  // When the prologue requested every item of this warp (they fit in its
+  // ring), one wait for all copies replaces the per-item waits.
+  const bool per_item_wait = ic.r < nround;
+  bool first_wait = true;
   int xchunk = -1;                                   // round-local chunk of the x fragment held
   uint32_t xw[2][2][NT][8];                          // [v][pair][token tile][word]
   for (int r = 0; r < nround; ++r) {
@@ -488,7 +512,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
     const int ccpr = min(kChunkK, K - c0) >> 4;      // 16-element chunks of x in this round
     if (r > 0) __syncthreads();                      // every warp is done with the previous round's x
     // ---- x round -> int8 in shared memory (tokens < M only)
-    for (int m = warp / P; m < (single ? 0 : M); m += mstep) {
+    for (int m = warp / P; m < ((NT == 2 || single || direct) ? 0 : M); m += mstep) {
       int8_t* xrow = xs + m * S;
       const float sxm = sm.sx[m];
       int sum = 0;
@@ -501,17 +525,16 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
           for (int j = 0; j < kQB; ++j) {
             const int chu = ch0 + j * 32 * P;
             if (chu < ccpr) {
-              const int ch = rotated(chu, ccpr, xrot % ccpr);
-              v[j][0] = __ldg(src + 2 * ch);
-              v[j][1] = __ldg(src + 2 * ch + 1);
+              v[j][0] = __ldg(src + 2 * chu);
+              v[j][1] = __ldg(src + 2 * chu + 1);
             }
           }
 #pragma unroll
           for (int j = 0; j < kQB; ++j) {
             const int chu = ch0 + j * 32 * P;
             if (chu < ccpr) {
-              const int ch = rotated(chu, ccpr, xrot % ccpr);
-              const uint4 qv = quant16(v[j][0], v[j][1], sxm, sum, a.faithful);
+              const int ch = chu;
+              const uint4 qv = quant16(v[j][0], v[j][1], sxm, sum, FAITHFUL);
               if (blockIdx.x == 0 && a.xq_out) *reinterpret_cast<uint4*>(a.xq_out + roff + 16 * ch) = qv;
               *reinterpret_cast<uint4*>(xrow + 16 * xs_chunk(ch)) = qv;
             }
@@ -537,7 +560,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
       sum = __reduce_add_sync(0xffffffffu, sum);
       if (lane == 0) atomicAdd(&sm.rsum[m], sum);
     }
-    if (!single) __syncthreads();
+    if (!single && !direct) __syncthreads();
     xchunk = -1;
 
     // ---- this warp's items of round r
@@ -545,11 +568,40 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
       const int s = cslot;
       // this item's copies (the oldest group in flight) have landed, for
       // every lane of the warp
-      cp_async_wait(ring - 1);
-      __syncwarp();
-      const int grp = cc.g, u = cc.u;
-      const int first = grp * kc;                    // round-local chunk of the item's first sub-box
-      const int nsub = min(kc, ItemCursor::chunks(r, nchunks) - first);
+      if (per_item_wait) {
+        cp_async_wait(ring - 1);
+        __syncwarp();
+      } else if (first_wait) {
+        cp_async_wait(0);
+        __syncwarp();
+        first_wait = false;
+      }
+      const int u = cc.u;
+      const int lc = cc.g;                           // round-local chunk of the item (one chunk per item)
+      if (lc != xchunk) {
+#pragma unroll
+        for (int v = 0; v < 2; ++v)
+#pragma unroll
+          for (int pr = 0; pr < 2; ++pr)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+              const int m = nt * 8 + g;
+#pragma unroll
+              for (int c2 = 0; c2 < 2; ++c2) {
+                uint4 xv = make_uint4(0, 0, 0, 0);
+                const int xc = 32 * lc + 16 * v + 4 * t + 2 * pr + c2;    // 16-byte chunk in the round
+                if (m < M && (!direct || 16 * xc < K - r * kChunkK)) {
+                  if (direct)
+                    xv = __ldg(reinterpret_cast<const uint4*>(a.xq + static_cast<size_t>(m) * K + r * kChunkK) + xc);
+                  else
+                    xv = *reinterpret_cast<const uint4*>(xs + m * S + 16 * xs_chunk(xc));
+                }
+                xw[v][pr][nt][4 * c2 + 0] = xv.x; xw[v][pr][nt][4 * c2 + 1] = xv.y;
+                xw[v][pr][nt][4 * c2 + 2] = xv.z; xw[v][pr][nt][4 * c2 + 3] = xv.w;
+              }
+            }
+        xchunk = lc;
+      }
       int acc[4][NT][4];
 #pragma unroll
       for (int i = 0; i < 4; ++i)
@@ -557,56 +609,33 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
           for (int rr = 0; rr < 4; ++rr) acc[i][nt][rr] = 0;
-      for (int sb = 0; sb < nsub; ++sb) {
-        const int lc = first + sb;                   // round-local chunk
-        if (lc != xchunk) {
+      const uint8_t* box = wring + s * slot_bytes;
 #pragma unroll
-          for (int v = 0; v < 2; ++v)
+      for (int v = 0; v < 2; ++v) {
+        const int cw = 4 * v + t;                    // 16-byte chunk of the 128-byte row
+        const uint4 wa = *reinterpret_cast<const uint4*>(box + r0 * 128 + ((cw ^ r0) << 4));
+        const uint4 wb = *reinterpret_cast<const uint4*>(box + (r0 + 8) * 128 + ((cw ^ r0) << 4));
+        const uint32_t w0[4] = {wa.x, wa.y, wa.z, wa.w};
+        const uint32_t w1[4] = {wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
-            for (int pr = 0; pr < 2; ++pr)
+        for (int pr = 0; pr < 2; ++pr)
 #pragma unroll
-              for (int nt = 0; nt < NT; ++nt) {
-                const int m = nt * 8 + g;
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t mask = kCodeMask << (2 * i);
+            const uint32_t a0 = w0[2 * pr] & mask, a1 = w1[2 * pr] & mask;
+            const uint32_t a2 = w0[2 * pr + 1] & mask, a3 = w1[2 * pr + 1] & mask;
 #pragma unroll
-                for (int c2 = 0; c2 < 2; ++c2) {
-                  uint4 xv = make_uint4(0, 0, 0, 0);
-                  if (m < M)
-                    xv = *reinterpret_cast<const uint4*>(xs + m * S +
-                                                         16 * xs_chunk(32 * lc + 16 * v + 4 * t + 2 * pr + c2));
-                  xw[v][pr][nt][4 * c2 + 0] = xv.x; xw[v][pr][nt][4 * c2 + 1] = xv.y;
-                  xw[v][pr][nt][4 * c2 + 2] = xv.z; xw[v][pr][nt][4 * c2 + 3] = xv.w;
-                }
-              }
-          xchunk = lc;
-        }
-        const uint8_t* box = wring + s * slot_bytes + sb * kSubBytes;
-#pragma unroll
-        for (int v = 0; v < 2; ++v) {
-          const int cw = 4 * v + t;                  // 16-byte chunk of the 128-byte row
-          const uint4 wa = *reinterpret_cast<const uint4*>(box + r0 * 128 + ((cw ^ r0) << 4));
-          const uint4 wb = *reinterpret_cast<const uint4*>(box + (r0 + 8) * 128 + ((cw ^ r0) << 4));
-          const uint32_t w0[4] = {wa.x, wa.y, wa.z, wa.w};
-          const uint32_t w1[4] = {wb.x, wb.y, wb.z, wb.w};
-#pragma unroll
-          for (int pr = 0; pr < 2; ++pr)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const uint32_t mask = kCodeMask << (2 * i);
-              const uint32_t a0 = w0[2 * pr] & mask, a1 = w1[2 * pr] & mask;
-              const uint32_t a2 = w0[2 * pr + 1] & mask, a3 = w1[2 * pr + 1] & mask;
-#pragma unroll
-              for (int nt = 0; nt < NT; ++nt)
-                mma_u8s8(acc[i][nt], a0, a1, a2, a3, xw[v][pr][nt][i], xw[v][pr][nt][4 + i]);
-            }
-        }
+            for (int nt = 0; nt < NT; ++nt)
+              mma_u8s8(acc[i][nt], a0, a1, a2, a3, xw[v][pr][nt][i], xw[v][pr][nt][4 + i]);
+          }
       }
       // the slot is read: refill it with this warp's next item
       __syncwarp();
       cslot = cslot + 1 == ring ? 0 : cslot + 1;
       cc.next(warp, nround, nchunks, kc, U);
       issue_next();
-      // fields -> the unit's sums (4^i sum(c q) >> 2i is exact: at most 8 chunks
-      // of 512 k per item keep 64 * 2 * 127 * 4096 below 2^31)
+      // fields -> the unit's sums (4^i sum(c q) >> 2i is exact: 64 * 2 * 127
+      // * 512 < 2^31)
       int* au = acc_s + u * kUnitRows * NTOK;
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
@@ -638,18 +667,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
     report_status(a.status, kStatusTimeout);
     if (lane == 0) sm.failed = 1;
   }
-  // d = s_x s_w per token and row group (on a bf16 module bf16(bf16(s_w) s_x)),
-  // kept as the double 1 / d: RN_f32(a * (1/d)) is RN_f32(a / d) for every
-  // float32 (or bf16) numerator a -- a quotient of two floats lies at least
-  // 2^-49 (relative) from every float32 midpoint, and the double product is
-  // within 2^-52 of it
-  __syncthreads();                                   // s_w stored by its threads
-  if (threadIdx.x < M * a.ngroups) {
-    const int m = threadIdx.x / a.ngroups, gg = threadIdx.x - m * a.ngroups;
-    const float d = a.faithful ? bf16_round(__fmul_rn(bf16_round(sm.swg[gg]), sm.sx[m])) : __fmul_rn(sm.sx[m], sm.swg[gg]);
-    sm.rcp[m][gg] = __drcp_rn(static_cast<double>(d));
-  }
-  __syncthreads();
+  __syncthreads();                                   // s_w, the bias and the sums are in shared memory
 
   // ---------------- epilogue: U units x 16 rows x M tokens ----------------
   const int rows = U * kUnitRows;
@@ -661,9 +679,15 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
     int gi = 0;                                      // the row's group (scale)
 #pragma unroll
     for (int gg = 0; gg + 1 < kMaxGroups; ++gg) gi += (gg + 1 < a.ngroups && n >= a.group_end[gg]) ? 1 : 0;
+    // d = s_x s_w of the token and the row's group (on a bf16 module
+    // bf16(bf16(s_w) s_x)), used as the double 1 / d: RN_f32(a * (1/d)) is
+    // RN_f32(a / d) for every float32 (or bf16) numerator a -- a quotient of
+    // two floats lies at least 2^-49 (relative) from every float32 midpoint,
+    // and the double product is within 2^-52 of it
+    const float d = FAITHFUL ? bf16_round(__fmul_rn(bf16_round(sm.swg[gi]), sm.sx[m])) : __fmul_rn(sm.sx[m], sm.swg[gi]);
+    const double r = __drcp_rn(static_cast<double>(d));
     float y32;
-    const double r = sm.rcp[m][gi];
-    if (!a.faithful) {
+    if (!FAITHFUL) {
       y32 = __double2float_rn(static_cast<double>(static_cast<float>(accv)) * r);
       if (a.bias) y32 = __fadd_rn(y32, bf16_bits_to_f32(bias_s[rl]));
     } else {
@@ -679,9 +703,9 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
   }
 }
 
-template <int NT>
+template <int NT, bool FAITHFUL>
 cudaError_t launch_nt(const DecodeArgs& a, const DecodePlan& p, cudaStream_t stream) {
-  auto kern = decode_kernel<NT>;
+  auto kern = decode_kernel<NT, FAITHFUL>;
   static unsigned long long attr_done = 0;        // one bit per device
   cudaError_t ea = set_smem_attr_once(kern, 227 * 1024, &attr_done);
   if (ea != cudaSuccess) return ea;
@@ -704,50 +728,46 @@ cudaError_t launch_nt(const DecodeArgs& a, const DecodePlan& p, cudaStream_t str
 // flight per CTA.  A streaming probe on B200 (chained launches, all SMs)
 // found 64 KB per CTA as fast as any deeper ring at every decode shape, and
 // 128 KB per CTA slower.
-#ifndef BITLINEAR_DECODE_KC
-#define BITLINEAR_DECODE_KC 1       // chunks (2 KB each) per item
-#endif
 #ifndef BITLINEAR_DECODE_RING
 #define BITLINEAR_DECODE_RING 4     // largest ring per warp
 #endif
 
-DecodePlan plan_decode(int M, int N, int K, int num_sms) {
+DecodePlan plan_decode(int M, int N, int K, int num_sms, bool direct) {
   DecodePlan p;
   const int units_total = (N + kUnitRows - 1) / kUnitRows;
   p.grid = units_total < num_sms ? units_total : num_sms;
   if ((units_total + p.grid - 1) / p.grid > kMaxUnits) p.grid = (units_total + kMaxUnits - 1) / kMaxUnits;
   p.units_max = (units_total + p.grid - 1) / p.grid;
-  const int nchunks = (K + kBoxK - 1) / kBoxK;
-  // items of kc chunks when K has that many, else one chunk
-  p.kc = (BITLINEAR_DECODE_KC > 1 && nchunks >= 2 * BITLINEAR_DECODE_KC) ? BITLINEAR_DECODE_KC : 1;
+  // items of one chunk (the copy offsets of a lane are fixed for that size)
+  p.kc = 1;
   p.tail = (K % kBoxK) != 0;
-  p.slot_bytes = static_cast<size_t>(p.kc) * kSubBytes;
+  p.slot_bytes = kSubBytes;
   // shared-memory budget: two CTAs per SM for the 8-token kernel (the next
-  // kernel on the stream can start beside this one), one for 16 tokens
+  // kernel on the stream can start beside this one; the 16-token kernel's
+  // registers allow one); int8 x is not staged in shared memory
+  const int mx = direct ? 0 : M;
   const long long budget = M <= 8 ? 110 * 1024 : 220 * 1024;
-  const long long room = budget - static_cast<long long>(smem_layout(M, 0, p.slot_bytes, p.units_max).total);
+  const long long room = budget - static_cast<long long>(smem_layout(M, mx, 0, p.slot_bytes, p.units_max).total);
   long long ring = room > 0 ? room / (static_cast<long long>(kWarps) * static_cast<long long>(p.slot_bytes)) : 0;
   ring = ring > BITLINEAR_DECODE_RING ? BITLINEAR_DECODE_RING : ring;
-  if (ring < 2 && p.kc > 1) {                     // fall back to single-chunk loads
-    p.kc = 1;
-    p.slot_bytes = kSubBytes;
-    ring = room > 0 ? room / (static_cast<long long>(kWarps) * kSubBytes) : 0;
-    ring = ring > BITLINEAR_DECODE_RING ? BITLINEAR_DECODE_RING : ring;
-  }
   p.ring = ring < 1 ? 1 : static_cast<int>(ring);
-  p.smem = smem_layout(M, p.ring, p.slot_bytes, p.units_max).total;
+  p.smem = smem_layout(M, mx, p.ring, p.slot_bytes, p.units_max).total;
   return p;
 }
 
 cudaError_t launch_decode(DecodeArgs a, int num_sms, cudaStream_t stream) {
   if (a.M <= 0) return cudaSuccess;
-  const DecodePlan p = plan_decode(a.M, a.N, a.K, num_sms);
+  // above 8 tokens the activations come quantised, with their row sums
+  if (a.M > 8 && (a.xq == nullptr || a.rowsum == nullptr)) return cudaErrorInvalidValue;
+  if (a.xq != nullptr && a.rowsum == nullptr) return cudaErrorInvalidValue;
+  const DecodePlan p = plan_decode(a.M, a.N, a.K, num_sms, a.xq != nullptr);
   a.ring = p.ring;
   a.units_max = p.units_max;
   a.kc = p.kc;
   a.tail = p.tail;
   if (p.smem > 227 * 1024) return cudaErrorInvalidValue;
-  return a.M <= 8 ? launch_nt<1>(a, p, stream) : launch_nt<2>(a, p, stream);
+  if (a.faithful) return a.M <= 8 ? launch_nt<1, true>(a, p, stream) : launch_nt<2, true>(a, p, stream);
+  return a.M <= 8 ? launch_nt<1, false>(a, p, stream) : launch_nt<2, false>(a, p, stream);
 }
 
 }  // namespace bitlinear

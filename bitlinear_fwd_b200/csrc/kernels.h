@@ -121,8 +121,9 @@ cudaError_t launch_tc_i8_peak(int iters, int num_sms, uint32_t* status, cudaStre
 // ---- decode engine, M <= 16 (gemv_decode.cu) --------------------------------
 struct DecodeArgs {
   const uint16_t* x;      // bf16 [M, K], quantised inside the kernel; or null
-  const int8_t* xq;       // int8 [M, K] with s_x when x is null
+  const int8_t* xq;       // int8 [M, K] with s_x and rowsum when x is null
   const float* s_x;       // [M]
+  const int32_t* rowsum;  // [M] sum of q per token, with xq
   const uint8_t* packed;  // [N, K/4]
   const float* w_scale;   // [ngroups]
   const uint16_t* bias;   // [N] or null
@@ -153,7 +154,7 @@ struct DecodePlan {
   int grid, units_max, ring, kc, tail;
   size_t slot_bytes, smem;
 };
-DecodePlan plan_decode(int M, int N, int K, int num_sms);
+DecodePlan plan_decode(int M, int N, int K, int num_sms, bool direct);
 cudaError_t launch_decode(DecodeArgs a, int num_sms, cudaStream_t stream);
 
 // ---- prefill engine, tcgen05 GEMM (gemm_prefill.cu) -------------------------
