@@ -915,6 +915,49 @@ def reference_arm(args):
 
 # ---------------------------------------------------------------------------
 
+def run_case(name):
+    """One small case of one kernel, for ncu captures of a single kernel
+    (no timing, no JSON line): seeded inputs at the sizes the profiles in
+    profiles/ quote, each call repeated so that a capture can skip the first."""
+    import bitlinear_fwd_b200 as bl
+    dev = "cuda"
+    if name in ("gemm", "gemm8640"):
+        M, K, N = (2048, 3200, 8640) if name == "gemm" else (2048, 8640, 3200)
+        packed, s_w, _ = bl.bitlinear_pack_weights(synth.normal_f32(1, 1, (N, K), 0.02, device=dev))
+        x = synth.normal_bf16(1, 2, (M, K), device=dev)
+        for _ in range(3):
+            bl.bitlinear_forward(x, packed, s_w)
+    elif name == "decode":
+        K, N = 4096, 11008
+        packed, s_w, _ = bl.bitlinear_pack_weights(synth.normal_f32(1, 1, (N, K), 0.02, device=dev))
+        b = synth.normal_bf16(1, 3, (N,), 0.01, device=dev)
+        for M in (1, 4, 16):
+            bl.bitlinear_forward(synth.normal_bf16(1, 2 + M, (M, K), device=dev), packed, s_w, b,
+                                 flags=bl.WEIGHTS_RESIDENT)
+    elif name == "actq":
+        x = synth.normal_bf16(1, 2, (8192, 8640), device=dev)
+        for _ in range(2):
+            bl.bitlinear_quant_act(x)
+    elif name == "pack":
+        w = synth.normal_f32(1, 1, (28672, 8192), 0.01, device=dev)
+        for _ in range(2):
+            bl.bitlinear_pack_weights(w)
+    elif name == "dequant":
+        packed, s_w, _ = bl.bitlinear_pack_weights(synth.normal_f32(1, 1, (28672, 8192), 0.01, device=dev))
+        for _ in range(2):
+            bl.bitlinear_dequant_weights(packed, s_w)
+    elif name == "ksplit":
+        M, K, N = 4, 4096, 8192
+        x = synth.normal_bf16(1, 2, (M, K), device=dev)
+        packed, s_w, _ = bl.bitlinear_pack_weights(synth.normal_f32(1, 1, (N, K), 0.02, device=dev))
+        am = bl.bitlinear_act_absmax(x)
+        part = bl.bitlinear_forward_partial(x, am, packed)
+        for _ in range(2):
+            bl.bitlinear_epilogue_sum([part, part], am, s_w)
+    torch.cuda.synchronize()
+    print(json.dumps({"case": name, "ok": True}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -929,7 +972,13 @@ def main():
     ap.add_argument("--only", choices=["decode", "prefill", "dequant", "stack3b"], default=None,
                     help="run one workload only (profiling runs; no JSON contract line)")
     ap.add_argument("--copies", type=int, default=0, help="force the number of rotating weight copies")
+    ap.add_argument("--case", choices=["decode", "gemm", "gemm8640", "actq", "pack", "dequant", "ksplit"],
+                    default=None, help="run one small case of one kernel for an ncu capture, then exit")
     args = ap.parse_args()
+    if args.case:
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        run_case(args.case)
+        return 0
     args.warmup = max(3, args.warmup)
 
     if args.impl == "reference":

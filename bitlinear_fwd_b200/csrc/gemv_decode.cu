@@ -395,70 +395,43 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
       sm.rsum[threadIdx.x] = a.rowsum[threadIdx.x];
     }
   } else if (NT == 1 && single) {
-    uint4 v[kHold * NT][2];
+    // warp w takes token m = w / P; a lane holds C <= kHold chunks of it
+    const int m = warp / P;
+    const bool mine = m < M;
+    uint4 v[kHold][2];
 #pragma unroll
-    for (int i = 0; i < kHold * NT; ++i) {
-      const int j = (NT == 2 && i >= C) ? 1 : 0;     // token slot of this warp
-      const int m = warp / P + j * mstep;
-      const int ii = i - j * C;
-      v[i][0] = v[i][1] = make_uint4(0, 0, 0, 0);
-      if (i < NT * C && m < M && ch_first + ii * 32 * P < cpr) {
-        v[i][0] = __ldg(xl[j] + ii * xstep);
-        v[i][1] = __ldg(xl[j] + ii * xstep + 1);
+    for (int i = 0; i < kHold; ++i)
+      if (i < C) {
+        const bool in = mine && ch_first + i * 32 * P < cpr;
+        v[i][0] = in ? __ldg(xl[0] + i * xstep) : make_uint4(0, 0, 0, 0);
+        v[i][1] = in ? __ldg(xl[0] + i * xstep + 1) : make_uint4(0, 0, 0, 0);
       }
-    }
-    uint32_t mx[NT];
+    uint32_t mx = 0;
 #pragma unroll
-    for (int j = 0; j < NT; ++j) mx[j] = 0;
-#pragma unroll
-    for (int i = 0; i < kHold * NT; ++i) {
-      if (i < NT * C) {
-        const uint32_t am = absmax16_bits(v[i][0], v[i][1]);   // zeros where nothing was loaded
-        if (NT == 2 && i >= C) mx[NT - 1] = max(mx[NT - 1], am);
-        else mx[0] = max(mx[0], am);
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < NT; ++j) {
-      const int m = warp / P + j * mstep;
-      const uint32_t r = __reduce_max_sync(0xffffffffu, mx[j]);
-      if (lane == 0 && m < M) atomicMax(&sm.amax[m], r);
-    }
+    for (int i = 0; i < kHold; ++i)
+      if (i < C) mx = max(mx, absmax16_bits(v[i][0], v[i][1]));   // zeros where nothing was loaded
+    mx = __reduce_max_sync(0xffffffffu, mx);
+    if (lane == 0 && mine) atomicMax(&sm.amax[m], mx);
     __syncthreads();
-    float sxr[NT];
-#pragma unroll
-    for (int j = 0; j < NT; ++j) {
-      const int m = min(warp / P + j * mstep, M - 1);
-      sxr[j] = act_scale(bf16_bits_to_f32(sm.amax[m]), FAITHFUL);
-    }
+    const float sxm = act_scale(bf16_bits_to_f32(sm.amax[min(m, M - 1)]), FAITHFUL);
     if (threadIdx.x < M) {
-      const float sxv = act_scale(bf16_bits_to_f32(sm.amax[threadIdx.x]), FAITHFUL);
+      // warp 0 holds token 0's scale already
+      const float sxv = threadIdx.x == 0 ? sxm : act_scale(bf16_bits_to_f32(sm.amax[threadIdx.x]), FAITHFUL);
       sm.sx[threadIdx.x] = sxv;
       if (blockIdx.x == 0 && a.sx_out) a.sx_out[threadIdx.x] = sxv;
     }
-    int sum[NT];
+    int sum = 0;
 #pragma unroll
-    for (int j = 0; j < NT; ++j) sum[j] = 0;
-#pragma unroll
-    for (int i = 0; i < kHold * NT; ++i) {
-      const int j = (NT == 2 && i >= C) ? 1 : 0;
-      const int m = warp / P + j * mstep;
-      const int ch = ch_first + (i - j * C) * 32 * P;
-      if (i < NT * C && m < M && ch < cpr) {
-        int ps = 0;
-        const uint4 qv = quant16(v[i][0], v[i][1], j ? sxr[NT - 1] : sxr[0], ps, FAITHFUL);
-        if (j) sum[NT - 1] += ps;
-        else sum[0] += ps;
+    for (int i = 0; i < kHold; ++i) {
+      const int ch = ch_first + i * 32 * P;
+      if (i < C && mine && ch < cpr) {
+        const uint4 qv = quant16(v[i][0], v[i][1], sxm, sum, FAITHFUL);
         *reinterpret_cast<uint4*>(xs + m * S + 16 * xs_chunk(ch)) = qv;
         if (blockIdx.x == 0 && a.xq_out) *reinterpret_cast<uint4*>(a.xq_out + static_cast<size_t>(m) * K + 16 * ch) = qv;
       }
     }
-#pragma unroll
-    for (int j = 0; j < NT; ++j) {
-      const int m = warp / P + j * mstep;
-      const int r = __reduce_add_sync(0xffffffffu, sum[j]);
-      if (lane == 0 && m < M) atomicAdd(&sm.rsum[m], r);
-    }
+    sum = __reduce_add_sync(0xffffffffu, sum);
+    if (lane == 0 && mine) atomicAdd(&sm.rsum[m], sum);
   } else if (NT == 1 && a.x) {
     for (int m = warp / P; m < M; m += mstep) {
       const uint4* row = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(m) * K);
