@@ -123,6 +123,17 @@ __device__ __forceinline__ int xs_chunk(int ch) { return ch ^ (((ch >> 3) & 1) <
 
 __device__ __forceinline__ int mma_row_to_box(int g) { return (g >> 1) | ((g & 1) << 2); }
 
+// Place of (row, token) in a unit's int32 sums [16 rows][ntok tokens]: the
+// token index is rotated by a function of the row so that the 32 lanes of
+// one red.shared (rows pi(g) or pi(g) + 8, tokens 2t or 2t + 1) hit 32
+// different banks; a plain [row][token] layout put two (8 tokens) or four
+// (16 tokens) rows in one bank group.
+template <int NTOK>
+__device__ __forceinline__ int sum_idx(int row, int m) {
+  const int f = NTOK == 8 ? ((row >> 2) & 1) : (((row >> 1) & 1) + 8 * ((row >> 2) & 1));
+  return row * NTOK + ((m + f) & (NTOK - 1));
+}
+
 // largest |x| of 16 bf16 values, as bf16 bits (finite values order like bits & 0x7FFF)
 __device__ __forceinline__ uint32_t absmax16_bits(uint4 lo, uint4 hi) {
   uint32_t m = 0;
@@ -618,12 +629,12 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
           cv[rr] = acc[0][nt][rr] + (acc[1][nt][rr] >> 2) + (acc[2][nt][rr] >> 4) + (acc[3][nt][rr] >> 6);
         const int m0 = nt * 8 + 2 * t;
         if (m0 < M) {
-          red_shared_add(au + r0 * NTOK + m0, cv[0]);
-          red_shared_add(au + (r0 + 8) * NTOK + m0, cv[2]);
+          red_shared_add(au + sum_idx<NTOK>(r0, m0), cv[0]);
+          red_shared_add(au + sum_idx<NTOK>(r0 + 8, m0), cv[2]);
         }
         if (m0 + 1 < M) {
-          red_shared_add(au + r0 * NTOK + m0 + 1, cv[1]);
-          red_shared_add(au + (r0 + 8) * NTOK + m0 + 1, cv[3]);
+          red_shared_add(au + sum_idx<NTOK>(r0, m0 + 1), cv[1]);
+          red_shared_add(au + sum_idx<NTOK>(r0 + 8, m0 + 1), cv[3]);
         }
       }
     }
@@ -648,7 +659,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
     const int m = idx / rows, rl = idx - m * rows;
     const int n = u_begin * kUnitRows + rl;
     if (n >= N) continue;
-    const int accv = acc_s[rl * NTOK + m] - sm.rsum[m];
+    const int accv = acc_s[(rl >> 4) * kUnitRows * NTOK + sum_idx<NTOK>(rl & 15, m)] - sm.rsum[m];
     int gi = 0;                                      // the row's group (scale)
 #pragma unroll
     for (int gg = 0; gg + 1 < kMaxGroups; ++gg) gi += (gg + 1 < a.ngroups && n >= a.group_end[gg]) ? 1 : 0;
