@@ -5,23 +5,27 @@
 // packed weights once.
 //
 // Work split.  The N weight rows form 16-row units; the grid is one wave of
-// CTAs (at most one per SM) and CTA c owns a contiguous, balanced range of
-// units over the whole of K.  CTAs never talk to each other.  K is cut into
-// 512-k chunks (the last one maybe partial), and the chunks into rounds of
-// eight (4096 k: the x of one round sits in shared memory as int8).
+// CTAs (one per SM; two per SM for the 8-token kernel on matrices of 8 or
+// more units per SM) and CTA c owns a contiguous, balanced range of units
+// over the whole of K.  CTAs never talk to each other.  K is cut into 512-k
+// chunks (the last one maybe partial), and the chunks into rounds of eight
+// (4096 k: the x of one round sits in shared memory as int8).
 //
 // Inside a CTA every one of the 8 warps streams and computes:
-//   * An item is one chunk of one unit (16 rows x 128 bytes).  A round's
-//     items are numbered chunk-major, and warp w takes the contiguous w-th
-//     eighth of them, so a warp's consecutive items share a chunk (its x
-//     fragment is loaded once per chunk) and the shares differ by at most
-//     one item.
+//   * An item is one chunk of two consecutive units in the 8-token kernel
+//     (32 rows x 128 bytes: one wait, one cursor step and one x fragment
+//     per 4 KB, and eight independent MMA chains) and of one unit in the
+//     16-token kernel.  A round's items are numbered chunk-major, and warp w
+//     takes the contiguous w-th eighth of them, so a warp's consecutive
+//     items share a chunk (its x fragment is loaded once per chunk) and the
+//     shares differ by at most one item.
 //   * Each warp streams its own items through its own ring of shared-memory
 //     slots: every lane copies 4 x 16 bytes of an item with cp.async, at
 //     per-lane offsets fixed for the whole kernel (128-byte rows, written in
 //     the 128-byte-swizzled order that keeps the fragment reads below
 //     conflict-free), one copy group per item, up to `ring` items ahead;
-//     pieces beyond N or K are zero-filled.  The warp waits for the oldest
+//     pieces beyond N or K, and the missing unit of a CTA's last pair, are
+//     zero-filled.  The warp waits for the oldest
 //     group (once for all of them when its whole share fitted in the ring)
 //     and refills its slot once it has read it.  No warp ever waits for
 //     another warp's copies.  When the weights are resident the first
@@ -33,7 +37,11 @@
 //     s_x) as int8 into shared memory, one round at a time, with the sum of q
 //     per token.  For K <= 4096 each lane's share of x (at most 8 x 32
 //     bytes per token) is read once and held in registers between the two
-//     steps; otherwise x is read again for the quantising step.
+//     steps; otherwise x is read again for the quantising step.  With one
+//     token and a full round, warp w quantises exactly the chunk its own
+//     items use, so no block barrier separates the quantising from the
+//     items.  A lane's x fragment loads use offsets worked out once (lanes
+//     of tokens that do not exist read 512 zero bytes).
 //   * int8 x (above 8 tokens the act-quant kernel quantises x once; also the
 //     pre-quantised and K-split calls): the scales and row sums are read, and
 //     each warp loads its x fragments straight from global memory.
@@ -41,8 +49,10 @@
 //     256-k half and issues mma.sync m16n8k32 (weights as A, u8; tokens as B,
 //     s8; a second 8-token tile for M > 8).  The codes c = u + 1 enter
 //     unshifted: A_i = word & (0x03030303 << 2i) holds 4^i c per byte lane,
-//     so field i accumulates 4^i sum(c q); the fields are combined with
-//     exact shifts and added to the unit's int32 sums in shared memory.
+//     so field i accumulates 4^i sum(c q); the fields of one unit are
+//     combined with exact shifts before the next unit's MMAs (one unit's
+//     field accumulators live at a time) and added to the unit's int32 sums
+//     in shared memory.
 //   * Epilogue: acc = sum(c q) - sum(q) = sum(u q); y = acc / (s_x s_w)
 //     (+ bias) -> bf16, with s_w the scale of the row's layer when several
 //     layers are stacked, the division done as a product with the double
@@ -80,6 +90,10 @@ constexpr int kQB = 2;                                // the same in the quantis
 constexpr int kHold = 8;                              // 32-byte x chunks per lane and token held in
                                                       // registers by the one-pass path
 constexpr uint32_t kCodeMask = 0x03030303u;
+// units per item: two for the 8-token kernel (one wait, one cursor step and
+// one x fragment per 4 KB, eight independent MMA chains); one for the
+// 16-token kernel, whose accumulators and x fragments fill its registers
+__host__ __device__ constexpr int units_per_item(int nt) { return nt == 1 ? 2 : 1; }
 constexpr float kRoundMagic = 12582912.0f;            // 1.5 * 2^23
 
 __device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
@@ -195,6 +209,7 @@ __device__ __forceinline__ int bytesum16(uint4 v, int sum) {
 }
 
 struct SmemTail {
+  uint4 zero[32];                    // 512 zero bytes: the x fragment of a token that does not exist
   uint64_t stall;                    // never signalled (forced-timeout test hook)
   uint32_t amax[16];                 // absmax per token (bf16 bits)
   int rsum[16];                      // sum of q per token
@@ -224,43 +239,53 @@ __host__ __device__ SmemLayout smem_layout(int M, int xrows, int ring, size_t sl
   return L;
 }
 
-// The items of one warp, in order.  A round's chunks (the last one of K maybe
-// partial) form groups of kc, the last group maybe shorter; its T = groups x U
-// items are numbered chunk group major (item j: group j / U, unit j % U), and
-// warp w takes the contiguous range [w T / 8, (w + 1) T / 8) of them.  The
-// shares differ by at most one item, and the consecutive items of a warp
-// mostly share a chunk group, so its x fragment is loaded once per group.
+// The items of one warp, in order.  An item is one chunk of UP consecutive
+// units (UP = 2 for the 8-token kernel, 1 for the 16-token one); a CTA's U
+// units form PU = ceil(U / UP) unit groups, the last one maybe short.  A
+// round's T = chunks x PU items are numbered chunk major (item j: chunk j /
+// PU, group j % PU), and warp w takes the contiguous range [w T / 8, (w + 1)
+// T / 8) of them.  The shares differ by at most one item, and the
+// consecutive items of a warp mostly share a chunk, so its x fragment is
+// loaded once per chunk.  The cursor moves by increments; only a new round
+// costs divisions.
 struct ItemCursor {
-  int r, g, u, left;                               // round, item (group g, unit u), items left in the round
+  int r, g, p, left;                               // round, item (chunk g, group p), items left in the round
   __device__ __forceinline__ static int chunks(int r, int nchunks) {
     return min(nchunks - kRoundChunks * r, kRoundChunks);
   }
-  __device__ __forceinline__ static int groups(int r, int nchunks, int kc) { return (chunks(r, nchunks) + kc - 1) / kc; }
-  __device__ __forceinline__ void begin_round(int warp, int nchunks, int kc, int U) {
-    const int T = groups(r, nchunks, kc) * U;
+  __device__ __forceinline__ void begin_round(int warp, int nchunks, int PU) {
+    const int T = chunks(r, nchunks) * PU;
     const int jb = warp * T / kWarps;
     left = (warp + 1) * T / kWarps - jb;
-    g = jb / U;
-    u = jb - g * U;
+    g = jb / PU;
+    p = jb - g * PU;
   }
-  __device__ __forceinline__ void settle(int warp, int nround, int nchunks, int kc, int U) {
+  // moves past empty rounds; true when the round changed
+  __device__ __forceinline__ bool settle(int warp, int nround, int nchunks, int PU) {
+    bool moved = false;
     while (r < nround && left == 0) {
       ++r;
-      if (r < nround) begin_round(warp, nchunks, kc, U);
+      moved = true;
+      if (r < nround) begin_round(warp, nchunks, PU);
     }
+    return moved;
   }
-  __device__ __forceinline__ void start(int warp, int nround, int nchunks, int kc, int U) {
+  __device__ __forceinline__ void start(int warp, int nround, int nchunks, int PU) {
     r = 0;
-    begin_round(warp, nchunks, kc, U);
-    settle(warp, nround, nchunks, kc, U);
+    begin_round(warp, nchunks, PU);
+    settle(warp, nround, nchunks, PU);
   }
-  __device__ __forceinline__ void next(int warp, int nround, int nchunks, int kc, int U) {
+  // next item; true when it is not the group after the current one in the
+  // same chunk (a new chunk or a new round)
+  __device__ __forceinline__ bool next(int warp, int nround, int nchunks, int PU) {
     --left;
-    if (++u == U) {
-      u = 0;
+    bool jump = false;
+    if (++p == PU) {
+      p = 0;
       ++g;
+      jump = true;
     }
-    settle(warp, nround, nchunks, kc, U);
+    return settle(warp, nround, nchunks, PU) || jump;
   }
 };
 
@@ -268,15 +293,15 @@ template <int NT, bool FAITHFUL>
 __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
     decode_kernel(const DecodeArgs a) {
   constexpr int NTOK = NT * 8;
+  constexpr int UP = units_per_item(NT);             // units per item
+  constexpr int kSlotBytes = UP * kSubBytes;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   const int ring = a.ring;
-  const int kc = a.kc;                               // chunks per 3-D item
-  const size_t slot_bytes = static_cast<size_t>(kc) * kSubBytes;
   // int8 x with its row sums is read straight from global memory (no x in
   // shared memory); bf16 x is quantised into shared memory
   const bool direct = a.xq != nullptr && a.rowsum != nullptr;
-  const SmemLayout L = smem_layout(a.M, direct ? 0 : a.M, ring, slot_bytes, a.units_max);
+  const SmemLayout L = smem_layout(a.M, direct ? 0 : a.M, ring, kSlotBytes, a.units_max);
   int8_t* xs = reinterpret_cast<int8_t*>(base + L.xs);
   int* acc_s = reinterpret_cast<int*>(base + L.acc);            // [unit][row][token]
   uint16_t* bias_s = reinterpret_cast<uint16_t*>(base + L.bias);
@@ -290,10 +315,11 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
   const int units_total = (N + kUnitRows - 1) / kUnitRows;
   const int u_begin = static_cast<int>(static_cast<long long>(blockIdx.x) * units_total / gridDim.x);
   const int U = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * units_total / gridDim.x) - u_begin;
+  const int PU = (U + UP - 1) / UP;                 // unit groups of this CTA
   const int nchunks = (K + kBoxK - 1) / kBoxK;       // 512-k chunks, the last maybe partial
   const int nround = (K + kChunkK - 1) / kChunkK;
   const uint32_t row_bytes = static_cast<uint32_t>(K) / 4;
-  uint8_t* wring = base + L.ring + static_cast<size_t>(warp) * ring * slot_bytes;   // this warp's ring
+  uint8_t* wring = base + L.ring + static_cast<size_t>(warp) * ring * kSlotBytes;   // this warp's ring
 
   if (threadIdx.x == 0) {
     mbar_init(&sm.stall, 1);
@@ -304,38 +330,47 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
     sm.amax[threadIdx.x] = 0u;
     sm.rsum[threadIdx.x] = 0;
   }
+  if (threadIdx.x < 32) sm.zero[threadIdx.x] = make_uint4(0, 0, 0, 0);
   for (int i = threadIdx.x; i < U * kUnitRows * NTOK; i += kThreads) acc_s[i] = 0;
   __syncthreads();
 
   // ---- this warp's weight stream: every lane copies its own 16-byte
   // pieces of an item (row p >> 3, piece p & 7 of each 128-byte chunk row,
-  // p = lane, lane + 32, ...) into the slot's 128-byte-swizzled layout; one
-  // copy group per item; pieces beyond N or K are zero-filled
+  // p = lane, lane + 32, ..., per unit of the item) into the slot's
+  // 128-byte-swizzled layout; one copy group per item; pieces beyond N or K
+  // and units beyond the CTA's range are zero-filled
   ItemCursor ic;                                     // next item to issue
-  ic.start(warp, nround, nchunks, kc, U);
+  ic.start(warp, nround, nchunks, PU);
+  const ItemCursor cstart = ic;                      // the first item, for the consumer
   int islot = 0;                                     // ring slot of the next copy
-  // this lane's pieces of a chunk item (kc = 1): rows (lane >> 3) + 4 j,
-  // piece lane & 7 of each row, j = 0..3; their source and destination
-  // offsets are fixed, only the item's first row and chunk change
+  // this lane's pieces of a unit: rows (lane >> 3) + 4 j, piece lane & 7 of
+  // each row, j = 0..3; their source and destination offsets are fixed, only
+  // the item's first row and chunk change
   const int prow = lane >> 3, pq = lane & 7;
-  const uint32_t psrc = static_cast<uint32_t>(prow) * row_bytes + 16u * pq;   // + 4 j row_bytes
+  const uint32_t psrc = static_cast<uint32_t>(prow) * row_bytes + 16u * pq;   // + (16 e + 4 j) row_bytes
   const uint32_t pdst0 = prow * 128 + ((pq ^ prow) << 4);          // rows prow, prow + 8
   const uint32_t pdst1 = (prow + 4) * 128 + ((pq ^ (prow + 4)) << 4);   // rows prow + 4, prow + 12
+  // rows of this CTA's units that exist (the last unit of the matrix may be short)
+  const int lim0 = min(U * kUnitRows, N - u_begin * kUnitRows);
   auto issue_next = [&]() {
     if (ic.r < nround) {
       const int c = kRoundChunks * ic.r + ic.g;     // chunk of the item
-      const int n0 = (u_begin + ic.u) * kUnitRows;  // first row of the unit
-      uint8_t* dst = wring + islot * slot_bytes;
+      const int r0g = UP * kUnitRows * ic.p;         // first row of the item in the CTA's range
+      const int lim = lim0 - r0g;                    // rows of the item's units that exist
+      uint8_t* dst = wring + islot * kSlotBytes;
       const bool kin = static_cast<uint32_t>(c) * (kBoxK / 4) + 16u * pq < row_bytes;
-      const uint8_t* src = a.packed + static_cast<size_t>(n0) * row_bytes + static_cast<uint32_t>(c) * (kBoxK / 4) + psrc;
+      const uint8_t* src = a.packed + static_cast<size_t>(u_begin * kUnitRows + r0g) * row_bytes +
+                           static_cast<uint32_t>(c) * (kBoxK / 4) + psrc;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const bool valid = kin && n0 + prow + 4 * j < N;
-        cp_async16(dst + ((j & 1) ? pdst1 : pdst0) + (j >> 1) * 1024, valid ? src + static_cast<size_t>(4 * j) * row_bytes : a.packed,
-                   valid ? 16u : 0u);
-      }
+      for (int e = 0; e < UP; ++e)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const bool valid = kin && kUnitRows * e + prow + 4 * j < lim;
+          cp_async16(dst + e * kSubBytes + ((j & 1) ? pdst1 : pdst0) + (j >> 1) * 1024,
+                     valid ? src + static_cast<size_t>(kUnitRows * e + 4 * j) * row_bytes : a.packed, valid ? 16u : 0u);
+        }
       islot = islot + 1 == ring ? 0 : islot + 1;
-      ic.next(warp, nround, nchunks, kc, U);
+      ic.next(warp, nround, nchunks, PU);
     }
     cp_async_commit();                               // one group per call, empty when nothing is left
   };
@@ -474,7 +509,14 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
   } else {
     if (threadIdx.x < M) sm.sx[threadIdx.x] = a.s_x[threadIdx.x];
   }
-  __syncthreads();
+  // One token and a full round of 8 chunks in the one-pass path: warp w
+  // quantised exactly chunk w, and its items are exactly the units of chunk
+  // w, so it reads only x it wrote itself; the scales and row sums are read
+  // after the barrier before the epilogue.
+  if (NT == 1 && single && M == 1 && nchunks == kRoundChunks)
+    __syncwarp();
+  else
+    __syncthreads();
 
   // forced-timeout test: a wait that nothing completes runs out, and the
   // CTA takes the same path as after any wait that gives up
@@ -482,14 +524,18 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
   ok = __all_sync(0xffffffffu, ok);
 
   const int r0 = mma_row_to_box(g);                  // sub-box rows r0 and r0 + 8
-  ItemCursor cc;                                     // next item to consume
-  cc.start(warp, nround, nchunks, kc, U);
+  ItemCursor cc = cstart;                            // next item to consume
   int cslot = 0;                                     // ring slot of the next item to consume
   // When the prologue requested every item of this warp (they fit in its
   // ring), one wait for all copies replaces the per-item waits.
   const bool per_item_wait = ic.r < nround;
   bool first_wait = true;
   int xchunk = -1;                                   // round-local chunk of the x fragment held
+  // bf16 x (8 tokens at most): this lane's token row in shared memory, or
+  // the zero bytes; the offsets of its pair-p pieces within a 256-k half
+  const uint8_t* xtok = g < M ? reinterpret_cast<const uint8_t*>(xs) + g * S + 64 * t
+                              : reinterpret_cast<const uint8_t*>(sm.zero);
+  const int xpo[2] = {32 * (t >> 1), 32 * (1 ^ (t >> 1))};
   uint32_t xw[2][2][NT][8];                          // [v][pair][token tile][word]
   for (int r = 0; r < nround; ++r) {
     const int c0 = r * kChunkK;
@@ -560,81 +606,110 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
         __syncwarp();
         first_wait = false;
       }
-      const int u = cc.u;
-      const int lc = cc.g;                           // round-local chunk of the item (one chunk per item)
+      const int ug = cc.p;                           // unit group of the item
+      const int lc = cc.g;                           // round-local chunk of the item
       if (lc != xchunk) {
+        if (NT == 2 || direct) {                    // bf16 x comes with 8 tokens at most
 #pragma unroll
-        for (int v = 0; v < 2; ++v)
+          for (int v = 0; v < 2; ++v)
+#pragma unroll
+            for (int pr = 0; pr < 2; ++pr)
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt) {
+                const int m = nt * 8 + g;
+#pragma unroll
+                for (int c2 = 0; c2 < 2; ++c2) {
+                  // every lane loads (a token and chunk that exist where its
+                  // own do not) and keeps zeros for missing tokens and k
+                  const int xc = 32 * lc + 16 * v + 4 * t + 2 * pr + c2;    // 16-byte chunk in the round
+                  const bool xin = m < M && 16 * xc < K - r * kChunkK;
+                  const int mr = xin ? m : 0, xr = xin ? xc : 0;
+                  uint4 xv = __ldg(reinterpret_cast<const uint4*>(a.xq + static_cast<size_t>(mr) * K + r * kChunkK) + xr);
+                  if (!xin) xv = make_uint4(0, 0, 0, 0);
+                  xw[v][pr][nt][4 * c2 + 0] = xv.x; xw[v][pr][nt][4 * c2 + 1] = xv.y;
+                  xw[v][pr][nt][4 * c2 + 2] = xv.z; xw[v][pr][nt][4 * c2 + 3] = xv.w;
+                }
+              }
+        } else {
+          // chunk lc of this lane's token in shared memory (the 512 zero
+          // bytes for a token that does not exist); the 16-byte pieces are at
+          // 256 v + 64 t + 32 (pr ^ (t >> 1)) + 16 c2, the swizzle of
+          // xs_chunk written out for this lane
+          const uint8_t* xb = xtok + (g < M ? 512 * lc : 0);
+#pragma unroll
+          for (int v = 0; v < 2; ++v)
+#pragma unroll
+            for (int pr = 0; pr < 2; ++pr)
+#pragma unroll
+              for (int c2 = 0; c2 < 2; ++c2) {
+                const uint4 xv = *reinterpret_cast<const uint4*>(xb + xpo[pr] + 256 * v + 16 * c2);
+                xw[v][pr][0][4 * c2 + 0] = xv.x; xw[v][pr][0][4 * c2 + 1] = xv.y;
+                xw[v][pr][0][4 * c2 + 2] = xv.z; xw[v][pr][0][4 * c2 + 3] = xv.w;
+              }
+        }
+        xchunk = lc;
+      }
+      // per unit: 16 MMAs in four independent chains (one per field), then
+      // the fields -> one sum per output (4^i sum(c q) >> 2i is exact: 64 * 2
+      // * 127 * 512 < 2^31); only one unit's field accumulators are live
+      int cv[UP][NT][4];
+      const uint8_t* box = wring + s * kSlotBytes;
+#pragma unroll
+      for (int e = 0; e < UP; ++e) {
+        int acc[4][NT][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr) acc[i][nt][rr] = 0;
+#pragma unroll
+        for (int v = 0; v < 2; ++v) {
+          const int cw = 4 * v + t;                  // 16-byte chunk of the 128-byte row
+          const uint4 wa = *reinterpret_cast<const uint4*>(box + e * kSubBytes + r0 * 128 + ((cw ^ r0) << 4));
+          const uint4 wb = *reinterpret_cast<const uint4*>(box + e * kSubBytes + (r0 + 8) * 128 + ((cw ^ r0) << 4));
+          const uint32_t w0[4] = {wa.x, wa.y, wa.z, wa.w};
+          const uint32_t w1[4] = {wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
           for (int pr = 0; pr < 2; ++pr)
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-              const int m = nt * 8 + g;
+            for (int i = 0; i < 4; ++i) {
+              const uint32_t mask = kCodeMask << (2 * i);
+              const uint32_t a0 = w0[2 * pr] & mask, a1 = w1[2 * pr] & mask;
+              const uint32_t a2 = w0[2 * pr + 1] & mask, a3 = w1[2 * pr + 1] & mask;
 #pragma unroll
-              for (int c2 = 0; c2 < 2; ++c2) {
-                uint4 xv = make_uint4(0, 0, 0, 0);
-                const int xc = 32 * lc + 16 * v + 4 * t + 2 * pr + c2;    // 16-byte chunk in the round
-                if (m < M && (!direct || 16 * xc < K - r * kChunkK)) {
-                  if (direct)
-                    xv = __ldg(reinterpret_cast<const uint4*>(a.xq + static_cast<size_t>(m) * K + r * kChunkK) + xc);
-                  else
-                    xv = *reinterpret_cast<const uint4*>(xs + m * S + 16 * xs_chunk(xc));
-                }
-                xw[v][pr][nt][4 * c2 + 0] = xv.x; xw[v][pr][nt][4 * c2 + 1] = xv.y;
-                xw[v][pr][nt][4 * c2 + 2] = xv.z; xw[v][pr][nt][4 * c2 + 3] = xv.w;
-              }
+              for (int nt = 0; nt < NT; ++nt)
+                mma_u8s8(acc[i][nt], a0, a1, a2, a3, xw[v][pr][nt][i], xw[v][pr][nt][4 + i]);
             }
-        xchunk = lc;
-      }
-      int acc[4][NT][4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
+        }
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-          for (int rr = 0; rr < 4; ++rr) acc[i][nt][rr] = 0;
-      const uint8_t* box = wring + s * slot_bytes;
-#pragma unroll
-      for (int v = 0; v < 2; ++v) {
-        const int cw = 4 * v + t;                    // 16-byte chunk of the 128-byte row
-        const uint4 wa = *reinterpret_cast<const uint4*>(box + r0 * 128 + ((cw ^ r0) << 4));
-        const uint4 wb = *reinterpret_cast<const uint4*>(box + (r0 + 8) * 128 + ((cw ^ r0) << 4));
-        const uint32_t w0[4] = {wa.x, wa.y, wa.z, wa.w};
-        const uint32_t w1[4] = {wb.x, wb.y, wb.z, wb.w};
-#pragma unroll
-        for (int pr = 0; pr < 2; ++pr)
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint32_t mask = kCodeMask << (2 * i);
-            const uint32_t a0 = w0[2 * pr] & mask, a1 = w1[2 * pr] & mask;
-            const uint32_t a2 = w0[2 * pr + 1] & mask, a3 = w1[2 * pr + 1] & mask;
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-              mma_u8s8(acc[i][nt], a0, a1, a2, a3, xw[v][pr][nt][i], xw[v][pr][nt][4 + i]);
-          }
+          for (int rr = 0; rr < 4; ++rr)
+            cv[e][nt][rr] = acc[0][nt][rr] + (acc[1][nt][rr] >> 2) + (acc[2][nt][rr] >> 4) + (acc[3][nt][rr] >> 6);
       }
       // the slot is read: refill it with this warp's next item
       __syncwarp();
       cslot = cslot + 1 == ring ? 0 : cslot + 1;
-      cc.next(warp, nround, nchunks, kc, U);
+      cc.next(warp, nround, nchunks, PU);
       issue_next();
-      // fields -> the unit's sums (4^i sum(c q) >> 2i is exact: 64 * 2 * 127
-      // * 512 < 2^31)
-      int* au = acc_s + u * kUnitRows * NTOK;
+      // the units' sums; a short group's missing unit is skipped
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        int cv[4];
+      for (int e = 0; e < UP; ++e) {
+        const int u = UP * ug + e;
+        if (UP > 1 && u >= U) break;
+        int* au = acc_s + u * kUnitRows * NTOK;
 #pragma unroll
-        for (int rr = 0; rr < 4; ++rr)
-          cv[rr] = acc[0][nt][rr] + (acc[1][nt][rr] >> 2) + (acc[2][nt][rr] >> 4) + (acc[3][nt][rr] >> 6);
-        const int m0 = nt * 8 + 2 * t;
-        if (m0 < M) {
-          red_shared_add(au + sum_idx<NTOK>(r0, m0), cv[0]);
-          red_shared_add(au + sum_idx<NTOK>(r0 + 8, m0), cv[2]);
-        }
-        if (m0 + 1 < M) {
-          red_shared_add(au + sum_idx<NTOK>(r0, m0 + 1), cv[1]);
-          red_shared_add(au + sum_idx<NTOK>(r0 + 8, m0 + 1), cv[3]);
+        for (int nt = 0; nt < NT; ++nt) {
+          const int m0 = nt * 8 + 2 * t;
+          if (m0 < M) {
+            red_shared_add(au + sum_idx<NTOK>(r0, m0), cv[e][nt][0]);
+            red_shared_add(au + sum_idx<NTOK>(r0 + 8, m0), cv[e][nt][2]);
+          }
+          if (m0 + 1 < M) {
+            red_shared_add(au + sum_idx<NTOK>(r0, m0 + 1), cv[e][nt][1]);
+            red_shared_add(au + sum_idx<NTOK>(r0 + 8, m0 + 1), cv[e][nt][3]);
+          }
         }
       }
     }
@@ -719,13 +794,16 @@ cudaError_t launch_nt(const DecodeArgs& a, const DecodePlan& p, cudaStream_t str
 DecodePlan plan_decode(int M, int N, int K, int num_sms, bool direct) {
   DecodePlan p;
   const int units_total = (N + kUnitRows - 1) / kUnitRows;
-  p.grid = units_total < num_sms ? units_total : num_sms;
+  // One CTA per SM leaves room for the next kernel of the stream to start
+  // beside this one; on the widest matrices (8 units per SM or more) two
+  // 8-token CTAs per SM, both computing, stream faster.
+  const int cap = (M <= 8 && units_total >= 8 * num_sms) ? 2 * num_sms : num_sms;
+  p.grid = units_total < cap ? units_total : cap;
   if ((units_total + p.grid - 1) / p.grid > kMaxUnits) p.grid = (units_total + kMaxUnits - 1) / kMaxUnits;
   p.units_max = (units_total + p.grid - 1) / p.grid;
   // items of one chunk (the copy offsets of a lane are fixed for that size)
-  p.kc = 1;
   p.tail = (K % kBoxK) != 0;
-  p.slot_bytes = kSubBytes;
+  p.slot_bytes = static_cast<size_t>(units_per_item(M <= 8 ? 1 : 2)) * kSubBytes;
   // shared-memory budget: two CTAs per SM for the 8-token kernel (the next
   // kernel on the stream can start beside this one; the 16-token kernel's
   // registers allow one); int8 x is not staged in shared memory
@@ -747,7 +825,6 @@ cudaError_t launch_decode(DecodeArgs a, int num_sms, cudaStream_t stream) {
   const DecodePlan p = plan_decode(a.M, a.N, a.K, num_sms, a.xq != nullptr);
   a.ring = p.ring;
   a.units_max = p.units_max;
-  a.kc = p.kc;
   a.tail = p.tail;
   if (p.smem > 227 * 1024) return cudaErrorInvalidValue;
   if (a.faithful) return a.M <= 8 ? launch_nt<1, true>(a, p, stream) : launch_nt<2, true>(a, p, stream);

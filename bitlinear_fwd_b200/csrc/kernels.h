@@ -137,7 +137,7 @@ struct DecodeArgs {
   int ngroups;
   int group_end[kMaxGroups];
   int faithful;           // bf16-module rounding of the quantisation and the epilogue
-  int ring, units_max, kc, tail;  // set by launch_decode
+  int ring, units_max, tail;      // set by launch_decode
   int weights_early;      // the packed weights, w_scale and bias may be read before the dependency wait
   uint64_t wait_ns;       // limit of the main-loop waits (drains keep kWaitLimitNs)
   int stall;              // test hook: first wait on a barrier nothing signals
@@ -151,7 +151,7 @@ constexpr uint64_t kTestWaitLimitNs = 1000ull * 1000ull;   // 1 ms
 uint64_t launch_wait_ns();
 int launch_stall();
 struct DecodePlan {
-  int grid, units_max, ring, kc, tail;
+  int grid, units_max, ring, tail;
   size_t slot_bytes, smem;
 };
 DecodePlan plan_decode(int M, int N, int K, int num_sms, bool direct);
