@@ -81,6 +81,15 @@ def peaks():
     return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
 
 
+def forward_launches(M, K):
+    """Kernels one bitlinear_forward launches: the act-quant kernel and the
+    GEMM above 16 tokens; the decode kernel alone up to 8 tokens (and up to
+    K = 8192 from 2 tokens), else the act-quant kernel before it."""
+    if M > 16:
+        return 2
+    return 2 if (M > 8 or (M >= 2 and K > 8192)) else 1
+
+
 def decode_bytes(M, N, K, bias=True):
     """Algorithmic bytes of one BitLinear forward: 2-bit packed weights,
     bf16 x in, bf16 y out, bf16 bias, fp32 s_w."""
@@ -363,7 +372,7 @@ def run_decode(args, hbm_gbs, l2_bytes, peak_kind):
     return {"value": value, "ms": ms, "bytes_step": bytes_step, "roofline": roof, "copies": copies,
             "graphs": graphs, "probs": probs,
             # the decode kernel, plus the act-quant kernel above 8 tokens
-            "launches_per_step": sum(2 if p.M > 8 else 1 for p in probs)}
+            "launches_per_step": sum(forward_launches(p.M, p.K) for p in probs)}
 
 
 def run_e2e(args, probs, steps):
@@ -540,7 +549,9 @@ def run_stack3b(hbm_gbs, M=1, layers=26, reps=20, int8_tops=None):
 
     out = {"workload": f"3B-class projection stack, {layers} layers, M={M}", "layers": layers, "M": M}
     wbytes = layers * (3 * H * H + H * H + 2 * F * H + H * F) // 4
-    for name, fn, launches in (("grouped", grouped, 4), ("separate", separate, 7)):
+    # per layer: grouped q/k/v, o, grouped gate/up, down; or the 7 projections
+    ks = {"grouped": (H, H, H, F), "separate": (H, H, H, H, H, H, F)}
+    for name, fn in (("grouped", grouped), ("separate", separate)):
         fn()
         torch.cuda.synchronize()
         g = torch.cuda.CUDAGraph()
@@ -559,7 +570,7 @@ def run_stack3b(hbm_gbs, M=1, layers=26, reps=20, int8_tops=None):
         out[name] = {"us_per_pass": round(us, 1), "tokens_per_s": round(M / (us * 1e-6), 1),
                      "weights_gbs": round(wbytes / (us * 1e-6) / 1e9, 1),
                      "frac_of_hbm": round(wbytes / (us * 1e-6) / 1e9 / hbm_gbs, 4),
-                     "launches_per_pass": launches * layers * (2 if M > 16 else 1)}   # act quant + GEMM
+                     "launches_per_pass": layers * sum(forward_launches(M, k) for k in ks[name])}
         if M > 16 and int8_tops:
             ops = 2 * M * layers * (3 * H * H + H * H + 2 * F * H + H * F)
             tops = ops / (us * 1e-6) / 1e12
@@ -649,7 +660,7 @@ def run_ffn100b(hbm_gbs, int8_tops, Ms=(1, 8, 64, 512), layers=13, reps=10):
         us = e0.elapsed_time(e1) * 1e3 / reps
         ops = layers * 3 * 2 * M * F * H
         row = {"M": M, "us_per_pass": round(us, 1), "tokens_per_s": round(M / (us * 1e-6), 1),
-               "launches_per_pass": 3 * layers * (2 if M > 16 else 1)}
+               "launches_per_pass": layers * (2 * forward_launches(M, H) + forward_launches(M, F))}
         if M <= 16:
             gbs = wbytes / (us * 1e-6) / 1e9
             row.update({"bound": "hbm", "weights_gbs": round(gbs, 1), "frac": round(gbs / hbm_gbs, 4)})
