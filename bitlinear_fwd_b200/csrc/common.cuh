@@ -234,6 +234,18 @@ __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// Per-thread register budget of a warpgroup (4 aligned warps, all of whose
+// threads execute it): lowered so that another warpgroup can raise its own
+// from the registers the block was launched with.
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // Shared-memory matrix descriptor for a K-major operand tile stored as
 // rows of 128 bytes with the 128-byte swizzle (16-byte chunk c of row r at
 // chunk position c ^ (r % 8)), 8-row groups 1024 bytes apart.

@@ -28,11 +28,14 @@
 //                (stage & 1), into accumulator buffer (tile & 1); commits free
 //                the shared stage and the A stage
 //   warp 2       tensor-memory allocation
-//   warps 4..7   weight unpack: thread = weight row; its 64 packed bytes become
-//                64 registers of codes c = u + 1 (one word -> four registers
-//                of four consecutive k) and two tcgen05.st of 32 columns; the
-//                swizzled rows keep a quarter-warp's reads in distinct banks
-//   warps 8..15  epilogue of the previous tile while the MMAs of the next one
+//   warps 4..11  weight unpack, two warps per tensor-memory lane quarter, one
+//                per 128-k half of a stage: thread = weight row; its 32
+//                packed bytes of the half become 32 registers of codes c =
+//                u + 1 (one word -> four registers of four consecutive k)
+//                and one tcgen05.st of 32 columns; the swizzled rows keep a
+//                quarter-warp's reads in distinct banks.  (One warp per
+//                quarter took longer per stage than the stage's MMAs.)
+//   warps 12..19 epilogue of the previous tile while the MMAs of the next one
 //                run; warps w and w + 4 share a lane quarter of tensor memory
 //                and take one half of the tile's tokens each: tcgen05.ld of a
 //                row's 96 accumulators (the next 32 columns load while 32 are
@@ -42,6 +45,9 @@
 //                stores with TMA (plain stores when y's rows are not 16-byte
 //                multiples or a debug output is asked for); s_w is the scale
 //                of the row's group (stacked layers)
+// Registers: 20 warps launch at 96 per thread; then the warpgroups set
+// their own budgets (setmaxnreg): 56 for warps 0..3, 72 for the unpack
+// warps, 136 for the epilogue.
 // Barriers: per shared stage full (TMA bytes landed) and empty (MMAs done);
 // per A stage ready (written) and afree (MMAs done); per accumulator buffer
 // acc_full (tile's MMAs done) and acc_empty (epilogue has read it).
@@ -65,7 +71,16 @@ constexpr int BT = BITLINEAR_GEMM_BT;        // tokens per tile (MMA N)
 constexpr int BK = 256;                      // k per block (stage)
 constexpr int STAGES = 3;                    // shared-memory operand stages
 constexpr int ASTAGES = 2;                   // tensor-memory stages of unpacked weights
-constexpr int kThreads = 512;
+constexpr int kThreads = 640;                // 20 warps: see the roles above
+// Register budgets per warpgroup after the set-up (setmaxnreg): the TMA,
+// MMA and allocation warps need few, the unpack warps hold 32 codes, the
+// epilogue warps two 32-column accumulator chunks.  Launched at 96 per
+// thread (640 x 96 = 61440 of the SM's 65536); the budgets below sum to
+// 32 x (4 x 56 + 8 x 72 + 8 x 136) = 60416, within the launch's share, so
+// the raise never waits on registers that no warpgroup gives back.
+constexpr uint32_t kRegsRoles = 56, kRegsUnpack = 72, kRegsEpi = 136;
+static_assert(4 * kRegsRoles + 8 * kRegsUnpack + 8 * kRegsEpi <= kThreads / 32 * 96,
+              "the warpgroups' register budgets fit the launch's");
 constexpr int kEpiWarps = 8;                 // two per tensor-memory lane quarter
 constexpr int kEpiCols = BT / 2;             // tokens of a tile per epilogue warp
 constexpr int kEpiChunks = kEpiCols / 32;
@@ -129,7 +144,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&empty[s], 1);
     }
     for (int s = 0; s < ASTAGES; ++s) {
-      mbar_init(&ready[s], 4);
+      mbar_init(&ready[s], 8);                     // the eight unpack warps
       mbar_init(&afree[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -155,7 +170,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   const uint32_t tmem_a = tmem_base + 2 * BT;     // A stages after the two accumulators
 
-  if (warp == 0) {
+  // Each warpgroup sets its register budget at the head of its role (every
+  // thread of the warpgroup, converged after the barrier above).
+  if (warp < 4) {
+   setmaxnreg_dec<kRegsRoles>();
+   if (warp == 0) {
     if (lane == 0) {
       // ---------------- TMA producer ----------------
       int g = 0;                                  // k-blocks issued by this CTA
@@ -238,9 +257,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         *drain_bad = 1;
       }
     }
-  } else if (warp >= 4 && warp < 8) {
+   }
+  } else if (warp < 12) {
+    setmaxnreg_dec<kRegsUnpack>();
     // ---------------- weight unpack into tensor memory ----------------
+    // Two warps per tensor-memory lane quarter, one per 128-k half of a
+    // stage (a single warp's chain of loads, unpacking, store and arrive
+    // took longer than the stage's MMAs).
     const int q = warp & 3;
+    const int hh = (warp - 4) >> 2;               // the half of each stage this warp unpacks
     const int row = 32 * q + lane;
     const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
     // The weight rows are 64 bytes with TMA's 64-byte swizzle: 16-byte piece
@@ -257,15 +282,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           *failed = 1;
           break;
         }
-        const uint4* wp = reinterpret_cast<const uint4*>(smem + kOffWp + s * kWpBytes + row * 64);
-        uint4 pc[4];
-#pragma unroll
-        for (int p = 0; p < 4; ++p) pc[p] = wp[p ^ sw];
-        tc_fence_after();
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {             // k 128h .. 128h + 127: 32 columns
-          const uint32_t w[8] = {pc[2 * h].x, pc[2 * h].y, pc[2 * h].z, pc[2 * h].w,
-                                 pc[2 * h + 1].x, pc[2 * h + 1].y, pc[2 * h + 1].z, pc[2 * h + 1].w};
+        // a second half beyond K gets no MMA: nothing to write, but its
+        // warp still arrives
+        if (hh == 0 || kb * BK + 128 < a.K) {
+          const uint4* wp = reinterpret_cast<const uint4*>(smem + kOffWp + s * kWpBytes + row * 64);
+          const uint4 p0 = wp[(2 * hh) ^ sw], p1 = wp[(2 * hh + 1) ^ sw];
+          tc_fence_after();
+          const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
           uint32_t codes[32];
 #pragma unroll
           for (int jj = 0; jj < 8; ++jj) {        // word jj = k 16jj .. 16jj + 15 of the half
@@ -274,19 +297,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             codes[4 * jj + 2] = (w[jj] >> 4) & kCodeMask;
             codes[4 * jj + 3] = (w[jj] >> 6) & kCodeMask;
           }
-          tmem_st_32x32b_x32(tmem_a + lane_base + as * kACols + 32 * h, codes);
+          tmem_st_32x32b_x32(tmem_a + lane_base + as * kACols + 32 * hh, codes);
+          tmem_wait_st();
         }
-        tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&ready[as]);
       }
     }
-  } else if (warp >= 8) {
+  } else {
+    setmaxnreg_inc<kRegsEpi>();
     // ---------------- epilogue ----------------
     const int q = warp & 3;
-    const int et = threadIdx.x - 256;             // 0..255
-    const int half = (warp - 8) >> 2;             // which half of the tile's tokens
+    const int et = threadIdx.x - 384;             // 0..255
+    const int half = (warp - 12) >> 2;            // which half of the tile's tokens
     const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
     pdl_wait_primary();
     float swg[kMaxGroups];                         // s_w of each row group
