@@ -83,11 +83,10 @@ def peaks():
 
 def forward_launches(M, K):
     """Kernels one bitlinear_forward launches: the act-quant kernel and the
-    GEMM above 16 tokens; the decode kernel alone up to 8 tokens (and up to
-    K = 8192 from 2 tokens), else the act-quant kernel before it."""
-    if M > 16:
-        return 2
-    return 2 if (M > 8 or (M >= 2 and K > 8192)) else 1
+    GEMM above 16 tokens; the decode kernel alone up to 8 tokens, the
+    act-quant kernel before it above 8 (K does not change the count)."""
+    del K
+    return 2 if M > 8 else 1
 
 
 def decode_bytes(M, N, K, bias=True):

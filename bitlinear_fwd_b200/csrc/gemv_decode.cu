@@ -214,7 +214,7 @@ struct SmemTail {
   uint32_t amax[16];                 // absmax per token (bf16 bits)
   int rsum[16];                      // sum of q per token
   float sx[16];                      // s_x per token
-  float swg[kMaxGroups];             // s_w of each row group
+  double rcp[kMaxGroups * 16];       // 1 / (s_x s_w) per row group and token, [group][token]
   int failed;                        // a wait of this CTA timed out
 };
 
@@ -378,6 +378,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
   // (with the weights when those are resident) and stored to shared memory
   // only before the epilogue, so no thread waits for them on the way to x
   uint16_t bvals[2] = {0, 0};
+  // thread g M + m (< M x groups) forms 1 / (s_x s_w) of token m and row group g
   float swv = 0.0f;
   auto load_params = [&]() {
 #pragma unroll
@@ -386,7 +387,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
       const int n = u_begin * kUnitRows + i;
       if (i < U * kUnitRows && a.bias && n < N) bvals[k] = a.bias[n];
     }
-    if (threadIdx.x < a.ngroups) swv = a.w_scale[threadIdx.x];
+    if (threadIdx.x < M * a.ngroups) swv = a.w_scale[threadIdx.x / M];
   };
   if (a.weights_early) {
     for (int i = 0; i < ring; ++i) issue_next();
@@ -444,18 +445,22 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
     // warp w takes token m = w / P; a lane holds C <= kHold chunks of it
     const int m = warp / P;
     const bool mine = m < M;
+    // (the loops leave at i = C, the same for every thread, so the unrolled
+    // iterations beyond it cost one branch rather than being predicated off)
     uint4 v[kHold][2];
 #pragma unroll
-    for (int i = 0; i < kHold; ++i)
-      if (i < C) {
-        const bool in = mine && ch_first + i * 32 * P < cpr;
-        v[i][0] = in ? __ldg(xl[0] + i * xstep) : make_uint4(0, 0, 0, 0);
-        v[i][1] = in ? __ldg(xl[0] + i * xstep + 1) : make_uint4(0, 0, 0, 0);
-      }
+    for (int i = 0; i < kHold; ++i) {
+      if (i >= C) break;
+      const bool in = mine && ch_first + i * 32 * P < cpr;
+      v[i][0] = in ? __ldg(xl[0] + i * xstep) : make_uint4(0, 0, 0, 0);
+      v[i][1] = in ? __ldg(xl[0] + i * xstep + 1) : make_uint4(0, 0, 0, 0);
+    }
     uint32_t mx = 0;
 #pragma unroll
-    for (int i = 0; i < kHold; ++i)
-      if (i < C) mx = max(mx, absmax16_bits(v[i][0], v[i][1]));   // zeros where nothing was loaded
+    for (int i = 0; i < kHold; ++i) {
+      if (i >= C) break;
+      mx = max(mx, absmax16_bits(v[i][0], v[i][1]));   // zeros where nothing was loaded
+    }
     mx = __reduce_max_sync(0xffffffffu, mx);
     if (lane == 0 && mine) atomicMax(&sm.amax[m], mx);
     __syncthreads();
@@ -470,7 +475,8 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
 #pragma unroll
     for (int i = 0; i < kHold; ++i) {
       const int ch = ch_first + i * 32 * P;
-      if (i < C && mine && ch < cpr) {
+      if (i >= C) break;
+      if (mine && ch < cpr) {
         const uint4 qv = quant16(v[i][0], v[i][1], sxm, sum, FAITHFUL);
         *reinterpret_cast<uint4*>(xs + m * S + 16 * xs_chunk(ch)) = qv;
         if (blockIdx.x == 0 && a.xq_out) *reinterpret_cast<uint4*>(a.xq_out + static_cast<size_t>(m) * K + 16 * ch) = qv;
@@ -484,9 +490,14 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
       uint32_t mx = 0;
       // kXB 32-byte loads in flight per lane before any is used
       for (int ch0 = part * 32 + lane; ch0 < cpr; ch0 += 32 * P * kXB) {
+        // loads of this pass that start inside the row for the warp's first
+        // lane (the same for every thread of the warp: the loops leave early
+        // instead of running predicated-off iterations)
+        const int nj = min(kXB, (cpr - (ch0 - lane) + 32 * P - 1) / (32 * P));
         uint4 v[kXB][2];
 #pragma unroll
         for (int j = 0; j < kXB; ++j) {
+          if (j >= nj) break;
           const int chu = ch0 + j * 32 * P;
           v[j][0] = v[j][1] = make_uint4(0, 0, 0, 0);
           if (chu < cpr) {
@@ -495,7 +506,10 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
           }
         }
 #pragma unroll
-        for (int j = 0; j < kXB; ++j) mx = max(mx, absmax16_bits(v[j][0], v[j][1]));
+        for (int j = 0; j < kXB; ++j) {
+          if (j >= nj) break;
+          mx = max(mx, absmax16_bits(v[j][0], v[j][1]));
+        }
       }
       mx = __reduce_max_sync(0xffffffffu, mx);
       if (lane == 0) atomicMax(&sm.amax[m], mx);
@@ -719,7 +733,17 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
     const int i = threadIdx.x + k * kThreads;
     if (i < U * kUnitRows) bias_s[i] = bvals[k];
   }
-  if (threadIdx.x < a.ngroups) sm.swg[threadIdx.x] = swv;
+  if (threadIdx.x < M * a.ngroups) {
+    // d = s_x s_w of the token and the group (on a bf16 module bf16(bf16(s_w)
+    // s_x)), kept as the double 1 / d: RN_f32(a * (1/d)) is RN_f32(a / d) for
+    // every float32 (or bf16) numerator a -- a quotient of two floats lies at
+    // least 2^-49 (relative) from every float32 midpoint, and the double
+    // product is within 2^-52 of it.  s_x of token m is in shared memory
+    // since the x phase (for one token, written by this warp).
+    const float sx = sm.sx[threadIdx.x % M];
+    const float d = FAITHFUL ? bf16_round(__fmul_rn(bf16_round(swv), sx)) : __fmul_rn(sx, swv);
+    sm.rcp[threadIdx.x] = __drcp_rn(static_cast<double>(d));
+  }
   // every copy this thread issued has landed before the CTA exits
   cp_async_wait(0);
   if (!ok) {
@@ -729,22 +753,26 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
   __syncthreads();                                   // s_w, the bias and the sums are in shared memory
 
   // ---------------- epilogue: U units x 16 rows x M tokens ----------------
+  // output idx = m rows + rl: thread t starts at idx = t and steps by
+  // kThreads = dm rows + drl (no division per output)
   const int rows = U * kUnitRows;
-  for (int idx = threadIdx.x; idx < rows * M; idx += kThreads) {
-    const int m = idx / rows, rl = idx - m * rows;
+  const int dm = kThreads / rows, drl = kThreads - dm * rows;
+  int m = static_cast<int>(threadIdx.x) / rows, rl = static_cast<int>(threadIdx.x) - m * rows;
+  for (; m < M; m += dm, rl += drl) {
+    if (rl >= rows) {
+      rl -= rows;
+      ++m;
+      if (m >= M) break;
+    }
     const int n = u_begin * kUnitRows + rl;
     if (n >= N) continue;
     const int accv = acc_s[(rl >> 4) * kUnitRows * NTOK + sum_idx<NTOK>(rl & 15, m)] - sm.rsum[m];
-    int gi = 0;                                      // the row's group (scale)
+    int gi = 0;                                      // the row's group (scale), when layers are stacked
+    if (a.ngroups > 1) {
 #pragma unroll
-    for (int gg = 0; gg + 1 < kMaxGroups; ++gg) gi += (gg + 1 < a.ngroups && n >= a.group_end[gg]) ? 1 : 0;
-    // d = s_x s_w of the token and the row's group (on a bf16 module
-    // bf16(bf16(s_w) s_x)), used as the double 1 / d: RN_f32(a * (1/d)) is
-    // RN_f32(a / d) for every float32 (or bf16) numerator a -- a quotient of
-    // two floats lies at least 2^-49 (relative) from every float32 midpoint,
-    // and the double product is within 2^-52 of it
-    const float d = FAITHFUL ? bf16_round(__fmul_rn(bf16_round(sm.swg[gi]), sm.sx[m])) : __fmul_rn(sm.sx[m], sm.swg[gi]);
-    const double r = __drcp_rn(static_cast<double>(d));
+      for (int gg = 0; gg + 1 < kMaxGroups; ++gg) gi += (gg + 1 < a.ngroups && n >= a.group_end[gg]) ? 1 : 0;
+    }
+    const double r = sm.rcp[gi * M + m];
     float y32;
     if (!FAITHFUL) {
       y32 = __double2float_rn(static_cast<double>(static_cast<float>(accv)) * r);
