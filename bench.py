@@ -85,10 +85,9 @@ def peaks():
 
 def forward_launches(M, K):
     """Kernels one bitlinear_forward launches: the act-quant kernel and the
-    GEMM above 16 tokens; the decode kernel alone up to 8 tokens, the
-    act-quant kernel before it above 8 (K does not change the count)."""
-    del K
-    return 2 if M > 8 else 1
+    GEMM above 16 tokens; the decode kernel alone up to 8 tokens (at 8
+    tokens only up to K = 8192), else the act-quant kernel before it."""
+    return 2 if (M > 8 or (M == 8 and K > 8192)) else 1
 
 
 def decode_bytes(M, N, K, bias=True):

@@ -126,12 +126,13 @@ int forward_impl_g(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packe
   int32_t* rowsum = reinterpret_cast<int32_t*>(base + L.off_rs);
   int8_t* xq = reinterpret_cast<int8_t*>(base + L.off_xq);
   if (decode) {
-    // Above 8 tokens the activations are quantised once by the act-quant
-    // kernel, and the GEMV reads int8 x: every CTA of the GEMV needs all of
-    // x, and quantising it 148 times over costs more than the extra launch.
-    // (At 2-8 tokens and K = 28672 the act-quant kernel, one CTA per token,
-    // took longer than the GEMV's own re-reads of bf16 x.)
-    const bool pre = M > 8;
+    // Above 8 tokens, and at 8 tokens when K spans more than two 4096-k
+    // rounds, the activations are quantised once by the act-quant kernel and
+    // the GEMV reads int8 x: every CTA of the GEMV needs all of x, and
+    // quantising it 148 times over (re-reading bf16 x per round) costs more
+    // than the extra launch.  At 2-4 tokens and K = 28672 the act-quant
+    // kernel (one CTA per token) took longer than the re-reads.
+    const bool pre = M > 8 || (M == 8 && K > 8192);
     if (pre) {
       e = launch_act_quant(x, int(M), int(K), xq, s_x, rowsum, status, resident, stream, faithful);
       if (e != cudaSuccess) return BITLINEAR_ERR_CUDA;
