@@ -999,6 +999,14 @@ def run_case(name):
         for M in (1, 4, 16):
             bl.bitlinear_forward(synth.normal_bf16(1, 2 + M, (M, K), device=dev), packed, s_w, b,
                                  flags=bl.WEIGHTS_RESIDENT)
+    elif name == "decodewide":
+        # the 100B-class gate projection (28672 x 8192) at M = 1: the
+        # weight stream, two CTAs per SM
+        K, N = 8192, 28672
+        packed, s_w, _ = bl.bitlinear_pack_weights(synth.normal_f32(1, 1, (N, K), 0.02, device=dev))
+        x = synth.normal_bf16(1, 2, (1, K), device=dev)
+        for _ in range(3):
+            bl.bitlinear_forward(x, packed, s_w, flags=bl.WEIGHTS_RESIDENT)
     elif name == "actq":
         x = synth.normal_bf16(1, 2, (8192, 8640), device=dev)
         for _ in range(2):
@@ -1037,7 +1045,8 @@ def main():
     ap.add_argument("--only", choices=["decode", "prefill", "dequant", "stack3b"], default=None,
                     help="run one workload only (profiling runs; no JSON contract line)")
     ap.add_argument("--copies", type=int, default=0, help="force the number of rotating weight copies")
-    ap.add_argument("--case", choices=["decode", "gemm", "gemm8640", "actq", "pack", "dequant", "ksplit"],
+    ap.add_argument("--case", choices=["decode", "decodewide", "gemm", "gemm8640", "actq", "pack", "dequant",
+                                       "ksplit"],
                     default=None, help="run one small case of one kernel for an ncu capture, then exit")
     args = ap.parse_args()
     if args.case:

@@ -105,6 +105,26 @@ __device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, 
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// the same with a zero accumulator in (the first MMA of a chain): no
+// register has to be cleared for it
+__device__ __forceinline__ void mma_u8s8_first(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 "
+      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%10, %10, %10, %10};"
+      : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(0));
+}
+
+// floor(a / 2^(32 - sh)) + c on the multiply-add pipe (mad.hi: the high word
+// of the 64-bit product a 2^sh, plus c); the field sums are multiples of the
+// divisor, so this is their exact shift
+__device__ __forceinline__ int mad_hi(int a, int b, int c) {
+  int d;
+  asm("mad.hi.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
 // 16-byte asynchronous copy global -> shared (L2 only); src_bytes = 0 writes
 // zeros and reads nothing
 __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc, uint32_t src_bytes) {
@@ -361,14 +381,25 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
       const bool kin = static_cast<uint32_t>(c) * (kBoxK / 4) + 16u * pq < row_bytes;
       const uint8_t* src = a.packed + static_cast<size_t>(u_begin * kUnitRows + r0g) * row_bytes +
                            static_cast<uint32_t>(c) * (kBoxK / 4) + psrc;
+      // an item wholly inside N and K (every item but a CTA's last group and
+      // the chunk at K's end; the same for the whole warp) needs no checks
+      if (lim >= UP * kUnitRows && static_cast<uint32_t>(c + 1) * (kBoxK / 4) <= row_bytes) {
 #pragma unroll
-      for (int e = 0; e < UP; ++e)
+        for (int e = 0; e < UP; ++e)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const bool valid = kin && kUnitRows * e + prow + 4 * j < lim;
-          cp_async16(dst + e * kSubBytes + ((j & 1) ? pdst1 : pdst0) + (j >> 1) * 1024,
-                     valid ? src + static_cast<size_t>(kUnitRows * e + 4 * j) * row_bytes : a.packed, valid ? 16u : 0u);
-        }
+          for (int j = 0; j < 4; ++j)
+            cp_async16(dst + e * kSubBytes + ((j & 1) ? pdst1 : pdst0) + (j >> 1) * 1024,
+                       src + static_cast<size_t>(kUnitRows * e + 4 * j) * row_bytes, 16u);
+      } else {
+#pragma unroll
+        for (int e = 0; e < UP; ++e)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const bool valid = kin && kUnitRows * e + prow + 4 * j < lim;
+            cp_async16(dst + e * kSubBytes + ((j & 1) ? pdst1 : pdst0) + (j >> 1) * 1024,
+                       valid ? src + static_cast<size_t>(kUnitRows * e + 4 * j) * row_bytes : a.packed, valid ? 16u : 0u);
+          }
+      }
       islot = islot + 1 == ring ? 0 : islot + 1;
       ic.next(warp, nround, nchunks, PU);
     }
@@ -672,12 +703,6 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
       for (int e = 0; e < UP; ++e) {
         int acc[4][NT][4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int rr = 0; rr < 4; ++rr) acc[i][nt][rr] = 0;
-#pragma unroll
         for (int v = 0; v < 2; ++v) {
           const int cw = 4 * v + t;                  // 16-byte chunk of the 128-byte row
           const uint4 wa = *reinterpret_cast<const uint4*>(box + e * kSubBytes + r0 * 128 + ((cw ^ r0) << 4));
@@ -692,15 +717,20 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
               const uint32_t a0 = w0[2 * pr] & mask, a1 = w1[2 * pr] & mask;
               const uint32_t a2 = w0[2 * pr + 1] & mask, a3 = w1[2 * pr + 1] & mask;
 #pragma unroll
-              for (int nt = 0; nt < NT; ++nt)
-                mma_u8s8(acc[i][nt], a0, a1, a2, a3, xw[v][pr][nt][i], xw[v][pr][nt][4 + i]);
+              for (int nt = 0; nt < NT; ++nt) {
+                if (v == 0 && pr == 0)
+                  mma_u8s8_first(acc[i][nt], a0, a1, a2, a3, xw[v][pr][nt][i], xw[v][pr][nt][4 + i]);
+                else
+                  mma_u8s8(acc[i][nt], a0, a1, a2, a3, xw[v][pr][nt][i], xw[v][pr][nt][4 + i]);
+              }
             }
         }
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
           for (int rr = 0; rr < 4; ++rr)
-            cv[e][nt][rr] = acc[0][nt][rr] + (acc[1][nt][rr] >> 2) + (acc[2][nt][rr] >> 4) + (acc[3][nt][rr] >> 6);
+            cv[e][nt][rr] = mad_hi(acc[3][nt][rr], 1 << 26,
+                                   mad_hi(acc[2][nt][rr], 1 << 28, mad_hi(acc[1][nt][rr], 1 << 30, acc[0][nt][rr])));
       }
       // the slot is read: refill it with this warp's next item
       __syncwarp();
