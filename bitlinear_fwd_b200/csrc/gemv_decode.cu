@@ -581,7 +581,9 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
   const uint8_t* xtok = g < M ? reinterpret_cast<const uint8_t*>(xs) + g * S + 64 * t
                               : reinterpret_cast<const uint8_t*>(sm.zero);
   const int xpo[2] = {32 * (t >> 1), 32 * (1 ^ (t >> 1))};
-  uint32_t xw[2][2][NT][8];                          // [v][pair][token tile][word]
+  // [v][pair][token tile][field]: the two B words of the field's MMA (x
+  // words i and 4 + i) side by side, as the MMA takes them
+  uint2 xw[2][2][NT][4];
   for (int r = 0; r < nround; ++r) {
     const int c0 = r * kChunkK;
     const int ccpr = min(kChunkK, K - c0) >> 4;      // 16-element chunks of x in this round
@@ -671,8 +673,13 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
                   const int mr = xin ? m : 0, xr = xin ? xc : 0;
                   uint4 xv = __ldg(reinterpret_cast<const uint4*>(a.xq + static_cast<size_t>(mr) * K + r * kChunkK) + xr);
                   if (!xin) xv = make_uint4(0, 0, 0, 0);
-                  xw[v][pr][nt][4 * c2 + 0] = xv.x; xw[v][pr][nt][4 * c2 + 1] = xv.y;
-                  xw[v][pr][nt][4 * c2 + 2] = xv.z; xw[v][pr][nt][4 * c2 + 3] = xv.w;
+                  if (c2 == 0) {
+                    xw[v][pr][nt][0].x = xv.x; xw[v][pr][nt][1].x = xv.y;
+                    xw[v][pr][nt][2].x = xv.z; xw[v][pr][nt][3].x = xv.w;
+                  } else {
+                    xw[v][pr][nt][0].y = xv.x; xw[v][pr][nt][1].y = xv.y;
+                    xw[v][pr][nt][2].y = xv.z; xw[v][pr][nt][3].y = xv.w;
+                  }
                 }
               }
         } else {
@@ -688,8 +695,13 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
 #pragma unroll
               for (int c2 = 0; c2 < 2; ++c2) {
                 const uint4 xv = *reinterpret_cast<const uint4*>(xb + xpo[pr] + 256 * v + 16 * c2);
-                xw[v][pr][0][4 * c2 + 0] = xv.x; xw[v][pr][0][4 * c2 + 1] = xv.y;
-                xw[v][pr][0][4 * c2 + 2] = xv.z; xw[v][pr][0][4 * c2 + 3] = xv.w;
+                if (c2 == 0) {
+                  xw[v][pr][0][0].x = xv.x; xw[v][pr][0][1].x = xv.y;
+                  xw[v][pr][0][2].x = xv.z; xw[v][pr][0][3].x = xv.w;
+                } else {
+                  xw[v][pr][0][0].y = xv.x; xw[v][pr][0][1].y = xv.y;
+                  xw[v][pr][0][2].y = xv.z; xw[v][pr][0][3].y = xv.w;
+                }
               }
         }
         xchunk = lc;
@@ -719,9 +731,9 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
 #pragma unroll
               for (int nt = 0; nt < NT; ++nt) {
                 if (v == 0 && pr == 0)
-                  mma_u8s8_first(acc[i][nt], a0, a1, a2, a3, xw[v][pr][nt][i], xw[v][pr][nt][4 + i]);
+                  mma_u8s8_first(acc[i][nt], a0, a1, a2, a3, xw[v][pr][nt][i].x, xw[v][pr][nt][i].y);
                 else
-                  mma_u8s8(acc[i][nt], a0, a1, a2, a3, xw[v][pr][nt][i], xw[v][pr][nt][4 + i]);
+                  mma_u8s8(acc[i][nt], a0, a1, a2, a3, xw[v][pr][nt][i].x, xw[v][pr][nt][i].y);
               }
             }
         }
