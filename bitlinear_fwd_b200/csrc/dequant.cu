@@ -10,6 +10,14 @@
 // packed word (16 weights, k = 16g + 4i + j at bits 8j + 2i) into 32 output
 // bytes, written as two 16-byte stores; a packed row of K/16 words becomes the
 // K bf16 values of the same row, so word w maps to output bytes [32w, 32w+32).
+// Each output word (two bf16 values, k and k + 1 = bytes j and j + 1 of
+// field i) is one byte permutation of the eight bytes {bf16(+v), 0, 0,
+// bf16(-v), 0, 0}: a code c selects bytes 4 - 2c and 5 - 2c (2 -> +v, 1 -> 0,
+// 0 -> -v), so the selector of a pair of codes (c0, c1) is 0x5454 - (c0 +
+// 256 c1) 0x22, and (word >> 2i) & 0x03030303 holds c0 + 256 c1 for both
+// pairs of field i.  Four instructions per output word instead of a compare
+// and select per value (the loop was issue-bound).  A word holding the
+// invalid code 3 exports unspecified values.
 #include "kernels.h"
 
 namespace bitlinear {
@@ -18,21 +26,18 @@ namespace {
 
 __global__ void __launch_bounds__(256) dequant_kernel(const uint32_t* __restrict__ packed, size_t words,
                                                       const float* __restrict__ w_scale, uint4* __restrict__ out) {
+  // bytes 0-1: bf16(+v), 2-3: zero; bytes 4-5: bf16(-v), 6-7: zero
   const uint32_t pos = f32_to_bf16_bits(__fdiv_rn(1.0f, *w_scale));
   const uint32_t neg = pos ^ 0x8000u;
-  // bf16 bits of u for the codes 0, 1, 2 (u = -1, 0, 1); code 3 never occurs
-  // in packed weights and exports as 0
   for (size_t idx = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; idx < words;
        idx += static_cast<size_t>(gridDim.x) * blockDim.x) {
     const uint32_t wd = __ldg(packed + idx);
     uint32_t o[8];
 #pragma unroll
-    for (int e = 0; e < 16; e += 2) {              // output element e = 4i + j
-      const uint32_t c0 = (wd >> (8 * (e & 3) + 2 * (e >> 2))) & 3u;
-      const uint32_t c1 = (wd >> (8 * ((e + 1) & 3) + 2 * ((e + 1) >> 2))) & 3u;
-      const uint32_t b0 = c0 == 2u ? pos : (c0 == 0u ? neg : 0u);
-      const uint32_t b1 = c1 == 2u ? pos : (c1 == 0u ? neg : 0u);
-      o[e >> 1] = b0 | (b1 << 16);
+    for (int i = 0; i < 4; ++i) {                  // output words 2i (k = 4i, 4i+1) and 2i + 1 (k = 4i+2, 4i+3)
+      const uint32_t u = (wd >> (2 * i)) & 0x03030303u;
+      o[2 * i] = __byte_perm(pos, neg, 0x5454u - u * 0x22u);           // the selector uses the low 16 bits
+      o[2 * i + 1] = __byte_perm(pos, neg, 0x5454u - (u >> 16) * 0x22u);
     }
     out[2 * idx] = make_uint4(o[0], o[1], o[2], o[3]);
     out[2 * idx + 1] = make_uint4(o[4], o[5], o[6], o[7]);
