@@ -713,6 +713,9 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
       const uint8_t* box = wring + s * kSlotBytes;
 #pragma unroll
       for (int e = 0; e < UP; ++e) {
+        // the missing unit of a CTA's last group (odd unit count) is all
+        // zeros: no MMAs for it (the same for the whole warp)
+        if (UP > 1 && e > 0 && UP * ug + e >= U) break;
         int acc[4][NT][4];
 #pragma unroll
         for (int v = 0; v < 2; ++v) {
