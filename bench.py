@@ -19,9 +19,12 @@ Also on the line:
                 the tcgen05 GEMM's own roofline against the int8 peak
   e2e           the decode metric with host buffers: the step's six bf16
                 inputs copied in from one pinned buffer and its outputs back
-                to one, the six calls between, one sync per step; beside it
-                (per_call_host_api) bitlinear_forward_host_async copying every
-                call's input in and output out
+                to a pinned buffer, the six calls between, double-buffered on
+                three streams so that neighbouring steps' copies run beside a
+                step's calls, one wait per step for its outputs on the host;
+                beside it the same steps run serially (e2e.serial) and
+                bitlinear_forward_host_async copying every call's input in
+                and output out (e2e.per_call_host_api)
   dequant_export, stack3b_decode
                 the bf16 export kernel's GB/s, and the 3B-class 26-layer
                 projection stack at M=1 with and without grouped calls
@@ -376,13 +379,17 @@ def run_decode(args, hbm_gbs, l2_bytes, peak_kind):
 
 
 def run_e2e(args, probs, steps):
-    """The headline metric end to end with host buffers, two ways.
+    """The headline metric end to end with host buffers, three ways.
 
-    Step-batched (the reported value): the step's six inputs sit in one
-    pinned host buffer and are copied to the device in one copy, the six
-    bitlinear_forward calls run on device views of it, and the six outputs
-    come back in one copy to one pinned buffer; the step is captured as a
-    CUDA graph and each step is one graph launch plus one synchronisation.
+    Step-batched: the step's six inputs sit in one pinned host buffer and
+    are copied to the device in one copy, the six bitlinear_forward calls
+    run on device views of it, and the six outputs come back in one copy to
+    a pinned buffer.  Pipelined (the reported value), the same copies and
+    calls double-buffered on three streams, so that the copies of the
+    neighbouring steps run beside a step's calls, with one wait per step for
+    that step's outputs in host memory; serial (reported beside it), copy
+    in, calls and copy out one after the other, one graph launch and one
+    synchronisation per step.
 
     Per call (reported beside it): every bitlinear_forward_host_async call
     copies its own bf16 x in and its bf16 y out (12 copies, 6 kernels per
@@ -480,15 +487,100 @@ def run_e2e(args, probs, steps):
     torch.cuda.synchronize()
     ok = bool(torch.equal(yh, yd.cpu()))
     del bgraphs
+
+    # pipelined (the reported value): the same copies and calls, with two
+    # device input and output buffers and two pinned output buffers, on three
+    # streams -- step i+1's input copy and step i-1's output copy run beside
+    # step i's six calls; the host waits for step i-1's outputs to land in
+    # host memory before it issues step i+1
+    s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    xd2 = [xd, torch.empty_like(xd)]
+    yd2 = [yd, torch.empty_like(yd)]
+    yh2 = [yh, torch.empty_like(yh).pin_memory()]
+    xv2 = [[b[xo[i]:xo[i + 1]].view(p.M, p.K) for i, p in enumerate(probs)] for b in xd2]
+    yv2 = [[b[yo[i]:yo[i + 1]].view(p.M, p.N) for i, p in enumerate(probs)] for b in yd2]
+    dws2 = [dws, [bl.workspace(p.M, p.N, p.K, "cuda") for p in probs]]
+
+    def calls(b, r):
+        for p, x, y, ws in zip(probs, xv2[b], yv2[b], dws2[b]):
+            bl.bitlinear_forward(x, p.packed[r % copies], p.s_w, p.bias, ws=ws, out=y, flags=bl.WEIGHTS_RESIDENT)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        calls(1, 0)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    pgraphs = {}
+    for b in range(2):
+        for r in range(copies):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                calls(b, r)
+            pgraphs[(b, r)] = g
+
+    def pipelined(nsteps):
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_cmp = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
+        done = [None] * nsteps
+        cur = torch.cuda.current_stream()
+        for s in (s_in, s_cmp, s_out):
+            s.wait_stream(cur)
+
+        def issue(i):
+            b = i % 2
+            s_in.wait_event(ev_cmp[b])              # step i-2's calls have read xd[b]
+            with torch.cuda.stream(s_in):
+                xd2[b].copy_(xh, non_blocking=True)
+            ev_in[b].record(s_in)
+            s_cmp.wait_event(ev_in[b])
+            s_cmp.wait_event(ev_out[b])             # step i-2's outputs have left yd[b]
+            with torch.cuda.stream(s_cmp):
+                pgraphs[(b, i % copies)].replay()
+            ev_cmp[b].record(s_cmp)
+            s_out.wait_event(ev_cmp[b])
+            with torch.cuda.stream(s_out):
+                yh2[b].copy_(yd2[b], non_blocking=True)
+            ev_out[b].record(s_out)
+            done[i] = ev_out[b]
+
+        issue(0)
+        for i in range(nsteps):
+            if i + 1 < nsteps:
+                issue(i + 1)
+            done[i].synchronize()                   # step i's outputs are in host memory
+        cur.wait_stream(s_out)
+
+    pipelined(4)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    pipelined(steps)
+    e1.record()
+    e1.synchronize()
+    sync_all()
+    ms_p = elapsed_max_over_ranks(e0.elapsed_time(e1))
+    torch.cuda.synchronize()
+    last = (steps - 1) % 2
+    ok_p = bool(torch.equal(yh2[last], yd2[last].cpu())) and bool(torch.equal(yh2[last], yh))
+    del pgraphs
     world = world_size()
-    return {"value": round(whole_job_gbs(bytes_step, steps, ms_b, world), 2), "unit": "GB/s",
+    return {"value": round(whole_job_gbs(bytes_step, steps, ms_p, world), 2), "unit": "GB/s",
             "h2d_bytes_per_step": int(sum(2 * n for n in xsz)),
             "d2h_bytes_per_step": int(sum(2 * n for n in ysz)),
-            "us_per_step": round(ms_b * 1e3 / steps, 2),
+            "us_per_step": round(ms_p * 1e3 / steps, 2),
             "api": "per step: one copy of the six bf16 inputs from one pinned host buffer, six "
-                   "bitlinear_forward calls on device views, one copy of the six outputs to one pinned "
-                   "host buffer; captured once as a CUDA graph, one graph launch and one stream sync per step",
-            "outputs_match_device": ok,
+                   "bitlinear_forward calls on device views (one CUDA graph), one copy of the six outputs "
+                   "to a pinned host buffer; double-buffered on three streams (copy in, calls, copy out) "
+                   "so the copies of neighbouring steps run beside a step's calls; the host waits for "
+                   "each step's outputs in host memory (one event sync per step, at most one step ahead)",
+            "outputs_match_device": ok and ok_p,
+            "serial": {
+                "value": round(whole_job_gbs(bytes_step, steps, ms_b, world), 2), "unit": "GB/s",
+                "us_per_step": round(ms_b * 1e3 / steps, 2),
+                "api": "the same copies and calls, copy in, calls and copy out one after the other in one "
+                       "CUDA graph per step; one graph launch and one stream sync per step"},
             "per_call_host_api": {
                 "value": round(whole_job_gbs(bytes_step, steps, ms, world), 2), "unit": "GB/s",
                 "us_per_step": round(ms * 1e3 / steps, 2),
