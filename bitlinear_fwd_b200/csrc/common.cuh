@@ -101,7 +101,7 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 }
 
 // ---------------------------------------------------------------------------
-// TMA (no multicast)
+// TMA: tile loads into this CTA's own shared memory, L2 prefetch
 // ---------------------------------------------------------------------------
 // Brings a global line into L2 (not L1): safe on data the previous kernel of
 // the stream may still write, since L2 is the point of coherence.

@@ -250,7 +250,8 @@ int bitlinear_forward_host_async(const uint16_t* x_host, int64_t M, int64_t K, c
  * allocator, paths that must never allocate).  It takes no workspace: the
  * library uses one fixed device array of BITLINEAR_NOALLOC_SCRATCH_BYTES
  * bytes, held by every GPU that loads the library until the process exits.
- * The paper has no counterpart to this entry point.
+ * It is an interface convenience; the BitLinear definition it computes is
+ * the one bitlinear_forward follows.
  *   - Returns BITLINEAR_ERR_WORKSPACE when bitlinear_workspace_bytes(M, N, K)
  *     exceeds that fixed size (roughly M * K <= 16 MiB), and
  *     BITLINEAR_ERR_SHAPE for an invalid shape; other arguments and errors
@@ -274,8 +275,8 @@ int bitlinear_forward_noalloc(const uint16_t* x, int64_t M, int64_t K, const uin
  * bitlinear_forward_noalloc on the current device: reads and clears its
  * status word (synchronises `stream`).  Returns BITLINEAR_OK, or
  * BITLINEAR_ERR_TIMEOUT if a device-side bounded wait of a noalloc call gave
- * up since the last reset (each noalloc call resets it when it starts).  The
- * paper has no counterpart to this entry point either. */
+ * up since the last reset (each noalloc call resets it when it starts).  It
+ * is an interface convenience, like bitlinear_forward_noalloc. */
 int bitlinear_noalloc_check_status(void* stream);
 
 /* Reads and clears the status word of a workspace (synchronises
