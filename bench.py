@@ -494,7 +494,7 @@ def run_e2e(args, probs, steps):
     # step i's six calls; the host waits for step i-1's outputs to land in
     # host memory before it issues step i+1
     s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
-    xd2 = [xd, torch.empty_like(xd)]
+    xd2 = [xd, xd.clone()]                      # both hold the step's inputs before the warm-up call
     yd2 = [yd, torch.empty_like(yd)]
     yh2 = [yh, torch.empty_like(yh).pin_memory()]
     xv2 = [[b[xo[i]:xo[i + 1]].view(p.M, p.K) for i, p in enumerate(probs)] for b in xd2]
